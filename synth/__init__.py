@@ -1,0 +1,14 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the bench.
+
+Holds no arithmetic of the method itself; see :mod:`synth.workloads`.
+"""
+from .workloads import (  # noqa: F401
+    BLK,
+    CONFIGS,
+    Workload,
+    chunk_seed,
+    chunk_tokens,
+    direct_blocks,
+    prior,
+    random_bf16,
+)
