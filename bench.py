@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse KV attention hot path on B200.
+
+Workload: the 48-chunk sweep at its headline point, chunk 48 (batch 1,
+24 heads, head_dim 128, bf16; chunks of T=4, H=30, W=52 latent tokens =
+49 blocks, 32 pad rows; 2303 history blocks; top-64 per query block plus the
+49 own-chunk blocks = 113 selected blocks; geometric prior g ~ Beta(0.5, 2)
+with 30% zeros, lambda = 2, g_ref = 0.2).  The cache of the 47 earlier
+chunks is built before timing.
+
+One step = one pass of the whole path over chunk 48:
+  bsa_kv_append (K, V) -> bsa_tokens_to_blocks (Q) -> bsa_route ->
+  bsa_attn -> bsa_blocks_to_tokens (O)
+and the chunk's blocks are rewritten in place every step.
+
+Printed JSON line (rank 0):
+  value         selected attention FLOPs / step time (TFLOP/s), whole job
+  attn          bsa_attn alone: ms per call and TFLOP/s
+  roofline      bsa_attn against the measured dense bf16 peak
+  e2e           same metric with host inputs/outputs copied inside the step
+  cpu_baseline  the fp64 oracle on a bounded sample (rank 0, N = 1)
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun): every rank runs an independent problem of the same
+size (its own heads of another layer) - weak scaling, no collective on the
+data path; the time reported is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+CONFIG_KEY = 4
+CHUNK = 48
+BLK = 128
+METRIC = "bsa_attn selected-block TFLOP/s at chunk 48 (48-chunk sweep), 1 B200"
+L2_FLUSH_BYTES = 256 << 20
+KERNELS_PER_STEP = 7  # append, tokens->blocks, pool_q, pool_score, topk, attn, blocks->tokens
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--chunk", type=int, default=CHUNK)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return rank, world, local, pg
+
+
+def max_over_ranks(x: float, pg, device) -> float:
+    if pg is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg, device):
+    if pg is not None:
+        if device.type == "cuda":
+            pg.barrier(device_ids=[device.index])
+        else:
+            pg.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.samples = []
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", sel, "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [s for (t, s) in self.samples if t0 <= t <= t1]
+        if not rows:  # short region: take the samples nearest to it
+            rows = [s for (t, s) in self.samples if t0 - 0.3 <= t <= t1 + 0.3]
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            parts = [p.strip() for p in r.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+class State:
+    """Device-resident inputs and preallocated outputs of one rank's problem."""
+
+    def __init__(self, w, chunk, device, seed_rank=0):
+        import block_sparse_kv_bsa_b200 as bsa
+        self.bsa = bsa
+        self.w = w
+        T, H, W = w.grid
+        self.grid = (T, H, W)
+        nbc = w.blocks_per_chunk
+        self.n_own = nbc
+        self.n_hist = nbc * (chunk - 1)
+        self.device = device
+        self.cache = bsa.KVCache(w.B, w.Hh, w.D, self.n_hist + nbc, device=device)
+        # A different rank solves a different, equally sized problem.
+        wr = w if seed_rank == 0 else synth.Workload(**{**w.__dict__, "key": w.key + 100 * seed_rank})
+        for c in range(1, chunk):
+            t = synth.chunk_tokens(wr, c, device=device, want=("k", "v"))
+            bsa.bsa_kv_append(self.cache, t["k"], t["v"], T, H, W)
+        self.own_first = self.cache.n_blocks
+        t = synth.chunk_tokens(wr, chunk, device=device)
+        self.k_tok, self.v_tok, self.q_tok = t["k"], t["v"], t["q"]
+        g = synth.prior(wr, chunk, nbc, self.n_hist)
+        self.g = torch.from_numpy(g).to(device) if g is not None else None
+        self.q_blk = torch.empty((w.B, w.Hh, nbc * BLK, w.D), dtype=torch.bfloat16, device=device)
+        self.max_sel = bsa.route_max_sel(w.top_k[0], self.n_hist, nbc)
+        self.idx = torch.empty((w.B, w.Hh, nbc, self.max_sel), dtype=torch.int32, device=device)
+        self.cnt = torch.empty((w.B, w.Hh, nbc), dtype=torch.int32, device=device)
+        ws = bsa.bsa_route_workspace_size(w.B, w.Hh, w.D, nbc, self.n_hist)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
+        self.o_blk = torch.empty_like(self.q_blk)
+        self.lse = torch.empty((w.B, w.Hh, nbc * BLK), dtype=torch.float32, device=device)
+        self.o_tok = torch.empty_like(self.q_tok)
+        self.q_valid = None
+        self.attn_events = []
+        torch.cuda.synchronize(device)
+        self.q_valid = self.cache.block_valid[self.own_first:self.own_first + nbc].clone()
+
+    def step(self, time_attn=False):
+        bsa, w = self.bsa, self.w
+        T, H, W = self.grid
+        self.cache.n_blocks = self.own_first
+        bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W)
+        bsa.bsa_tokens_to_blocks(self.q_tok, T, H, W, out=self.q_blk)
+        bsa.bsa_route(self.q_blk, self.cache, self.n_hist, self.own_first, self.n_own,
+                      w.top_k[0], g=self.g, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale,
+                      q_valid=self.q_valid, max_sel=self.max_sel, idx=self.idx, cnt=self.cnt,
+                      workspace=self.ws)
+        if time_attn:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+        bsa.bsa_attn(self.q_blk, self.cache, self.idx, self.cnt, q_valid=self.q_valid,
+                     sm_scale=w.sm_scale, o=self.o_blk, lse=self.lse)
+        if time_attn:
+            e1.record()
+            self.attn_events.append((e0, e1))
+        bsa.bsa_blocks_to_tokens(self.o_blk, T, H, W, out=self.o_tok)
+
+    def selected_flops(self) -> float:
+        c = self.cnt.to(torch.float64).sum().item()
+        return c * 4.0 * BLK * BLK * self.w.D
+
+
+def run_ours(args, rank, world, local, pg):
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = synth.CONFIGS[CONFIG_KEY]
+    st = State(w, args.chunk, device, seed_rank=rank)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    for _ in range(max(args.warmup, 3)):
+        st.step()
+    st.bsa.raise_on_device_error(device)
+    flops = st.selected_flops()
+
+    clocks = ClockSampler(device) if rank == 0 else None
+    time.sleep(0.25)
+    barrier(pg, device)
+    torch.cuda.synchronize(device)
+    t_wall0 = time.time()
+    step_ms = []
+    st.attn_events = []
+    for _ in range(args.steps):
+        flush.zero_()  # L2 flush between steps, outside the timed events
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        st.step(time_attn=True)
+        e1.record()
+        step_ms.append((e0, e1))
+    torch.cuda.synchronize(device)
+    barrier(pg, device)
+    t_wall1 = time.time()
+    st.bsa.raise_on_device_error(device)
+    total_ms = sum(a.elapsed_time(b) for a, b in step_ms)
+    attn_ms = [a.elapsed_time(b) for a, b in st.attn_events]
+    total_ms = max_over_ranks(total_ms, pg, device)
+    attn_avg = max_over_ranks(sum(attn_ms) / len(attn_ms), pg, device)
+    clock_info = None
+    if clocks is not None:
+        time.sleep(0.3)
+        clocks.stop()
+        clock_info = clocks.summary(t_wall0, t_wall1)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(st, args, device, pg, flops)
+
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    peaks = load_peaks()
+    attn_tflops = flops / (attn_avg * 1e-3) / 1e12
+    out = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; N(0,1) Q/K/V with per-tile N(0,0.5^2) offsets on Q/K; "
+                "g ~ Beta(0.5,2) with 30% zeros)",
+        "config": {"workload": "48-chunk sweep, chunk 48: B1 Hh24 D128, chunk 4x30x52 "
+                               "(49 blocks), 2303 history blocks, top-64 + own chunk, prior",
+                   "chunk": args.chunk, "global_batch": w.B * world, "heads": w.Hh,
+                   "head_dim": w.D, "selected_blocks_per_query_block": st.max_sel,
+                   "parallelism": f"independent problem per rank x{world}",
+                   "l2": "flushed between steps (256 MB write outside the timed events); "
+                         "step inputs also exceed L2"},
+        "attn": {"ms_per_call": round(attn_avg, 4), "tflops": round(attn_tflops, 2),
+                 "selected_gflop_per_call": round(flops / 1e9, 3)},
+        "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
+                     "peak_source": f"{peaks['source']} burst dense bf16 (cuBLAS)",
+                     "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clock_info,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(st, args.cpu_seconds)
+    if pg is not None:
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_e2e(st, args, device, pg, flops):
+    """Same step with host inputs: H2D of the chunk's K, V, Q tokens and g from
+    pinned memory, the five calls, D2H of O tokens and LSE."""
+    k_h = st.k_tok.cpu().pin_memory()
+    v_h = st.v_tok.cpu().pin_memory()
+    q_h = st.q_tok.cpu().pin_memory()
+    g_h = st.g.cpu().pin_memory() if st.g is not None else None
+    o_h = torch.empty(st.o_tok.shape, dtype=st.o_tok.dtype).pin_memory()
+    l_h = torch.empty(st.lse.shape, dtype=st.lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (k_h, v_h, q_h) + ((g_h,) if g_h is not None else ()))
+    d2h = o_h.numel() * o_h.element_size() + l_h.numel() * l_h.element_size()
+    steps = max(3, min(args.steps, 50))
+
+    def one():
+        st.k_tok.copy_(k_h, non_blocking=True)
+        st.v_tok.copy_(v_h, non_blocking=True)
+        st.q_tok.copy_(q_h, non_blocking=True)
+        if g_h is not None:
+            st.g.copy_(g_h, non_blocking=True)
+        st.step()
+        o_h.copy_(st.o_tok, non_blocking=True)
+        l_h.copy_(st.lse, non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize(device)
+    barrier(pg, device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, pg, device)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    return {"value": round(flops * world / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+# ---------------------------------------------------------------------------
+# the oracle, timed on the host cores
+# ---------------------------------------------------------------------------
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample_step(inputs, n_items):
+    """The oracle's whole path for one head of chunk 48: Gilbert scatter of the
+    head's K/V/Q, pooling and fused top-K routing of its 49 query blocks, and
+    attention of the first ``n_items`` query blocks.  Returns the selected
+    attention FLOPs done."""
+    import oracle
+    T, H, W = inputs["grid"]
+    D = inputs["D"]
+    kb = oracle.tokens_to_blocks(inputs["k_tok"], T, H, W)
+    vb = oracle.tokens_to_blocks(inputs["v_tok"], T, H, W)
+    qb = oracle.tokens_to_blocks(inputs["q_tok"], T, H, W)
+    n_hist = inputs["n_hist"]
+    kc = np.concatenate([inputs["k_hist"], kb], axis=2)
+    vc = np.concatenate([inputs["v_hist"], vb], axis=2)
+    valid = inputs["valid"]
+    nb = kb.shape[2]
+    q_blk = qb.reshape(1, 1, nb * BLK, D)
+    idx, _ = oracle.route(q_blk, kc, valid, n_hist, n_hist, nb, inputs["g"], 2.0, 0.2,
+                          1.0 / math.sqrt(D), inputs["top_k"])
+    flops = 0.0
+    for j in range(n_items):
+        sel = idx[0][0][j]
+        oracle.attn_block(q_blk, kc, vc, valid, int(valid[n_hist + j]), 0, 0, j, sel,
+                          1.0 / math.sqrt(D))
+        flops += len(sel) * 4.0 * BLK * BLK * D
+    return flops
+
+
+def oracle_inputs(st, head=0):
+    h = head
+    valid = st.cache.block_valid.cpu().numpy().astype(np.int64)
+    return {
+        "grid": st.grid, "D": st.w.D, "n_hist": st.n_hist, "top_k": st.w.top_k[0],
+        "k_tok": st.k_tok[:, :, h:h + 1].cpu().double().numpy(),
+        "v_tok": st.v_tok[:, :, h:h + 1].cpu().double().numpy(),
+        "q_tok": st.q_tok[:, :, h:h + 1].cpu().double().numpy(),
+        "k_hist": st.cache.k[:, h:h + 1, :st.n_hist].cpu().double().numpy(),
+        "v_hist": st.cache.v[:, h:h + 1, :st.n_hist].cpu().double().numpy(),
+        "valid": valid, "g": None if st.g is None else st.g.cpu().numpy(),
+    }
+
+
+def cpu_baseline(st, seconds):
+    inputs = oracle_inputs(st)
+    t0 = time.perf_counter()
+    flops = oracle_sample_step(inputs, 1)
+    dt = time.perf_counter() - t0
+    n = 1
+    # Grow the sample to about `seconds` of CPU work.
+    while dt < seconds and n < st.n_own:
+        n = min(st.n_own, max(n + 1, int(n * seconds / max(dt, 1e-3))))
+        t0 = time.perf_counter()
+        flops = oracle_sample_step(inputs, n)
+        dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(),
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"fp64 numpy oracle, head 0 of chunk 48: Gilbert scatter of K/V/Q, "
+                      f"route of all 49 query blocks, attention of {n} query blocks"}
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return
+    import block_sparse_kv_bsa_b200 as bsa  # noqa: F401  (only to build the state on the GPU)
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    w = synth.CONFIGS[CONFIG_KEY]
+    st = State(w, args.chunk, device)
+    for _ in range(2):
+        st.step()
+    torch.cuda.synchronize(device)
+    inputs = oracle_inputs(st)
+    n_items = 2
+    for _ in range(max(args.warmup, 3)):
+        oracle_sample_step(inputs, 1)
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        flops = oracle_sample_step(inputs, n_items)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    sample = (f"fp64 numpy oracle per step: head 0 of chunk 48, Gilbert scatter, route of 49 "
+              f"query blocks, attention of {n_items} query blocks")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+           "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+           "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+           "config": {"workload": "48-chunk sweep, chunk 48 (bounded oracle sample per step)",
+                      "chunk": args.chunk},
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": host_cores(),
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, rank, world)
+        return
+    rank, world, local, pg = dist_setup(args.gpus)
+    run_ours(args, rank, world, local, pg)
+
+
+if __name__ == "__main__":
+    main()

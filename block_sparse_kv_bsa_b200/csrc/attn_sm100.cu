@@ -1,0 +1,466 @@
+// attn_sm100.cu - bsa_attn: indexed block-sparse attention on tcgen05.
+//
+// "Velox: Spatial Memory Makes World Models Efficient", Methodology Step 6:
+// each query block attends only to the KV blocks of its route, and because
+// a block is exactly one 128-row attention tile, a skipped block costs
+// neither its QK^T tile product nor its K/V tile load.
+//
+// One CTA computes one (batch, head, query block) work item; CTAs are
+// numbered head-major so that the query blocks of a head run together and
+// share that head's own-chunk K/V tiles through L2.  Warp roles:
+//   warp 0      TMA producer: Q once, then the selected K and V tiles
+//               (128 rows x D bf16, 128-byte swizzled boxes of 64 columns)
+//               into two-stage rings, each stage guarded by full/empty
+//               mbarriers.  Tile row = ((b*Hh + h)*max_blocks + blk)*128.
+//   warp 1      allocates tensor memory; one lane issues tcgen05.mma:
+//               S_i = Q K_i^T into one of two TMEM S buffers (128 x 128
+//               fp32) and O += P_i V_i into the TMEM O tile (128 x D fp32),
+//               committing each group to an mbarrier.
+//   warps 2-5   softmax, one query row per thread (TMEM lane = row): load
+//               S_i, mask the pad keys of a tail block, online softmax in
+//               base 2 with a stale-maximum rule (O and the running sum are
+//               rescaled only when the row maximum grows by more than 2^8, so
+//               both stay referenced to the same maximum and the final O/l is
+//               exact), write P_i (bf16) to shared memory in the operand
+//               layout, and finally normalise O and write O and LSE.
+// TMEM: S buffers at columns 0 and 128, O at column 256 (512 allocated).
+// Every wait is bounded; a wait that gives up records
+// BSA_DEV_WAIT_TIMEOUT, stops the other roles through a shared flag, lets
+// in-flight copies and MMAs finish (bounded) and frees tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace bsa {
+
+constexpr int kAttnThreads = 192;
+constexpr int kStages = 2;
+constexpr long long kWaitLimit = 1LL << 31;  // SM clocks (about a second)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;    // log2 units
+
+template <int D>
+struct AttnLayout {
+  static constexpr int kTileBytes = kBlk * D * 2;      // 128 rows x D bf16
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kP = kV + kStages * kTileBytes;
+  static constexpr int kBars = kP + kBlk * kBlk * 2;   // P is 128 x 128 bf16
+  static constexpr int kNumBars = 16;
+  static constexpr int kMisc = kBars + kNumBars * 8;
+  static constexpr int kTotal = kMisc + 64;
+  static constexpr int kAlloc = kTotal + 1024;         // room to align to 1024
+};
+
+// mbarrier slots
+enum {
+  B_Q_FULL = 0,
+  B_K_FULL = 1,   // +stage
+  B_K_EMPTY = 3,  // +stage
+  B_V_FULL = 5,   // +stage
+  B_V_EMPTY = 7,  // +stage
+  B_S_FULL = 9,   // +buffer
+  B_S_FREE = 11,  // +buffer
+  B_P_FULL = 13,
+  B_O_READY = 14,
+  B_MMA_DONE = 15,
+};
+
+struct AttnArgs {
+  const int32_t* idx;
+  const int32_t* cnt;
+  const int32_t* block_valid;
+  const int32_t* q_valid;
+  __nv_bfloat16* o;
+  float* lse;
+  int32_t* d_err;
+  int Hh, n_q_blocks, max_sel, max_blocks, n_blocks;
+  float scale_log2;
+};
+
+__device__ __forceinline__ int route_count(const AttnArgs& a, long long item) {
+  int n = a.cnt[item];
+  if (n < 0 || n > a.max_sel) {
+    report(a.d_err, BSA_DEV_BAD_COUNT);
+    n = n < 0 ? 0 : a.max_sel;
+  }
+  return n;
+}
+
+__device__ __forceinline__ int route_block(const AttnArgs& a, long long item, int i) {
+  int blk = a.idx[item * a.max_sel + i];
+  if (blk < 0 || blk >= a.n_blocks) {
+    report(a.d_err, BSA_DEV_BAD_INDEX);
+    blk = 0;
+  }
+  return blk;
+}
+
+__device__ __forceinline__ int block_rows(const AttnArgs& a, int blk) {
+  int v = a.block_valid[blk];
+  if (v < 1 || v > kBlk) {
+    report(a.d_err, BSA_DEV_BAD_VALID);
+    v = v < 1 ? 1 : kBlk;
+  }
+  return v;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads, 1)
+bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
+  using L = AttnLayout<D>;
+  constexpr int kBoxes = D / 64;
+  constexpr uint32_t kTileBytes = L::kTileBytes;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBars);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + L::kMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const long long item = blockIdx.x;  // ((b*Hh + h)*n_q_blocks + j)
+  const long long bh = item / a.n_q_blocks;
+  const int j = static_cast<int>(item % a.n_q_blocks);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kNumBars; ++i) {
+      uint32_t count = 1;
+      if (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL) count = 128;
+      mbar_init(&bars[i], count);
+    }
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(s_tmem, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const int n = route_count(a, item);
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int q_row = static_cast<int>(item * kBlk);
+      mbar_expect_tx(&bars[B_Q_FULL], kTileBytes);
+      for (int bx = 0; bx < kBoxes; ++bx)
+        tma_load_2d(sm + L::kQ + bx * (kBlk * 128), &tm_q, bx * 64, q_row, &bars[B_Q_FULL]);
+      int issued_k = 0, issued_v = 0;
+      for (int i = 0; i < n; ++i) {
+        const int st = i % kStages;
+        const int blk = route_block(a, item, i);
+        const int row = static_cast<int>((bh * a.max_blocks + blk) * kBlk);
+        if (i >= kStages &&
+            !mbar_wait_bounded(&bars[B_K_EMPTY + st], ((i / kStages) - 1) & 1, s_abort, kWaitLimit))
+          break;
+        mbar_expect_tx(&bars[B_K_FULL + st], kTileBytes);
+        for (int bx = 0; bx < kBoxes; ++bx)
+          tma_load_2d(sm + L::kK + st * kTileBytes + bx * (kBlk * 128), &tm_k, bx * 64, row,
+                      &bars[B_K_FULL + st]);
+        issued_k = i + 1;
+        if (i >= kStages &&
+            !mbar_wait_bounded(&bars[B_V_EMPTY + st], ((i / kStages) - 1) & 1, s_abort, kWaitLimit))
+          break;
+        mbar_expect_tx(&bars[B_V_FULL + st], kTileBytes);
+        for (int bx = 0; bx < kBoxes; ++bx)
+          tma_load_2d(sm + L::kV + st * kTileBytes + bx * (kBlk * 128), &tm_v, bx * 64, row,
+                      &bars[B_V_FULL + st]);
+        issued_v = i + 1;
+      }
+      if (issued_v < n) {
+        report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
+        *s_abort = 1;
+      }
+      // Drain: every copy this thread issued must land before the CTA exits.
+      mbar_wait_bounded(&bars[B_Q_FULL], 0, nullptr, kWaitLimit);
+      for (int st = 0; st < kStages; ++st) {
+        int last_k = -1, last_v = -1;
+        for (int i = st; i < issued_k; i += kStages) last_k = i;
+        for (int i = st; i < issued_v; i += kStages) last_v = i;
+        if (last_k >= 0)
+          mbar_wait_bounded(&bars[B_K_FULL + st], (last_k / kStages) & 1, nullptr, kWaitLimit);
+        if (last_v >= 0)
+          mbar_wait_bounded(&bars[B_V_FULL + st], (last_v / kStages) & 1, nullptr, kWaitLimit);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t kIdQK = idesc_bf16(128, 128, 0);
+      constexpr uint32_t kIdPV = idesc_bf16(128, D, 1);
+      const uint32_t q_addr = smem_u32(sm + L::kQ);
+      const uint32_t p_addr = smem_u32(sm + L::kP);
+      bool ok = mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit);
+      auto issue_qk = [&](int t) {
+        const int st = t % kStages;
+        const uint32_t k_addr = smem_u32(sm + L::kK + st * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * (kBlk * 128) + (kk % 4) * 32;
+          tc_mma_ss(tmem + st * 128, smem_desc(q_addr + off, 16, 1024),
+                    smem_desc(k_addr + off, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars[B_S_FULL + st]);
+        tc_commit(&bars[B_K_EMPTY + st]);
+      };
+      if (ok) ok = mbar_wait_bounded(&bars[B_K_FULL + 0], 0, s_abort, kWaitLimit);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0);
+      }
+      for (int i = 0; ok && i < n; ++i) {
+        if (i + 1 < n) {
+          const int t = i + 1, st = t % kStages;
+          ok = mbar_wait_bounded(&bars[B_K_FULL + st], (t / kStages) & 1, s_abort, kWaitLimit);
+          if (ok && t >= kStages)
+            ok = mbar_wait_bounded(&bars[B_S_FREE + st], ((t / kStages) - 1) & 1, s_abort,
+                                   kWaitLimit);
+          if (!ok) break;
+          tc_fence_after();
+          issue_qk(t);
+        }
+        const int st = i % kStages;
+        ok = mbar_wait_bounded(&bars[B_P_FULL], i & 1, s_abort, kWaitLimit);
+        if (ok) ok = mbar_wait_bounded(&bars[B_V_FULL + st], (i / kStages) & 1, s_abort, kWaitLimit);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sm + L::kV + st * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
+          const uint32_t aoff = (kk / 4) * (kBlk * 128) + (kk % 4) * 32;
+          tc_mma_ss(tmem + 256, smem_desc(p_addr + aoff, 16, 1024),
+                    smem_desc(v_addr + kk * 2048, kBlk * 128, 1024), kIdPV,
+                    (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&bars[B_V_EMPTY + st]);
+        tc_commit(&bars[B_O_READY]);
+      }
+      if (!ok) {
+        report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
+        *s_abort = 1;
+      }
+      // Drain: all MMAs issued by this thread complete before TMEM is freed.
+      tc_commit(&bars[B_MMA_DONE]);
+      mbar_wait_bounded(&bars[B_MMA_DONE], 0, nullptr, kWaitLimit);
+    }
+  } else {
+    // ---------------- softmax / epilogue (warps 2..5) ----------------
+    const int wq = warp & 3;                 // TMEM lane window of this warp
+    const int r = wq * 32 + lane;            // query row owned by this thread
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    uint8_t* p_tile = sm + L::kP;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    int valid_next = n > 0 ? block_rows(a, route_block(a, item, 0)) : kBlk;
+    for (int i = 0; i < n; ++i) {
+      const int st = i % kStages;
+      const int valid = valid_next;
+      if (i + 1 < n) valid_next = block_rows(a, route_block(a, item, i + 1));
+      ok = mbar_wait_bounded(&bars[B_S_FULL + st], (i / kStages) & 1, s_abort, kWaitLimit);
+      if (!ok) break;
+      tc_fence_after();
+      float s[kBlk];
+      tmem_ld_cols<kBlk>(tmem + lane_base + st * 128, s);
+      tc_fence_before();
+      mbar_arrive(&bars[B_S_FREE + st]);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kBlk; ++c) {
+        if (c >= valid) s[c] = -INFINITY;
+        mx = fmaxf(mx, s[c]);
+      }
+      const float mx2 = mx * a.scale_log2;
+      float m_new = m_ref;
+      if (i == 0 || mx2 > m_ref + kRescaleThreshold) m_new = mx2;
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < kBlk; ++c) {
+        s[c] = ex2_approx(fmaf(s[c], a.scale_log2, -m_new));
+        rs += s[c];
+      }
+      if (i > 0) {
+        ok = mbar_wait_bounded(&bars[B_O_READY], (i - 1) & 1, s_abort, kWaitLimit);
+        if (!ok) break;
+        tc_fence_after();
+        if (m_new != m_ref) {
+          const float alpha = ex2_approx(m_ref - m_new);
+          l *= alpha;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld_cols<32>(tmem + lane_base + 256 + c * 32, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] *= alpha;
+            tmem_st32(tmem + lane_base + 256 + c * 32, o);
+          }
+          tc_wait_st();
+        }
+      }
+      l += rs;
+      m_ref = m_new;
+      // P row r -> 128B-swizzled K-major operand tile (two 64-key boxes).
+#pragma unroll
+      for (int c8 = 0; c8 < kBlk / 8; ++c8) {
+        uint4 pk;
+        pk.x = pack_bf16x2(s[c8 * 8 + 0], s[c8 * 8 + 1]);
+        pk.y = pack_bf16x2(s[c8 * 8 + 2], s[c8 * 8 + 3]);
+        pk.z = pack_bf16x2(s[c8 * 8 + 4], s[c8 * 8 + 5]);
+        pk.w = pack_bf16x2(s[c8 * 8 + 6], s[c8 * 8 + 7]);
+        const int box = c8 / 8, cc = c8 % 8;
+        *reinterpret_cast<uint4*>(p_tile + box * (kBlk * 128) + r * 128 + ((cc ^ (r & 7)) * 16)) = pk;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars[B_P_FULL]);
+    }
+    if (!ok) {
+      report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
+      *s_abort = 1;
+    }
+    // Epilogue.
+    const int q_valid = a.q_valid != nullptr ? a.q_valid[j] : kBlk;
+    const long long grow = item * kBlk + r;
+    __nv_bfloat16* orow = a.o + grow * D;
+    bool have = ok && n > 0 && r < q_valid;
+    if (ok && n > 0) {
+      ok = mbar_wait_bounded(&bars[B_O_READY], (n - 1) & 1, s_abort, kWaitLimit);
+      if (!ok) {
+        report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
+        *s_abort = 1;
+        have = false;
+      }
+      tc_fence_after();
+    }
+    const float inv_l = have ? 1.0f / l : 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = 0.f;
+      if (ok && n > 0) tmem_ld_cols<32>(tmem + lane_base + 256 + c * 32, o);
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        uint4 pk;
+        pk.x = pack_bf16x2(have ? o[e + 0] * inv_l : 0.f, have ? o[e + 1] * inv_l : 0.f);
+        pk.y = pack_bf16x2(have ? o[e + 2] * inv_l : 0.f, have ? o[e + 3] * inv_l : 0.f);
+        pk.z = pack_bf16x2(have ? o[e + 4] * inv_l : 0.f, have ? o[e + 5] * inv_l : 0.f);
+        pk.w = pack_bf16x2(have ? o[e + 6] * inv_l : 0.f, have ? o[e + 7] * inv_l : 0.f);
+        *reinterpret_cast<uint4*>(orow + c * 32 + e) = pk;
+      }
+    }
+    a.lse[grow] = have ? (m_ref + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D map over a bf16 matrix [rows, D]: boxes of 128 rows x 64 columns, 128B swizzle.
+static bool make_map(CUtensorMap* m, const void* base, long long rows, int D) {
+  auto enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool device_is_sm100() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return false;
+  return major == 10;
+}
+
+template <int D>
+static bsa_status launch_attn(const void* q, const bsa_kv_cache* c, const AttnArgs& a,
+                              long long items, cudaStream_t s) {
+  CUtensorMap tq, tk, tv;
+  const long long qrows = items * kBlk;
+  const long long crows = static_cast<long long>(c->B) * c->Hh * c->max_blocks * kBlk;
+  if (!make_map(&tq, q, qrows, D) || !make_map(&tk, c->k, crows, D) ||
+      !make_map(&tv, c->v, crows, D))
+    return BSA_ERR_CUDA;
+  const int smem = AttnLayout<D>::kAlloc;
+  if (cudaFuncSetAttribute(bsa_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return BSA_ERR_CUDA;
+  bsa_attn_kernel<D><<<static_cast<unsigned>(items), kAttnThreads, smem, s>>>(tq, tk, tv, a);
+  return launch_status();
+}
+
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" bsa_status bsa_attn(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
+                               const int32_t* idx, const int32_t* cnt, int n_q_blocks, int max_sel,
+                               float sm_scale, void* o_blk, float* lse, int32_t* d_err,
+                               void* stream) {
+  if (q_blk == nullptr || c == nullptr || idx == nullptr || cnt == nullptr || o_blk == nullptr ||
+      lse == nullptr || c->k == nullptr || c->v == nullptr || c->block_valid == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (c->B <= 0 || c->Hh <= 0 || n_q_blocks <= 0 || max_sel <= 0 || c->max_blocks <= 0 ||
+      c->n_blocks < 0 || c->n_blocks > c->max_blocks || !(sm_scale == sm_scale))
+    return BSA_ERR_INVALID_ARG;
+  if (c->D != 64 && c->D != 128) return BSA_ERR_UNSUPPORTED;
+  if (!aligned16(q_blk) || !aligned16(o_blk) || !aligned16(c->k) || !aligned16(c->v))
+    return BSA_ERR_INVALID_ARG;
+  const long long items = static_cast<long long>(c->B) * c->Hh * n_q_blocks;
+  const long long crows = static_cast<long long>(c->B) * c->Hh * c->max_blocks * kBlk;
+  if (items * kBlk >= (1LL << 31) || crows >= (1LL << 31)) return BSA_ERR_SHAPE;
+  if (!device_is_sm100()) return BSA_ERR_UNSUPPORTED;
+  AttnArgs a{};
+  a.idx = idx;
+  a.cnt = cnt;
+  a.block_valid = c->block_valid;
+  a.q_valid = q_valid;
+  a.o = static_cast<__nv_bfloat16*>(o_blk);
+  a.lse = lse;
+  a.d_err = d_err;
+  a.Hh = c->Hh;
+  a.n_q_blocks = n_q_blocks;
+  a.max_sel = max_sel;
+  a.max_blocks = c->max_blocks;
+  a.n_blocks = c->n_blocks;
+  a.scale_log2 = sm_scale * kLog2e;
+  cudaStream_t s = as_stream(stream);
+  return c->D == 128 ? launch_attn<128>(q_blk, c, a, items, s)
+                     : launch_attn<64>(q_blk, c, a, items, s);
+}

@@ -1,0 +1,270 @@
+// reorder.cu - Gilbert-ordered block storage: bsa_kv_append,
+// bsa_tokens_to_blocks, bsa_blocks_to_tokens and bsa_gilbert_perm.
+//
+// "Velox: Spatial Memory Makes World Models Efficient", Key Contributions 3
+// and Methodology Step 6: KV is stored as 128-token blocks along a
+// global-aligned Gilbert curve, so a block is a compact patch of latent
+// cells and skipping a block skips one contiguous tile load.
+//
+// The move is a pure HBM stream: every (token, head) row of D bf16 values is
+// read once and written once.  A CTA takes 32 curve slots x 8 heads; thread
+// t moves 16-byte vectors so that a warp reads 2 KB of consecutive heads of
+// one token and writes whole 256-byte cache rows.  Each thread keeps eight
+// vectors in flight per tensor.
+#include <stdio.h>
+
+#include "common.cuh"
+#include "gilbert.cuh"
+
+namespace bsa {
+
+constexpr int kRowsPerCta = 32;
+constexpr int kHeadsPerCta = 8;
+constexpr int kReorderThreads = 256;
+constexpr int kInflight = 8;
+
+struct ReorderArgs {
+  const uint4* src0;
+  uint4* dst0;
+  const uint4* src1;  // optional second tensor (V of an append)
+  uint4* dst1;
+  const int32_t* perm;  // [N] token -> curve slot
+  int32_t* block_valid; // optional: written for the chunk's blocks
+  int32_t* d_err;
+  int N;                // tokens in the chunk
+  int nb;               // blocks of the chunk
+  int B, Hh;
+  long long blk_stride; // blocks per (b, h) in the block tensor
+  int base_block;       // first block of the chunk in the block tensor
+};
+
+// kToBlocks: raster tokens -> block slots (scatter, zero pads).
+// !kToBlocks: block slots -> raster tokens (gather).
+template <int VPR, bool kToBlocks>
+__global__ void __launch_bounds__(kReorderThreads)
+reorder_kernel(ReorderArgs a) {
+  __shared__ int s_slot[kRowsPerCta];
+  const int r0 = blockIdx.x * kRowsPerCta;
+  const int h0 = blockIdx.y * kHeadsPerCta;
+  const int b = blockIdx.z;
+  const int rows_total = kToBlocks ? a.nb * kBlk : a.N;
+
+  if (threadIdx.x < kRowsPerCta) {
+    int r = r0 + threadIdx.x;
+    int slot = -1;
+    if (r < a.N) {
+      int p = __ldg(a.perm + r);
+      if (p < 0 || p >= a.N) {
+        report(a.d_err, BSA_DEV_BAD_PERM);
+      } else {
+        slot = p;
+      }
+    } else if (kToBlocks && r < rows_total) {
+      slot = r;  // pad slot: zero-filled
+    }
+    s_slot[threadIdx.x] = slot;
+    if (kToBlocks && a.block_valid != nullptr && blockIdx.y == 0 && b == 0 && r < rows_total &&
+        (r % kBlk) == 0) {
+      int blk = r / kBlk;
+      int v = a.N - blk * kBlk;
+      a.block_valid[a.base_block + blk] = v < kBlk ? v : kBlk;
+    }
+  }
+  __syncthreads();
+
+  constexpr int kVecPerRow = VPR;
+  constexpr int kWork = kRowsPerCta * kHeadsPerCta * kVecPerRow;
+  const long long tok_row_vecs = static_cast<long long>(a.Hh) * kVecPerRow;
+
+  for (int base = threadIdx.x; base < kWork; base += kReorderThreads * kInflight) {
+    uint4 v0[kInflight], v1[kInflight];
+    long long dsto[kInflight];
+    bool live[kInflight];
+#pragma unroll
+    for (int u = 0; u < kInflight; ++u) {
+      int e = base + u * kReorderThreads;
+      live[u] = false;
+      dsto[u] = 0;
+      if (e >= kWork) continue;
+      int v = e % kVecPerRow;
+      int hh = (e / kVecPerRow) % kHeadsPerCta;
+      int rr = e / (kVecPerRow * kHeadsPerCta);
+      int h = h0 + hh;
+      int r = r0 + rr;
+      int slot = s_slot[rr];
+      if (h >= a.Hh || r >= rows_total || slot < 0) continue;
+      long long blk_row = (static_cast<long long>(b) * a.Hh + h) * a.blk_stride * kBlk +
+                          static_cast<long long>(a.base_block) * kBlk + slot;
+      long long tok_row = (static_cast<long long>(b) * a.N + r) * tok_row_vecs +
+                          static_cast<long long>(h) * kVecPerRow;
+      live[u] = true;
+      if (kToBlocks) {
+        dsto[u] = blk_row * kVecPerRow + v;
+        if (r < a.N) {
+          v0[u] = ld_nc_v4(a.src0 + tok_row + v);
+          if (a.src1 != nullptr) v1[u] = ld_nc_v4(a.src1 + tok_row + v);
+        } else {
+          v0[u] = make_uint4(0, 0, 0, 0);
+          v1[u] = make_uint4(0, 0, 0, 0);
+        }
+      } else {
+        dsto[u] = tok_row + v;
+        v0[u] = ld_nc_v4(a.src0 + blk_row * kVecPerRow + v);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kInflight; ++u) {
+      if (!live[u]) continue;
+      st_v4(a.dst0 + dsto[u], v0[u]);
+      if (kToBlocks && a.dst1 != nullptr) st_v4(a.dst1 + dsto[u], v1[u]);
+    }
+  }
+}
+
+template <bool kToBlocks>
+static bsa_status launch_reorder(const ReorderArgs& a, int D, cudaStream_t s) {
+  const int rows = kToBlocks ? a.nb * kBlk : a.N;
+  dim3 grid((rows + kRowsPerCta - 1) / kRowsPerCta, (a.Hh + kHeadsPerCta - 1) / kHeadsPerCta,
+            a.B);
+  if (D == 128) {
+    reorder_kernel<16, kToBlocks><<<grid, kReorderThreads, 0, s>>>(a);
+  } else {
+    reorder_kernel<8, kToBlocks><<<grid, kReorderThreads, 0, s>>>(a);
+  }
+  return launch_status();
+}
+
+static bsa_status check_chunk(int B, int Hh, int D, int T, int H, int W) {
+  if (B <= 0 || Hh <= 0 || T <= 0 || H <= 0 || W <= 0) return BSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return BSA_ERR_UNSUPPORTED;
+  long long n = static_cast<long long>(T) * H * W;
+  if (n > (1LL << 24)) return BSA_ERR_SHAPE;
+  if (B > 65535) return BSA_ERR_SHAPE;
+  return BSA_OK;
+}
+
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" int bsa_abi_version(void) { return BSA_ABI_VERSION; }
+
+extern "C" const char* bsa_status_string(bsa_status s) {
+  switch (s) {
+    case BSA_OK: return "BSA_OK";
+    case BSA_ERR_INVALID_ARG: return "BSA_ERR_INVALID_ARG";
+    case BSA_ERR_SHAPE: return "BSA_ERR_SHAPE";
+    case BSA_ERR_CAPACITY: return "BSA_ERR_CAPACITY";
+    case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED";
+    case BSA_ERR_CUDA: return "BSA_ERR_CUDA";
+    case BSA_ERR_DEVICE_FAULT: return "BSA_ERR_DEVICE_FAULT";
+    case BSA_ERR_TIMEOUT: return "BSA_ERR_TIMEOUT";
+  }
+  return "BSA_UNKNOWN_STATUS";
+}
+
+extern "C" bsa_status bsa_gilbert_perm(int T, int H, int W, int32_t* host_perm) {
+  if (host_perm == nullptr || T <= 0 || H <= 0 || W <= 0) return BSA_ERR_INVALID_ARG;
+  long long n = static_cast<long long>(T) * H * W;
+  if (n > (1LL << 24)) return BSA_ERR_SHAPE;
+  for (int p = 0; p < static_cast<int>(n); ++p) {
+    V3 c = gilbert_cell(T, H, W, p);
+    if (c.t < 0 || c.t >= T || c.h < 0 || c.h >= H || c.w < 0 || c.w >= W) return BSA_ERR_SHAPE;
+    host_perm[(static_cast<long long>(c.t) * H + c.h) * W + c.w] = p;
+  }
+  return BSA_OK;
+}
+
+extern "C" bsa_status bsa_kv_append(bsa_kv_cache* c, const void* k_tok, const void* v_tok, int T,
+                                    int H, int W, const int32_t* d_perm, int32_t* d_err,
+                                    void* stream) {
+  if (c == nullptr || k_tok == nullptr || v_tok == nullptr || d_perm == nullptr ||
+      c->k == nullptr || c->v == nullptr || c->block_valid == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  bsa_status st = check_chunk(c->B, c->Hh, c->D, T, H, W);
+  if (st != BSA_OK) return st;
+  if (!aligned16(k_tok) || !aligned16(v_tok) || !aligned16(c->k) || !aligned16(c->v))
+    return BSA_ERR_INVALID_ARG;
+  if (c->max_blocks <= 0 || c->n_blocks < 0 || c->n_blocks > c->max_blocks)
+    return BSA_ERR_INVALID_ARG;
+  const int n = T * H * W;
+  const int nb = (n + kBlk - 1) / kBlk;
+  if (c->n_blocks + nb > c->max_blocks) return BSA_ERR_CAPACITY;
+  ReorderArgs a{};
+  a.src0 = static_cast<const uint4*>(k_tok);
+  a.dst0 = static_cast<uint4*>(c->k);
+  a.src1 = static_cast<const uint4*>(v_tok);
+  a.dst1 = static_cast<uint4*>(c->v);
+  a.perm = d_perm;
+  a.block_valid = c->block_valid;
+  a.d_err = d_err;
+  a.N = n;
+  a.nb = nb;
+  a.B = c->B;
+  a.Hh = c->Hh;
+  a.blk_stride = c->max_blocks;
+  a.base_block = c->n_blocks;
+  st = launch_reorder<true>(a, c->D, as_stream(stream));
+  if (st == BSA_OK) c->n_blocks += nb;
+  return st;
+}
+
+extern "C" bsa_status bsa_tokens_to_blocks(const void* x_tok, void* x_blk, int B, int Hh, int D,
+                                           int T, int H, int W, const int32_t* d_perm,
+                                           int32_t* d_err, void* stream) {
+  if (x_tok == nullptr || x_blk == nullptr || d_perm == nullptr) return BSA_ERR_INVALID_ARG;
+  bsa_status st = check_chunk(B, Hh, D, T, H, W);
+  if (st != BSA_OK) return st;
+  if (!aligned16(x_tok) || !aligned16(x_blk)) return BSA_ERR_INVALID_ARG;
+  const int n = T * H * W;
+  ReorderArgs a{};
+  a.src0 = static_cast<const uint4*>(x_tok);
+  a.dst0 = static_cast<uint4*>(x_blk);
+  a.perm = d_perm;
+  a.d_err = d_err;
+  a.N = n;
+  a.nb = (n + kBlk - 1) / kBlk;
+  a.B = B;
+  a.Hh = Hh;
+  a.blk_stride = a.nb;
+  a.base_block = 0;
+  return launch_reorder<true>(a, D, as_stream(stream));
+}
+
+extern "C" bsa_status bsa_blocks_to_tokens(const void* x_blk, void* x_tok, int B, int Hh, int D,
+                                           int T, int H, int W, const int32_t* d_perm,
+                                           int32_t* d_err, void* stream) {
+  if (x_tok == nullptr || x_blk == nullptr || d_perm == nullptr) return BSA_ERR_INVALID_ARG;
+  bsa_status st = check_chunk(B, Hh, D, T, H, W);
+  if (st != BSA_OK) return st;
+  if (!aligned16(x_tok) || !aligned16(x_blk)) return BSA_ERR_INVALID_ARG;
+  const int n = T * H * W;
+  ReorderArgs a{};
+  a.src0 = static_cast<const uint4*>(x_blk);
+  a.dst0 = static_cast<uint4*>(x_tok);
+  a.perm = d_perm;
+  a.d_err = d_err;
+  a.N = n;
+  a.nb = (n + kBlk - 1) / kBlk;
+  a.B = B;
+  a.Hh = Hh;
+  a.blk_stride = a.nb;
+  a.base_block = 0;
+  return launch_reorder<false>(a, D, as_stream(stream));
+}
+
+extern "C" bsa_status bsa_check_device_error(int32_t* d_err, void* stream, int32_t* code_out) {
+  if (d_err == nullptr) return BSA_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  int32_t code = 0;
+  if (cudaMemcpyAsync(&code, d_err, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BSA_ERR_CUDA;
+  if (code != 0) {
+    if (cudaMemsetAsync(d_err, 0, sizeof(int32_t), s) != cudaSuccess) return BSA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  if (code_out != nullptr) *code_out = code;
+  if (code == 0) return BSA_OK;
+  return code == BSA_DEV_WAIT_TIMEOUT ? BSA_ERR_TIMEOUT : BSA_ERR_DEVICE_FAULT;
+}

@@ -1,0 +1,342 @@
+// route.cu - bsa_route: per-query-block KV block selection.
+//
+// "Velox: Spatial Memory Makes World Models Efficient", Methodology Step 4
+// (a block importance computed from the mean query and mean key of each
+// block, softly boosted by geometric overlap: at most a 1 + lambda boost, none
+// without overlap) and Step 5 (a bounded top-K route with reserved blocks
+// added outside the budget).  The additive form used here is
+//   s'[j, n] = sm_scale * <qmean_j, kmean_n> + lambda * min(g[j, n] / g_ref, 1).
+//
+// Three launches, all stream-ordered, no host round trip:
+//   1. pool_q      mean of each query block's valid rows -> qm (workspace)
+//   2. pool_score  stream every history K block once, pool it in registers,
+//                  and score it against all query means of its head at once;
+//                  only the scores s' go to the workspace (the K stream is the
+//                  HBM-bound part of routing)
+//   3. topk        exact top-K per row by radix select on order-preserving
+//                  score keys, ties to the lower index, emitted in ascending
+//                  index order by a block-wide ordered compaction, followed by
+//                  the own-chunk blocks.
+// All sums run in fp32 in a fixed order, so results are deterministic.
+#include "common.cuh"
+
+namespace bsa {
+
+constexpr int kPoolThreads = 256;
+constexpr int kHistPerCta = 16;
+constexpr int kTopkThreads = 256;
+
+struct RouteArgs {
+  const uint4* q;          // [B, Hh, n_own*128, D] bf16
+  const uint4* kc;         // [B, Hh, max_blocks, 128, D] bf16
+  const int32_t* block_valid;
+  const int32_t* q_valid;  // [n_own] or null
+  const float* g;          // [B, n_own, n_hist] or null
+  float* qm;               // [B, Hh, n_own, D]
+  float* s;                // [B, Hh, n_own, n_hist]
+  int32_t* idx;
+  int32_t* cnt;
+  int32_t* d_err;
+  int B, Hh, n_own, n_hist, own_first, max_blocks, top_k, max_sel;
+  float sm_scale, lam, g_ref;
+};
+
+__device__ __forceinline__ int clamp_valid(int v, int32_t* d_err) {
+  if (v < 1 || v > kBlk) {
+    report(d_err, BSA_DEV_BAD_VALID);
+    return v < 1 ? 1 : kBlk;
+  }
+  return v;
+}
+
+// Column sums of the first `valid` rows of one 128 x D bf16 block held as
+// VPR 16-byte vectors per row.  Thread t owns vector column t % VPR and rows
+// t / VPR + RG*i.  Partial sums go to `red` [RG][D]; the caller reduces.
+template <int VPR>
+__device__ __forceinline__ void block_colsum_partial(const uint4* blk, int valid, float* red) {
+  constexpr int RG = kPoolThreads / VPR;
+  constexpr int RPT = kBlk / RG;
+  const int vc = threadIdx.x % VPR;
+  const int rg = threadIdx.x / VPR;
+  uint4 x[RPT];
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    int row = rg + RG * i;
+    x[i] = row < valid ? ld_nc_v4(blk + row * VPR + vc) : make_uint4(0, 0, 0, 0);
+  }
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int i = 0; i < RPT; ++i) {
+    acc[0] += bf16lo(x[i].x); acc[1] += bf16hi(x[i].x);
+    acc[2] += bf16lo(x[i].y); acc[3] += bf16hi(x[i].y);
+    acc[4] += bf16lo(x[i].z); acc[5] += bf16hi(x[i].z);
+    acc[6] += bf16lo(x[i].w); acc[7] += bf16hi(x[i].w);
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[rg * (VPR * 8) + vc * 8 + e] = acc[e];
+}
+
+// Finish the mean: out[d] = sum_rg red[rg][d] / valid (threads d < D).
+template <int VPR>
+__device__ __forceinline__ void block_mean_finish(const float* red, int valid, float* out) {
+  constexpr int D = VPR * 8;
+  constexpr int RG = kPoolThreads / VPR;
+  if (threadIdx.x < D) {
+    float t = 0.f;
+#pragma unroll 4
+    for (int rg = 0; rg < RG; ++rg) t += red[rg * D + threadIdx.x];
+    out[threadIdx.x] = t / static_cast<float>(valid);
+  }
+}
+
+template <int VPR>
+__global__ void __launch_bounds__(kPoolThreads) pool_q_kernel(RouteArgs a) {
+  constexpr int D = VPR * 8;
+  __shared__ float red[kPoolThreads / VPR * D];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  int valid = a.q_valid != nullptr ? a.q_valid[j] : a.block_valid[a.own_first + j];
+  valid = clamp_valid(valid, a.d_err);
+  const long long bh = static_cast<long long>(b) * a.Hh + h;
+  const uint4* blk = a.q + (bh * a.n_own + j) * kBlk * VPR;
+  block_colsum_partial<VPR>(blk, valid, red);
+  __syncthreads();
+  block_mean_finish<VPR>(red, valid, a.qm + (bh * a.n_own + j) * D);
+}
+
+template <int VPR>
+__global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(RouteArgs a) {
+  constexpr int D = VPR * 8;
+  constexpr int EPL = D / 32;  // elements of a mean per lane
+  extern __shared__ float sm[];
+  float* qm = sm;                                  // [n_own][D]
+  float* red = qm + a.n_own * D;                   // [RG][D]
+  float* km = red + (kPoolThreads / VPR) * D;      // [D]
+  const int h = blockIdx.y, b = blockIdx.z;
+  const long long bh = static_cast<long long>(b) * a.Hh + h;
+  const int n_first = blockIdx.x * kHistPerCta;
+
+  for (int i = threadIdx.x; i < a.n_own * D; i += kPoolThreads) qm[i] = a.qm[bh * a.n_own * D + i];
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int nn = 0; nn < kHistPerCta; ++nn) {
+    const int n = n_first + nn;
+    if (n >= a.n_hist) break;
+    const int valid = clamp_valid(a.block_valid[n], a.d_err);
+    const uint4* blk = a.kc + (bh * a.max_blocks + n) * kBlk * VPR;
+    __syncthreads();  // previous block's km / red are consumed
+    block_colsum_partial<VPR>(blk, valid, red);
+    __syncthreads();
+    block_mean_finish<VPR>(red, valid, km);
+    __syncthreads();
+    float kr[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) kr[e] = km[lane + 32 * e];
+    for (int j = warp; j < a.n_own; j += kPoolThreads / 32) {
+      float d = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) d = fmaf(qm[j * D + lane + 32 * e], kr[e], d);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+      if (lane == 0) {
+        float sc = a.sm_scale * d;
+        if (a.g != nullptr) {
+          float gv = a.g[(static_cast<long long>(b) * a.n_own + j) * a.n_hist + n];
+          sc += a.lam * fminf(gv / a.g_ref, 1.0f);
+        }
+        a.s[(bh * a.n_own + j) * a.n_hist + n] = sc;
+      }
+    }
+  }
+}
+
+// Order-preserving map of a float onto uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t score_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Block-wide exclusive prefix of a per-thread flag (threads in index order).
+// Returns this thread's exclusive count; *total gets the block total.
+__device__ __forceinline__ int block_excl_count(bool flag, int* warp_tot, int* total) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  unsigned m = __ballot_sync(0xffffffffu, flag);
+  int in_warp = __popc(m & ((1u << lane) - 1u));
+  if (lane == 0) warp_tot[warp] = __popc(m);
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kTopkThreads / 32; ++w) {
+    int c = warp_tot[w];
+    before += (w < warp) ? c : 0;
+    all += c;
+  }
+  __syncthreads();
+  *total = all;
+  return before + in_warp;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(RouteArgs a) {
+  __shared__ int hist[256];
+  __shared__ int warp_tot[kTopkThreads / 32];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_remaining;
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const long long row = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
+  int32_t* out = a.idx + row * a.max_sel;
+  const float* sr = a.s + row * a.n_hist;
+  const int K = a.top_k < a.n_hist ? a.top_k : a.n_hist;
+
+  if (K == a.n_hist) {
+    for (int n = threadIdx.x; n < a.n_hist; n += kTopkThreads) out[n] = n;
+  } else if (K > 0) {
+    uint32_t prefix = 0, pmask = 0;
+    int remaining = K;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = threadIdx.x; i < 256; i += kTopkThreads) hist[i] = 0;
+      __syncthreads();
+      for (int n = threadIdx.x; n < a.n_hist; n += kTopkThreads) {
+        uint32_t k = score_key(sr[n]);
+        if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int above = 0;
+        int d = 255;
+        for (; d > 0; --d) {
+          if (above + hist[d] >= remaining) break;
+          above += hist[d];
+        }
+        s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
+        s_remaining = remaining - above;
+      }
+      __syncthreads();
+      prefix = s_prefix;
+      remaining = s_remaining;
+      pmask |= 255u << shift;
+      __syncthreads();
+    }
+    const uint32_t thr = prefix;   // key of the K-th largest score
+    const int need_eq = remaining; // how many keys equal to thr are taken
+    int pos = 0, eq_seen = 0;
+    for (int base = 0; base < a.n_hist; base += kTopkThreads) {
+      const int n = base + threadIdx.x;
+      uint32_t k = n < a.n_hist ? score_key(sr[n]) : 0u;
+      bool gt = n < a.n_hist && k > thr;
+      bool eq = n < a.n_hist && k == thr;
+      int eq_tot, sel_tot;
+      int eq_rank = eq_seen + block_excl_count(eq, warp_tot, &eq_tot);
+      bool sel = gt || (eq && eq_rank < need_eq);
+      int at = pos + block_excl_count(sel, warp_tot, &sel_tot);
+      if (sel) out[at] = n;
+      pos += sel_tot;
+      eq_seen += eq_tot;
+    }
+  }
+  for (int i = threadIdx.x; i < a.n_own; i += kTopkThreads) out[K + i] = a.own_first + i;
+  for (int i = K + a.n_own + threadIdx.x; i < a.max_sel; i += kTopkThreads) out[i] = -1;
+  if (threadIdx.x == 0) a.cnt[row] = K + a.n_own;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+static void route_ws_layout(int B, int Hh, int D, int n_own, int n_hist, size_t* qm_bytes,
+                            size_t* s_bytes) {
+  *qm_bytes = align256(sizeof(float) * static_cast<size_t>(B) * Hh * n_own * D);
+  *s_bytes = align256(sizeof(float) * static_cast<size_t>(B) * Hh * n_own *
+                      static_cast<size_t>(n_hist > 0 ? n_hist : 0));
+}
+
+static size_t pool_score_smem(int D, int n_own) {
+  int vpr = D / 8;
+  return sizeof(float) * (static_cast<size_t>(n_own) * D + (kPoolThreads / vpr) * D + D);
+}
+
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" bsa_status bsa_route_workspace_size(int B, int Hh, int D, int n_q_blocks, int n_hist,
+                                               size_t* bytes) {
+  if (bytes == nullptr || B <= 0 || Hh <= 0 || n_q_blocks <= 0 || n_hist < 0)
+    return BSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return BSA_ERR_UNSUPPORTED;
+  size_t a, b;
+  route_ws_layout(B, Hh, D, n_q_blocks, n_hist, &a, &b);
+  *bytes = a + b;
+  return BSA_OK;
+}
+
+extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
+                                int n_hist, int own_first, int n_own, const float* g,
+                                float lambda, float g_ref, float sm_scale, int top_k, int32_t* idx,
+                                int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
+                                int32_t* d_err, void* stream) {
+  if (q_blk == nullptr || c == nullptr || idx == nullptr || cnt == nullptr ||
+      workspace == nullptr || c->k == nullptr || c->block_valid == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (c->B <= 0 || c->Hh <= 0 || n_own <= 0 || n_hist < 0 || top_k < 0 || max_sel <= 0)
+    return BSA_ERR_INVALID_ARG;
+  if (c->D != 64 && c->D != 128) return BSA_ERR_UNSUPPORTED;
+  if (!(sm_scale == sm_scale) || (g != nullptr && !(g_ref > 0.f)) || !(lambda == lambda))
+    return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q_blk) || !aligned16(c->k) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return BSA_ERR_INVALID_ARG;
+  if (own_first < n_hist || own_first < 0 || own_first + n_own > c->n_blocks ||
+      c->n_blocks > c->max_blocks || c->B > 65535 || c->Hh > 65535 || n_own > 65535)
+    return BSA_ERR_SHAPE;
+  const int K = top_k < n_hist ? top_k : n_hist;
+  if (max_sel < K + n_own) return BSA_ERR_CAPACITY;
+  size_t qm_b, s_b;
+  route_ws_layout(c->B, c->Hh, c->D, n_own, n_hist, &qm_b, &s_b);
+  if (ws_bytes < qm_b + s_b) return BSA_ERR_CAPACITY;
+  const size_t smem = pool_score_smem(c->D, n_own);
+  if (smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
+
+  RouteArgs a{};
+  a.q = static_cast<const uint4*>(q_blk);
+  a.kc = static_cast<const uint4*>(c->k);
+  a.block_valid = c->block_valid;
+  a.q_valid = q_valid;
+  a.g = g;
+  a.qm = static_cast<float*>(workspace);
+  a.s = reinterpret_cast<float*>(static_cast<char*>(workspace) + qm_b);
+  a.idx = idx;
+  a.cnt = cnt;
+  a.d_err = d_err;
+  a.B = c->B;
+  a.Hh = c->Hh;
+  a.n_own = n_own;
+  a.n_hist = n_hist;
+  a.own_first = own_first;
+  a.max_blocks = c->max_blocks;
+  a.top_k = top_k;
+  a.max_sel = max_sel;
+  a.sm_scale = sm_scale;
+  a.lam = lambda;
+  a.g_ref = g_ref;
+
+  cudaStream_t s = as_stream(stream);
+  dim3 qgrid(n_own, c->Hh, c->B);
+  dim3 sgrid((n_hist + kHistPerCta - 1) / kHistPerCta, c->Hh, c->B);
+  if (c->D == 128) {
+    if (n_hist > 0) {
+      if (cudaFuncSetAttribute(pool_score_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    }
+    pool_q_kernel<16><<<qgrid, kPoolThreads, 0, s>>>(a);
+    if (n_hist > 0) pool_score_kernel<16><<<sgrid, kPoolThreads, smem, s>>>(a);
+  } else {
+    if (n_hist > 0) {
+      if (cudaFuncSetAttribute(pool_score_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem)) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    }
+    pool_q_kernel<8><<<qgrid, kPoolThreads, 0, s>>>(a);
+    if (n_hist > 0) pool_score_kernel<8><<<sgrid, kPoolThreads, smem, s>>>(a);
+  }
+  topk_kernel<<<qgrid, kTopkThreads, 0, s>>>(a);
+  return launch_status();
+}

@@ -1,0 +1,206 @@
+/*
+ * bsa.h - C ABI of the block-sparse KV attention library (libbsa.so).
+ *
+ * The library implements, for one NVIDIA B200 (sm_100a), the attention
+ * path described in "Velox: Spatial Memory Makes World Models Efficient":
+ *
+ *   - a KV cache stored as 128-token blocks in a global-aligned
+ *     generalised Hilbert ("Gilbert") order (Key Contributions 3;
+ *     Methodology Step 6),                                 bsa_kv_append
+ *   - a per-query-block router that scores KV blocks from the mean query and
+ *     mean key of each block, adds a geometric overlap prior and keeps a
+ *     bounded top-K route plus the query block's own chunk (Methodology
+ *     Steps 4 and 5),                                      bsa_route
+ *   - an indexed block-sparse attention that touches only the selected
+ *     128-token blocks, skipping both the QK^T tile and the KV load of every
+ *     other block (Methodology Step 6),                    bsa_attn
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *   Ownership  The caller allocates and frees all device memory and passes
+ *              raw device pointers.  The library keeps no device state and
+ *              allocates nothing on the device; workspaces are passed in.
+ *   Streams    `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *              default stream).  All device work is asynchronous on it.
+ *   Types      Q, K, V and O are bf16; g and LSE are fp32; indices int32.
+ *   Layout     Dense, row-major, no strides:
+ *                token layout  [B, T*H*W, Hh, D]   raster (t, h, w) order
+ *                block layout  [B, Hh, n_blocks, 128, D]
+ *   Errors     Every call returns a bsa_status and never aborts.  Arguments
+ *              are checked before anything is launched (nothing is launched
+ *              when a check fails).  A launch failure maps to BSA_ERR_CUDA.
+ *              Problems only the device can see (an index outside the cache,
+ *              a count above max_sel, a bounded wait that gave up) are
+ *              written as a BSA_DEV_* code into the caller's int32 word
+ *              `d_err` (first error wins; the kernel then finishes without
+ *              touching memory outside its arguments) and are read back
+ *              with bsa_check_device_error.  d_err may be NULL to skip that
+ *              reporting.
+ *   Threads    Calls are thread-safe: there is no global mutable state
+ *              apart from the immutable function table.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BSA_ABI_VERSION 1
+#define BSA_BLOCK 128 /* tokens per KV block = attention tile height */
+
+typedef enum bsa_status {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad scalar */
+  BSA_ERR_SHAPE = 2,        /* sizes inconsistent with each other */
+  BSA_ERR_CAPACITY = 3,     /* cache or output buffer too small */
+  BSA_ERR_UNSUPPORTED = 4,  /* e.g. head_dim not 64 or 128, device not sm_100 */
+  BSA_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+  BSA_ERR_DEVICE_FAULT = 6, /* d_err held a BSA_DEV_* code */
+  BSA_ERR_TIMEOUT = 7       /* d_err held BSA_DEV_WAIT_TIMEOUT */
+} bsa_status;
+
+/* Codes a kernel writes into d_err (0 = no error). */
+#define BSA_DEV_OK 0
+#define BSA_DEV_BAD_INDEX 1    /* a route index outside [0, n_blocks) */
+#define BSA_DEV_BAD_COUNT 2    /* a route count outside [0, max_sel] */
+#define BSA_DEV_BAD_VALID 3    /* a block_valid entry outside [1, 128] */
+#define BSA_DEV_BAD_PERM 4     /* a permutation entry outside the chunk */
+#define BSA_DEV_WAIT_TIMEOUT 5 /* a bounded pipeline wait gave up */
+
+/*
+ * Caller-owned view of the block KV cache.
+ *   k, v         device bf16 [B, Hh, max_blocks, 128, D]
+ *   block_valid  device int32 [max_blocks]: valid rows of each block (128, or
+ *                the tail count of a chunk's last block); pad rows are zero.
+ *   n_blocks     blocks in use, [0, max_blocks]; bsa_kv_append writes at
+ *                [n_blocks, n_blocks + nb) and then advances it (host side).
+ *   D            64 or 128.
+ */
+typedef struct bsa_kv_cache {
+  void *k;
+  void *v;
+  int32_t *block_valid;
+  int32_t B, Hh, D;
+  int32_t max_blocks;
+  int32_t n_blocks;
+} bsa_kv_cache;
+
+/* Returns BSA_ABI_VERSION of the loaded library. */
+int bsa_abi_version(void);
+
+/* Static, NUL-terminated name of a status code. */
+const char *bsa_status_string(bsa_status status);
+
+/*
+ * Gilbert order of a T x H x W latent chunk (host only, no device work).
+ * Velox, Key Contributions 3 and Methodology Step 6: neighbouring latent
+ * cells are stored contiguously, and every chunk of one shape shares one
+ * order ("global-aligned"), so block n of any chunk covers the same cells.
+ *   host_perm  host int32 [T*H*W], written: host_perm[i] is the curve
+ *              position of raster token i = (t*H + h)*W + w.  Consecutive
+ *              positions are grid neighbours (unit steps).
+ * Errors: BSA_ERR_INVALID_ARG (null pointer, non-positive extent),
+ *         BSA_ERR_SHAPE (T*H*W above 2^24).
+ */
+bsa_status bsa_gilbert_perm(int T, int H, int W, int32_t *host_perm);
+
+/*
+ * Append one chunk to the cache (Velox, Key Contributions 3): token i of the
+ * chunk goes to row perm[i] % 128 of block n_blocks + perm[i] / 128 for every
+ * head; the tail pad rows of the last block are zeroed; block_valid is set
+ * for the nb = ceil(T*H*W / 128) new blocks; cache->n_blocks += nb.
+ *   k_tok, v_tok  device bf16 [B, T*H*W, Hh, D] (cache's B, Hh, D)
+ *   d_perm        device int32 [T*H*W], the table from bsa_gilbert_perm
+ *                 (any permutation of [0, T*H*W) is accepted; entries
+ *                 outside that range raise BSA_DEV_BAD_PERM and are skipped)
+ * Errors: BSA_ERR_INVALID_ARG, BSA_ERR_CAPACITY (n_blocks + nb > max_blocks,
+ *         cache unchanged), BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA.
+ */
+bsa_status bsa_kv_append(bsa_kv_cache *cache, const void *k_tok, const void *v_tok,
+                         int T, int H, int W, const int32_t *d_perm,
+                         int32_t *d_err, void *stream);
+
+/*
+ * The same scatter for a single tensor, e.g. the query chunk before routing:
+ *   x_tok [B, T*H*W, Hh, D]  ->  x_blk [B, Hh, nb*128, D] (pad rows zeroed).
+ * The pages do not state how Q is ordered; it shares the KV order so a query
+ * block and a KV block of the same chunk cover the same cells.
+ */
+bsa_status bsa_tokens_to_blocks(const void *x_tok, void *x_blk, int B, int Hh, int D,
+                                int T, int H, int W, const int32_t *d_perm,
+                                int32_t *d_err, void *stream);
+
+/* Inverse gather, e.g. the attention output back to raster tokens:
+ *   x_blk [B, Hh, nb*128, D]  ->  x_tok [B, T*H*W, Hh, D]. */
+bsa_status bsa_blocks_to_tokens(const void *x_blk, void *x_tok, int B, int Hh, int D,
+                                int T, int H, int W, const int32_t *d_perm,
+                                int32_t *d_err, void *stream);
+
+/* Device workspace bsa_route needs, in bytes (256-byte aligned pieces). */
+bsa_status bsa_route_workspace_size(int B, int Hh, int D, int n_q_blocks, int n_hist,
+                                    size_t *bytes);
+
+/*
+ * Route every (batch, head, query block) (Velox, Methodology Steps 4-5):
+ *   qm[j] = mean of the valid rows of query block j,
+ *   km[n] = mean of the valid rows of history block n (n < n_hist),
+ *   s[j,n] = sm_scale * <qm[j], km[n]>  (+ lambda * min(g[b,j,n] / g_ref, 1)
+ *            when g is given; g is shared by all heads),
+ *   route = the top_k largest s over the history (ties to the lower block
+ *           index; every history block when top_k >= n_hist), sorted
+ *           ascending, followed by the own chunk [own_first, own_first+n_own).
+ * Arithmetic is fp32 with a fixed reduction order.
+ *   q_blk      device bf16 [B, Hh, n_own*128, D] (block order)
+ *   q_valid    device int32 [n_own] valid rows per query block, or NULL to
+ *              use cache->block_valid[own_first + j]
+ *   g          device fp32 [B, n_own, n_hist] or NULL
+ *   idx        device int32 [B, Hh, n_own, max_sel]; entries past cnt are -1
+ *   cnt        device int32 [B, Hh, n_own] = min(top_k, n_hist) + n_own
+ *   workspace  device, at least bsa_route_workspace_size bytes, 256-aligned
+ * Errors: BSA_ERR_INVALID_ARG, BSA_ERR_SHAPE (e.g. own chunk outside the
+ *         cache, history overlapping it), BSA_ERR_CAPACITY (max_sel too
+ *         small, workspace too small), BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA.
+ */
+bsa_status bsa_route(const void *q_blk, const bsa_kv_cache *cache, const int32_t *q_valid,
+                     int n_hist, int own_first, int n_own, const float *g,
+                     float lambda, float g_ref, float sm_scale, int top_k,
+                     int32_t *idx, int32_t *cnt, int max_sel,
+                     void *workspace, size_t ws_bytes, int32_t *d_err, void *stream);
+
+/*
+ * Indexed block-sparse attention (Velox, Methodology Step 6).  For query row
+ * r of block j of head (b, h), over the valid rows k of the blocks
+ * idx[b,h,j,0:cnt[b,h,j]] (order irrelevant, no causal mask):
+ *   O_r   = sum_k softmax_k(sm_scale * q_r . k_k) v_k      (bf16 out)
+ *   LSE_r = log sum_k exp(sm_scale * q_r . k_k)            (fp32, natural log)
+ * Rows r >= q_valid[j], and every row of a query block with an empty route,
+ * get O = 0 and LSE = -inf.  bf16 tensor-core products, fp32 accumulation.
+ *   q_blk   device bf16 [B, Hh, n_q_blocks*128, D]
+ *   q_valid device int32 [n_q_blocks] or NULL (all 128)
+ *   idx,cnt device int32 as produced by bsa_route
+ *   o_blk   device bf16 [B, Hh, n_q_blocks*128, D]
+ *   lse     device fp32 [B, Hh, n_q_blocks*128]
+ * Errors: BSA_ERR_INVALID_ARG, BSA_ERR_UNSUPPORTED (D not 64/128, no sm_100
+ *         device), BSA_ERR_CUDA; on the device BSA_DEV_BAD_INDEX,
+ *         BSA_DEV_BAD_COUNT, BSA_DEV_BAD_VALID, BSA_DEV_WAIT_TIMEOUT.
+ */
+bsa_status bsa_attn(const void *q_blk, const bsa_kv_cache *cache, const int32_t *q_valid,
+                    const int32_t *idx, const int32_t *cnt, int n_q_blocks, int max_sel,
+                    float sm_scale, void *o_blk, float *lse, int32_t *d_err, void *stream);
+
+/*
+ * Synchronise `stream`, read d_err, clear it, and map it to a status:
+ * BSA_OK, BSA_ERR_TIMEOUT (BSA_DEV_WAIT_TIMEOUT) or BSA_ERR_DEVICE_FAULT.
+ * The raw code is stored in *code_out when code_out is not NULL.
+ */
+bsa_status bsa_check_device_error(int32_t *d_err, void *stream, int32_t *code_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

@@ -1,0 +1,168 @@
+"""Shared helpers of the GPU parity tests: build a workload's state on the
+device through the library, and hand the same bf16 tensors to the oracle."""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+import torch
+
+import block_sparse_kv_bsa_b200 as bsa
+import synth
+
+BLK = 128
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+@dataclass
+class Step:
+    """Everything one query chunk's routing and attention needs."""
+    w: synth.Workload
+    cache: bsa.KVCache
+    q_tok: torch.Tensor
+    q_blk: torch.Tensor
+    g: Optional[torch.Tensor]
+    g_np: Optional[np.ndarray]
+    n_hist: int
+    own_first: int
+    n_own: int
+    q_valid: torch.Tensor
+    chunk: int
+    top_k: int
+
+
+def build_step(w: synth.Workload, device="cuda", chunk: Optional[int] = None,
+               top_k: Optional[int] = None, extra_blocks: int = 0) -> Step:
+    """Fill a cache with the workload's history, append the query chunk, and
+    lay out Q in block order.  ``chunk`` selects the query chunk of the
+    48-chunk sweep (1-based; default: the workload's own history length)."""
+    T, H, W = w.grid
+    nbc = w.blocks_per_chunk
+    if chunk is None:
+        chunk = w.hist_chunks + 1
+    hist_chunks = chunk - 1 if w.hist_direct == 0 else 0
+    n_hist = w.hist_direct + hist_chunks * nbc
+    cache = bsa.KVCache(w.B, w.Hh, w.D, n_hist + nbc + extra_blocks, device=device)
+    if w.hist_direct:
+        kd, vd = synth.direct_blocks(w, w.hist_direct, device=device)
+        cache.k[:, :, :w.hist_direct] = kd
+        cache.v[:, :, :w.hist_direct] = vd
+        cache.block_valid[:w.hist_direct] = BLK
+        cache.n_blocks = w.hist_direct
+    for c in range(1, hist_chunks + 1):
+        t = synth.chunk_tokens(w, c, device=device, want=("k", "v"))
+        bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+    qc = chunk if w.hist_direct == 0 else 1
+    t = synth.chunk_tokens(w, qc, device=device)
+    own_first = bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+    q_blk = bsa.bsa_tokens_to_blocks(t["q"], T, H, W)
+    g_np = synth.prior(w, qc, nbc, n_hist) if n_hist > 0 else None
+    g = torch.from_numpy(g_np).to(device) if g_np is not None else None
+    q_valid = cache.block_valid[own_first:own_first + nbc].clone()
+    return Step(w, cache, t["q"], q_blk, g, g_np, n_hist, own_first, nbc, q_valid, chunk,
+                w.top_k[0] if top_k is None else top_k)
+
+
+def route(step: Step, **kw):
+    return bsa.bsa_route(step.q_blk, step.cache, step.n_hist, step.own_first, step.n_own,
+                         step.top_k, g=step.g, lam=step.w.lam, g_ref=step.w.g_ref,
+                         sm_scale=step.w.sm_scale, q_valid=step.q_valid, **kw)
+
+
+def oracle_scores(step: Step, heads) -> np.ndarray:
+    """Oracle fused scores s' [B, len(heads), n_own, n_hist] on the same bf16 inputs."""
+    import oracle
+    q = f64(step.q_blk[:, heads])
+    kc = f64(step.cache.k[:, heads, :step.n_hist])
+    valid = step.cache.block_valid.cpu().numpy()
+    B, Hs, R, D = q.shape
+    qm = oracle.pool_blocks(q.reshape(B, Hs, step.n_own, BLK, D),
+                            [int(v) for v in valid[step.own_first:step.own_first + step.n_own]])
+    km = oracle.pool_blocks(kc, valid[:step.n_hist])
+    s = oracle.block_scores(qm, km, step.w.sm_scale)
+    return oracle.fuse_prior(s, step.g_np, step.w.lam, step.w.g_ref)
+
+
+def check_route_rows(idx: np.ndarray, cnt: np.ndarray, scores: np.ndarray, top_k: int,
+                     own_first: int, n_own: int, rel_tol: float = 1e-5) -> int:
+    """Compare GPU routes with the oracle's, row by row.
+
+    The route must equal the oracle's exactly, except that a block may be
+    swapped with another whose oracle score lies within ``rel_tol`` (relative
+    to max(|K-th score|, mean |score| of the row)) of the K-th score: fp32
+    on the GPU and fp64 in the oracle may order such near-ties differently.
+    Returns the number of rows that needed the near-tie rule.
+    """
+    import oracle
+    n_hist = scores.shape[-1]
+    K = min(top_k, n_hist)
+    ties = 0
+    B, Hs, J = cnt.shape
+    for b in range(B):
+        for h in range(Hs):
+            for j in range(J):
+                row = scores[b, h, j]
+                want = oracle.top_k_with_own(row, top_k, own_first, n_own)
+                assert int(cnt[b, h, j]) == K + n_own
+                got = idx[b, h, j, :K + n_own]
+                assert np.all(idx[b, h, j, K + n_own:] == -1)
+                assert np.array_equal(got[K:], np.arange(own_first, own_first + n_own))
+                assert np.all(np.diff(got[:K]) > 0), "route not sorted ascending"
+                if np.array_equal(got, want):
+                    continue
+                kth = np.sort(row)[::-1][K - 1]
+                tol = rel_tol * max(abs(kth), np.mean(np.abs(row)))
+                diff = set(got[:K].tolist()) ^ set(want[:K].tolist())
+                for n in diff:
+                    assert abs(row[n] - kth) <= tol, (b, h, j, n, row[n], kth, tol)
+                ties += 1
+    return ties
+
+
+def oracle_attn_items(step: Step, idx: torch.Tensor, cnt: torch.Tensor, items, sm_scale=None):
+    """Oracle O and LSE for the listed (b, h, j) items on the GPU's own route."""
+    import oracle
+    sm = step.w.sm_scale if sm_scale is None else sm_scale
+    valid = step.cache.block_valid.cpu().numpy()
+    qv = step.q_valid.cpu().numpy()
+    idx_np = idx.cpu().numpy()
+    cnt_np = cnt.cpu().numpy()
+    out = []
+    kv = {}
+    for (b, h, j) in items:
+        if (b, h) not in kv:
+            kv[(b, h)] = (f64(step.cache.k[b:b + 1, h:h + 1]), f64(step.cache.v[b:b + 1, h:h + 1]))
+        kc, vc = kv[(b, h)]
+        sel = [int(x) for x in idx_np[b, h, j, :cnt_np[b, h, j]]]
+        q = f64(step.q_blk[b:b + 1, h:h + 1, j * BLK:(j + 1) * BLK])
+        o, lse = oracle.attn_block(q, kc, vc, valid, int(qv[j]), 0, 0, 0, sel, sm)
+        out.append((o, lse))
+    return out
+
+
+def attn_errors(o_gpu: np.ndarray, lse_gpu: np.ndarray, o_ref: np.ndarray, lse_ref: np.ndarray,
+                q_valid: int):
+    """(relative L2 of O, max |O| error, max |LSE| error) over the valid rows,
+    after checking the pad rows are exactly O = 0 and LSE = -inf."""
+    assert np.all(o_gpu[q_valid:] == 0)
+    assert np.all(np.isneginf(lse_gpu[q_valid:]))
+    ov, rv = o_gpu[:q_valid], o_ref[:q_valid]
+    rel = float(np.linalg.norm(ov - rv) / max(np.linalg.norm(rv), 1e-30))
+    mabs = float(np.max(np.abs(ov - rv))) if q_valid else 0.0
+    lerr = float(np.max(np.abs(lse_gpu[:q_valid] - lse_ref[:q_valid]))) if q_valid else 0.0
+    return rel, mabs, lerr
+
+
+# Tolerances: O from bf16 inputs with fp32 accumulation against the fp64
+# oracle: relative L2 <= 1e-2 and max abs <= 2e-2.  LSE is fp32 throughout
+# apart from the bf16 inputs, and its error is dominated by fp32 rounding of
+# the running sum and by ex2.approx (relative error ~2^-22 per term):
+# |d LSE| <= 1e-3 leaves a wide margin.
+O_REL_L2 = 1e-2
+O_MAX_ABS = 2e-2
+LSE_MAX_ABS = 1e-3

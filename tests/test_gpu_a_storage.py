@@ -1,0 +1,122 @@
+"""GPU parity: Gilbert-ordered KV append and token/block reordering.
+
+Bit-exact against the oracle's scatter ("Velox: Spatial Memory Makes World
+Models Efficient", Key Contributions 3): the same bf16 values must land in
+the same cache slots, pads must be zero and block_valid must be right.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_kv_bsa_b200 as bsa
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy()
+
+
+def bf16_of(x: np.ndarray) -> np.ndarray:
+    """fp64 oracle values (exact bf16 numbers) -> their bf16 bit patterns."""
+    return torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy()
+
+
+@pytest.mark.parametrize("key", [1, 2, 5])
+def test_append_bit_exact(key):
+    w = synth.CONFIGS[key]
+    T, H, W = w.grid
+    n_chunks = 3
+    cache = bsa.KVCache(w.B, w.Hh, w.D, n_chunks * w.blocks_per_chunk + 1, device=DEV)
+    toks = []
+    for c in range(1, n_chunks + 1):
+        t = synth.chunk_tokens(w, c, device=DEV, want=("k", "v"))
+        first = bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+        assert first == (c - 1) * w.blocks_per_chunk
+        toks.append(t)
+    bsa.raise_on_device_error(DEV)
+    assert cache.n_blocks == n_chunks * w.blocks_per_chunk
+    nb = w.blocks_per_chunk
+    valid = cache.block_valid.cpu().numpy()
+    for c, t in enumerate(toks):
+        exp_k = oracle.tokens_to_blocks(t["k"].cpu().double().numpy(), T, H, W)
+        exp_v = oracle.tokens_to_blocks(t["v"].cpu().double().numpy(), T, H, W)
+        got_k = bits(cache.k[:, :, c * nb:(c + 1) * nb])
+        got_v = bits(cache.v[:, :, c * nb:(c + 1) * nb])
+        assert np.array_equal(got_k, bf16_of(exp_k))
+        assert np.array_equal(got_v, bf16_of(exp_v))
+        assert np.array_equal(valid[c * nb:(c + 1) * nb], oracle.block_valid_for(T, H, W))
+    assert valid[-1] == 0  # untouched spare block
+
+
+@pytest.mark.parametrize("key", [3, 4])
+def test_append_full_size_head_sample(key):
+    # Full-size chunk with padding (7800 -> 61 blocks, 6240 -> 49 blocks);
+    # the oracle checks a sample of heads bit for bit.
+    w = synth.CONFIGS[key]
+    T, H, W = w.grid
+    nb = w.blocks_per_chunk
+    cache = bsa.KVCache(w.B, w.Hh, w.D, 2 * nb, device=DEV)
+    t1 = synth.chunk_tokens(w, 1, device=DEV, want=("k", "v"))
+    t2 = synth.chunk_tokens(w, 2, device=DEV, want=("k", "v"))
+    bsa.bsa_kv_append(cache, t1["k"], t1["v"], T, H, W)
+    bsa.bsa_kv_append(cache, t2["k"], t2["v"], T, H, W)
+    bsa.raise_on_device_error(DEV)
+    for h in (0, w.Hh // 2, w.Hh - 1):
+        exp = oracle.tokens_to_blocks(t2["v"][:, :, h:h + 1].cpu().double().numpy(), T, H, W)
+        assert np.array_equal(bits(cache.v[:, h:h + 1, nb:2 * nb]), bf16_of(exp))
+        exp = oracle.tokens_to_blocks(t1["k"][:, :, h:h + 1].cpu().double().numpy(), T, H, W)
+        assert np.array_equal(bits(cache.k[:, h:h + 1, :nb]), bf16_of(exp))
+    pad = (nb * 128) - T * H * W
+    assert torch.all(cache.k[:, :, 2 * nb - 1, 128 - pad:] == 0)
+
+
+@pytest.mark.parametrize("grid,D", [((3, 5, 7), 64), ((1, 1, 1), 128), ((2, 8, 16), 128),
+                                    ((5, 30, 52), 64)])
+def test_tokens_blocks_round_trip(grid, D):
+    T, H, W = grid
+    x = synth.random_bf16((2, T * H * W, 3, D), seed=7, device=DEV)
+    blk = bsa.bsa_tokens_to_blocks(x, T, H, W)
+    back = bsa.bsa_blocks_to_tokens(blk, T, H, W)
+    bsa.raise_on_device_error(DEV)
+    assert torch.equal(back.view(torch.int16), x.view(torch.int16))
+    exp = oracle.tokens_to_blocks(x.cpu().double().numpy(), T, H, W)
+    assert np.array_equal(bits(blk).reshape(exp.shape), bf16_of(exp))
+
+
+def test_append_capacity_error_leaves_cache_unchanged():
+    w = synth.CONFIGS[1]
+    T, H, W = w.grid
+    cache = bsa.KVCache(w.B, w.Hh, w.D, w.blocks_per_chunk + 1, device=DEV)
+    t = synth.chunk_tokens(w, 1, device=DEV, want=("k", "v"))
+    bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+    before = cache.k.clone()
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+    assert e.value.status == 3
+    assert cache.n_blocks == w.blocks_per_chunk
+    assert torch.equal(cache.k, before)
+
+
+def test_bad_permutation_is_reported_not_faulted():
+    # A permutation entry outside the chunk is skipped and reported.
+    import ctypes
+    w = synth.CONFIGS[1]
+    T, H, W = w.grid
+    cache = bsa.KVCache(w.B, w.Hh, w.D, w.blocks_per_chunk, device=DEV)
+    t = synth.chunk_tokens(w, 1, device=DEV, want=("k", "v"))
+    perm = bsa.gilbert_perm_device(T, H, W, DEV).clone()
+    perm[5] = 10 ** 6
+    cs = cache.c_struct()
+    err = bsa.error_word(DEV)
+    st = bsa.lib().bsa_kv_append(ctypes.byref(cs), ctypes.c_void_p(t["k"].data_ptr()),
+                                 ctypes.c_void_p(t["v"].data_ptr()), T, H, W,
+                                 ctypes.c_void_p(perm.data_ptr()), ctypes.c_void_p(err.data_ptr()),
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    status, code = bsa.bsa_check_device_error(DEV)
+    assert status == 6 and code == 4
+    assert bsa.bsa_check_device_error(DEV) == (0, 0)  # cleared

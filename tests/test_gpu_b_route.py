@@ -1,0 +1,90 @@
+"""GPU parity: bsa_route against the oracle's pooled-score top-K.
+
+"Velox: Spatial Memory Makes World Models Efficient", Methodology Steps 4-5.
+Block indices must match the oracle exactly, apart from near-ties within
+1e-5 relative of the K-th score (fp32 on the GPU, fp64 in the oracle), where
+either choice is accepted.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_kv_bsa_b200 as bsa
+import synth
+from tests import _harness as hx
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _check(step, heads=None, top_k=None):
+    if top_k is not None:
+        step.top_k = top_k
+    idx, cnt = hx.route(step)
+    bsa.raise_on_device_error(DEV)
+    heads = list(range(step.w.Hh)) if heads is None else list(heads)
+    scores = hx.oracle_scores(step, heads)
+    ties = hx.check_route_rows(idx[:, heads].cpu().numpy(), cnt[:, heads].cpu().numpy(), scores,
+                               step.top_k, step.own_first, step.n_own)
+    rows = step.w.B * len(heads) * step.n_own
+    assert ties <= max(2, rows // 50), f"{ties} near-tie rows of {rows}"
+    return idx, cnt
+
+
+def test_route_config1_tiny():
+    _check(hx.build_step(synth.CONFIGS[1], DEV))
+
+
+def test_route_config2_block_offsets():
+    _check(hx.build_step(synth.CONFIGS[2], DEV))
+
+
+def test_route_config3_velox_budget_with_prior():
+    _check(hx.build_step(synth.CONFIGS[3], DEV))
+
+
+@pytest.mark.parametrize("top_k", [256, 32])
+def test_route_config5_head_sample(top_k):
+    _check(hx.build_step(synth.CONFIGS[5], DEV, top_k=top_k), heads=[0, 17, 39])
+
+
+@pytest.mark.parametrize("chunk", [1, 2, 3, 48])
+def test_route_config4_sweep_chunks(chunk):
+    # chunk 1: no history (own chunk only); chunk 2: K >= history (all);
+    # chunk 3: K < history; chunk 48: the headline size, one head checked.
+    step = hx.build_step(synth.CONFIGS[4], DEV, chunk=chunk)
+    _check(step, heads=[5] if chunk == 48 else [0, 23])
+
+
+def test_route_without_prior_equals_prior_of_zeros():
+    step = hx.build_step(synth.CONFIGS[3], DEV)
+    a, ca = hx.route(step)
+    g0 = step.g
+    step.g = torch.zeros_like(g0)
+    b, cb = hx.route(step)
+    step.g = None
+    c, cc = hx.route(step)
+    assert torch.equal(b, c) and torch.equal(cb, cc)
+    assert not torch.equal(a, c)  # the prior does change the route
+
+
+def test_route_all_equal_scores_take_lowest_indices():
+    # Q = 0 makes every model score 0, so with no prior the route is 0..K-1.
+    step = hx.build_step(synth.CONFIGS[2], DEV)
+    step.q_blk.zero_()
+    step.g = None
+    idx, cnt = hx.route(step)
+    K = step.top_k
+    exp = torch.arange(K, dtype=torch.int32, device=DEV)
+    assert torch.all(idx[..., :K] == exp)
+
+
+def test_route_rejects_bad_arguments():
+    step = hx.build_step(synth.CONFIGS[1], DEV)
+    with pytest.raises(bsa.BsaError) as e:     # max_sel too small
+        hx.route(step, max_sel=2)
+    assert e.value.status == 3
+    with pytest.raises(bsa.BsaError) as e:     # own chunk overlapping the history
+        bsa.bsa_route(step.q_blk, step.cache, step.n_hist + 1, step.own_first, step.n_own,
+                      step.top_k)
+    assert e.value.status == 2

@@ -1,0 +1,160 @@
+"""GPU parity: bsa_attn (tcgen05 / TMEM / TMA kernel) against the fp64 oracle.
+
+"Velox: Spatial Memory Makes World Models Efficient", Methodology Step 6:
+attention over exactly the keys of the selected blocks.  The oracle runs on
+the GPU's own route, so a near-tie routing swap can never show up here as an
+attention error.  Bar: O relative L2 <= 1e-2 and max abs <= 2e-2, LSE max
+abs <= 1e-3 over valid rows; pad query rows exactly O = 0, LSE = -inf.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_kv_bsa_b200 as bsa
+import synth
+from tests import _harness as hx
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _compare(step, idx, cnt, o, lse, items, sm_scale=None):
+    refs = hx.oracle_attn_items(step, idx, cnt, items, sm_scale=sm_scale)
+    o_np = o.cpu().double().numpy()
+    l_np = lse.cpu().double().numpy()
+    qv = step.q_valid.cpu().numpy()
+    worst = (0.0, 0.0, 0.0)
+    for (b, h, j), (ro, rl) in zip(items, refs):
+        rows = slice(j * 128, (j + 1) * 128)
+        rel, mabs, lerr = hx.attn_errors(o_np[b, h, rows], l_np[b, h, rows], ro, rl, int(qv[j]))
+        worst = tuple(max(x, y) for x, y in zip(worst, (rel, mabs, lerr)))
+        assert rel <= hx.O_REL_L2 and mabs <= hx.O_MAX_ABS and lerr <= hx.LSE_MAX_ABS, \
+            ((b, h, j), rel, mabs, lerr)
+    return worst
+
+
+def _all_items(step):
+    return [(b, h, j) for b in range(step.w.B) for h in range(step.w.Hh) for j in range(step.n_own)]
+
+
+def test_attn_config1_every_element():
+    step = hx.build_step(synth.CONFIGS[1], DEV)
+    idx, cnt = hx.route(step)
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    _compare(step, idx, cnt, o, lse, _all_items(step))
+
+
+def test_attn_config2_every_element():
+    step = hx.build_step(synth.CONFIGS[2], DEV)
+    idx, cnt = hx.route(step)
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    _compare(step, idx, cnt, o, lse, _all_items(step))
+
+
+def test_attn_config3_two_heads_with_tail_block():
+    step = hx.build_step(synth.CONFIGS[3], DEV)
+    idx, cnt = hx.route(step)
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    items = [(0, h, j) for h in (0, 23) for j in range(step.n_own)]
+    _compare(step, idx, cnt, o, lse, items)
+
+
+def test_attn_config4_chunk48_sample():
+    step = hx.build_step(synth.CONFIGS[4], DEV, chunk=48)
+    idx, cnt = hx.route(step)
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    items = [(0, h, j) for h in (0, 11, 23) for j in (0, 17, 48)]
+    _compare(step, idx, cnt, o, lse, items)
+
+
+@pytest.mark.parametrize("top_k", [256, 32])
+def test_attn_config5_sample(top_k):
+    step = hx.build_step(synth.CONFIGS[5], DEV, top_k=top_k)
+    idx, cnt = hx.route(step)
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    items = [(b, h, j) for b in (0, 1) for h in (0, 39) for j in (0, 31)]
+    _compare(step, idx, cnt, o, lse, items)
+
+
+def test_attn_dense_route_equals_dense_attention():
+    # Selecting every block is dense attention over the cache (config 5 shape
+    # with fewer heads): compare a full head against the oracle.
+    w = synth.CONFIGS[5]
+    step = hx.build_step(w, DEV, top_k=10 ** 6)
+    idx, cnt = hx.route(step)
+    assert torch.all(cnt == step.cache.n_blocks)
+    assert torch.equal(idx[0, 0, 0], torch.arange(step.cache.n_blocks, dtype=torch.int32, device=DEV))
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    items = [(1, 7, j) for j in range(step.n_own)]
+    _compare(step, idx, cnt, o, lse, items)
+
+
+def test_attn_index_order_invariance():
+    step = hx.build_step(synth.CONFIGS[2], DEV)
+    idx, cnt = hx.route(step)
+    o1, l1 = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    g = torch.Generator().manual_seed(3)
+    perm = torch.randperm(idx.shape[-1], generator=g).to(DEV)
+    idx2 = idx[..., perm].contiguous()
+    o2, l2 = bsa.bsa_attn(step.q_blk, step.cache, idx2, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    assert (o1.float() - o2.float()).abs().max().item() <= 1e-2
+    assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+def test_attn_empty_route_and_single_key():
+    w = synth.CONFIGS[1]
+    step = hx.build_step(w, DEV)
+    B, Hh, J = w.B, w.Hh, step.n_own
+    idx = torch.full((B, Hh, J, 1), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((B, Hh, J), dtype=torch.int32, device=DEV)
+    # (b, h, j) = (0, 1, 1) attends to one block whose only valid row is row 0.
+    step.cache.block_valid[3] = 1
+    idx[0, 1, 1, 0] = 3
+    cnt[0, 1, 1] = 1
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    assert torch.all(o[0, 0] == 0) and torch.all(torch.isneginf(lse[0, 0]))
+    assert torch.all(o[0, 1, :128] == 0)
+    v0 = step.cache.v[0, 1, 3, 0].float()
+    got = o[0, 1, 128:256].float()
+    assert torch.allclose(got, v0.expand_as(got), atol=1e-2)
+    k0 = step.cache.k[0, 1, 3, 0].double().cpu()
+    q = step.q_blk[0, 1, 128:256].double().cpu()
+    exp_lse = (q @ k0) * w.sm_scale
+    assert torch.allclose(lse[0, 1, 128:256].double().cpu(), exp_lse, atol=1e-3)
+
+
+def test_attn_zero_query_is_mean_of_values():
+    step = hx.build_step(synth.CONFIGS[2], DEV)
+    idx, cnt = hx.route(step)
+    step.q_blk.zero_()
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    sel = idx[0, 3, 5, :cnt[0, 3, 5]].long()
+    vals = step.cache.v[0, 3][sel].float().reshape(-1, step.w.D)
+    mean = vals.mean(0)
+    assert torch.allclose(o[0, 3, 5 * 128:6 * 128].float(), mean.expand(128, -1), atol=1e-2)
+    n_keys = int(step.cache.block_valid[sel].sum())
+    assert torch.allclose(lse[0, 3, 5 * 128:6 * 128],
+                          torch.full((128,), float(np.log(n_keys)), device=DEV), atol=1e-3)
+
+
+def test_attn_bad_index_reported_not_faulted():
+    step = hx.build_step(synth.CONFIGS[1], DEV)
+    idx, cnt = hx.route(step)
+    idx[0, 0, 0, 0] = 10 ** 6
+    bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    status, code = bsa.bsa_check_device_error(DEV)
+    assert status == 6 and code == 1
+    cnt[0, 0, 0] = idx.shape[-1] + 5
+    idx[0, 0, 0, 0] = 0
+    bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    status, code = bsa.bsa_check_device_error(DEV)
+    assert status == 6 and code == 2
