@@ -106,6 +106,14 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _dev(device) -> torch.device:
+    """A device with an explicit index (``cuda`` -> ``cuda:<current>``)."""
+    d = torch.device(device)
+    if d.type == "cuda" and d.index is None:
+        d = torch.device("cuda", torch.cuda.current_device())
+    return d
+
+
 def _stream(device) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
@@ -119,7 +127,7 @@ def _need(t: torch.Tensor, name: str, dtype, device=None, shape=None):
         raise ValueError(f"{name} must live on a CUDA device")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if device is not None and t.device != device:
+    if device is not None and t.device != _dev(device):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
@@ -131,7 +139,7 @@ _lock = threading.Lock()
 
 def error_word(device) -> torch.Tensor:
     """The per-device int32 word kernels report BSA_DEV_* codes into."""
-    device = torch.device(device)
+    device = _dev(device)
     with _lock:
         w = _err_words.get(device)
         if w is None:
@@ -170,7 +178,7 @@ def bsa_gilbert_perm(T: int, H: int, W: int) -> np.ndarray:
 
 def gilbert_perm_device(T: int, H: int, W: int, device) -> torch.Tensor:
     """The Gilbert table of a chunk shape on ``device``, computed once and cached."""
-    key = (int(T), int(H), int(W), torch.device(device))
+    key = (int(T), int(H), int(W), _dev(device))
     with _lock:
         t = _perm_cache.get(key)
     if t is None:
@@ -190,7 +198,7 @@ class KVCache:
 
     def __init__(self, B: int, Hh: int, D: int, max_blocks: int, device="cuda"):
         self.B, self.Hh, self.D, self.max_blocks = int(B), int(Hh), int(D), int(max_blocks)
-        self.device = torch.device(device)
+        self.device = _dev(device)
         shape = (self.B, self.Hh, self.max_blocks, BLK, self.D)
         self.k = torch.zeros(shape, dtype=torch.bfloat16, device=self.device)
         self.v = torch.zeros(shape, dtype=torch.bfloat16, device=self.device)
@@ -343,7 +351,7 @@ def bsa_attn(q_blk: torch.Tensor, cache: KVCache, idx: torch.Tensor, cnt: torch.
 
 def bsa_check_device_error(device="cuda", d_err: Optional[torch.Tensor] = None) -> Tuple[int, int]:
     """Synchronise, read and clear the device error word: (status, raw BSA_DEV_* code)."""
-    dev = torch.device(device)
+    dev = _dev(device)
     err = error_word(dev) if d_err is None else d_err
     code = ctypes.c_int32(0)
     st = _lib.bsa_check_device_error(_ptr(err), _stream(dev), ctypes.byref(code))

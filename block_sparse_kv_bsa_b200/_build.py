@@ -1,6 +1,8 @@
 """Build libbsa.so in-tree with nvcc for sm_100a (no GPU needed to compile).
 
-    python -m block_sparse_kv_bsa_b200._build [--verbose]
+    python block_sparse_kv_bsa_b200/_build.py [--verbose] [--force]
+
+(run it by path: importing the package would load the library it builds)
 
 Each ``csrc/*.cu`` file is compiled to an object in ``_build/`` and linked
 into ``block_sparse_kv_bsa_b200/libbsa.so`` with the CUDA runtime linked

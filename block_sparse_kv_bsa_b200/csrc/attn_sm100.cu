@@ -266,7 +266,8 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int st = i % kStages;
       const int valid = valid_next;
       if (i + 1 < n) valid_next = block_rows(a, route_block(a, item, i + 1));
-      ok = mbar_wait_bounded(&bars[B_S_FULL + st], (i / kStages) & 1, s_abort, kWaitLimit);
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded(&bars[B_S_FULL + st], (i / kStages) & 1, s_abort, kWaitLimit));
       if (!ok) break;
       tc_fence_after();
       float s[kBlk];
@@ -289,11 +290,16 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         rs += s[c];
       }
       if (i > 0) {
-        ok = mbar_wait_bounded(&bars[B_O_READY], (i - 1) & 1, s_abort, kWaitLimit);
+        // Every tcgen05.ld/st below is warp-collective: the branch decisions
+        // are made uniform across the warp, and a lane whose own maximum did
+        // not move scales by exactly 1.
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_O_READY], (i - 1) & 1, s_abort,
+                                                       kWaitLimit));
         if (!ok) break;
         tc_fence_after();
-        if (m_new != m_ref) {
-          const float alpha = ex2_approx(m_ref - m_new);
+        const bool grow = m_new != m_ref;
+        if (__any_sync(0xffffffffu, grow)) {
+          const float alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
           l *= alpha;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
@@ -333,7 +339,8 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __nv_bfloat16* orow = a.o + grow * D;
     bool have = ok && n > 0 && r < q_valid;
     if (ok && n > 0) {
-      ok = mbar_wait_bounded(&bars[B_O_READY], (n - 1) & 1, s_abort, kWaitLimit);
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded(&bars[B_O_READY], (n - 1) & 1, s_abort, kWaitLimit));
       if (!ok) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
         *s_abort = 1;
