@@ -44,7 +44,7 @@ DEV_CODES = {0: "BSA_DEV_OK", 1: "BSA_DEV_BAD_INDEX", 2: "BSA_DEV_BAD_COUNT",
 # Every symbol include/bsa.h declares (checked by the tests).
 EXPORTS = ("bsa_abi_version", "bsa_status_string", "bsa_gilbert_perm", "bsa_kv_append",
            "bsa_tokens_to_blocks", "bsa_blocks_to_tokens", "bsa_route_workspace_size",
-           "bsa_route", "bsa_attn", "bsa_check_device_error")
+           "bsa_route", "bsa_route_noalloc", "bsa_attn", "bsa_check_device_error")
 
 
 class BsaError(RuntimeError):
@@ -83,6 +83,8 @@ _sig = {
     "bsa_route_workspace_size": (_i, [_i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "bsa_route": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f, _i,
                        _p, _p, _i, _p, _sz, _p, _p]),
+    "bsa_route_noalloc": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f, _i,
+                               _p, _p, _i, _p, _p]),
     "bsa_attn": (_i, [_p, ctypes.POINTER(CCache), _p, _p, _p, _i, _i, _f, _p, _p, _p, _p]),
     "bsa_check_device_error": (_i, [_p, _p, ctypes.POINTER(ctypes.c_int32)]),
 }

@@ -18,6 +18,8 @@
 //                  index order by a block-wide ordered compaction, followed by
 //                  the own-chunk blocks.
 // All sums run in fp32 in a fixed order, so results are deterministic.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace bsa {
@@ -339,4 +341,59 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   }
   topk_kernel<<<qgrid, kTopkThreads, 0, s>>>(a);
   return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// bsa_route_noalloc: routing for callers that must not allocate device memory
+// ---------------------------------------------------------------------------
+// The router needs scratch for the query-block means and the fused scores.
+// bsa_route takes it from the caller; this variant keeps it in one fixed
+// array that lives in the library's own device image, so a caller never has
+// to obtain device memory for it.  The array exists once per GPU that loads
+// the library and stays resident until the process exits.
+namespace bsa {
+
+constexpr size_t kNoAllocScratchBytes = BSA_ROUTE_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxScratchDevices = 64;
+static void* g_scratch_addr[kMaxScratchDevices];
+static std::mutex g_scratch_mutex;
+
+// Device address of g_route_scratch on the current device.  Host code cannot
+// use the symbol itself (on the host it names a shadow object, not device
+// memory), so the address is looked up once per device, with that device
+// current, and cached.
+static bsa_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxScratchDevices) return BSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
+      return BSA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return BSA_OK;
+}
+
+}  // namespace bsa
+
+extern "C" bsa_status bsa_route_noalloc(const void* q_blk, const bsa_kv_cache* c,
+                                        const int32_t* q_valid, int n_hist, int own_first,
+                                        int n_own, const float* g, float lambda, float g_ref,
+                                        float sm_scale, int top_k, int32_t* idx, int32_t* cnt,
+                                        int max_sel, int32_t* d_err, void* stream) {
+  if (c == nullptr) return BSA_ERR_INVALID_ARG;
+  size_t need = 0;
+  bsa_status st = bsa_route_workspace_size(c->B, c->Hh, c->D, n_own, n_hist, &need);
+  if (st != BSA_OK) return st;
+  if (need > bsa::kNoAllocScratchBytes) return BSA_ERR_CAPACITY;
+  void* scratch = nullptr;
+  st = bsa::noalloc_scratch(&scratch);
+  if (st != BSA_OK) return st;
+  return bsa_route(q_blk, c, q_valid, n_hist, own_first, n_own, g, lambda, g_ref, sm_scale, top_k,
+                   idx, cnt, max_sel, scratch, bsa::kNoAllocScratchBytes, d_err, stream);
 }

@@ -193,6 +193,37 @@ bsa_status bsa_attn(const void *q_blk, const bsa_kv_cache *cache, const int32_t 
                     float sm_scale, void *o_blk, float *lse, int32_t *d_err, void *stream);
 
 /*
+ * bsa_route without a workspace argument, for callers that cannot allocate
+ * device memory themselves: for example code running inside another
+ * runtime's plugin or enqueue hook, where the host framework owns every
+ * device allocation and forbids new ones, or a latency-bound loop that cannot
+ * afford cudaMalloc's implicit device synchronisation.  There is no
+ * counterpart in the Velox page; it only changes where bsa_route's scratch
+ * lives.
+ *   Scratch   a fixed array of BSA_ROUTE_NOALLOC_SCRATCH_BYTES (16 MiB) in
+ *             the library's device image, present on every GPU that loads the
+ *             library until the process exits.  The call allocates nothing
+ *             (no cudaMalloc, no allocating library routine).
+ *   Set-up    the first call on a device looks up that device's address of
+ *             the array (cudaGetSymbolAddress, with the device current) and
+ *             caches it; make that first call before any stream capture.
+ *   Sharing   every call on a device uses the same array.  Nothing in it has
+ *             to start at zero (each call writes every entry it reads), but
+ *             calls that overlap on the GPU (different streams, or threads
+ *             without ordering) race on it and must be serialised by the
+ *             caller.
+ * Arguments, results and errors are those of bsa_route; in addition a
+ * problem whose workspace (bsa_route_workspace_size) exceeds the scratch size
+ * returns BSA_ERR_CAPACITY without launching anything.
+ */
+#define BSA_ROUTE_NOALLOC_SCRATCH_BYTES (16u << 20)
+bsa_status bsa_route_noalloc(const void *q_blk, const bsa_kv_cache *cache, const int32_t *q_valid,
+                             int n_hist, int own_first, int n_own, const float *g,
+                             float lambda, float g_ref, float sm_scale, int top_k,
+                             int32_t *idx, int32_t *cnt, int max_sel, int32_t *d_err,
+                             void *stream);
+
+/*
  * Synchronise `stream`, read d_err, clear it, and map it to a status:
  * BSA_OK, BSA_ERR_TIMEOUT (BSA_DEV_WAIT_TIMEOUT) or BSA_ERR_DEVICE_FAULT.
  * The raw code is stored in *code_out when code_out is not NULL.
