@@ -427,21 +427,19 @@ def oracle_inputs(st, head=0):
 
 
 def cpu_baseline(st, seconds):
-    inputs = oracle_inputs(st)
-    t0 = time.perf_counter()
-    flops = oracle_sample_step(inputs, 1)
-    dt = time.perf_counter() - t0
-    n = 1
-    # Grow the sample to about `seconds` of CPU work.
-    while dt < seconds and n < st.n_own:
-        n = min(st.n_own, max(n + 1, int(n * seconds / max(dt, 1e-3))))
+    """Oracle throughput on whole heads of chunk 48 (scatter, route of all 49
+    query blocks, attention of all 49), adding heads until about `seconds`."""
+    flops, dt, heads = 0.0, 0.0, 0
+    while dt < seconds and heads < st.w.Hh:
+        inputs = oracle_inputs(st, head=heads)
         t0 = time.perf_counter()
-        flops = oracle_sample_step(inputs, n)
-        dt = time.perf_counter() - t0
+        flops += oracle_sample_step(inputs, st.n_own)
+        dt += time.perf_counter() - t0
+        heads += 1
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(),
             "kind": "oracle", "seconds": round(dt, 2),
-            "sample": f"fp64 numpy oracle, head 0 of chunk 48: Gilbert scatter of K/V/Q, "
-                      f"route of all 49 query blocks, attention of {n} query blocks"}
+            "sample": f"fp64 numpy oracle on heads 0-{heads - 1} of chunk 48 (of 24): Gilbert "
+                      f"scatter of K/V/Q, route of all 49 query blocks, attention of all 49"}
 
 
 def run_reference(args, rank, world):

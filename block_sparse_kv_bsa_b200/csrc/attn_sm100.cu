@@ -36,7 +36,8 @@
 
 namespace bsa {
 
-constexpr int kAttnThreads = 192;
+constexpr int kSoftmaxThreads = 256;  // two warpgroups, one per 64-column half
+constexpr int kAttnThreads = 64 + kSoftmaxThreads;
 constexpr int kStages = 2;
 constexpr long long kWaitLimit = 1LL << 31;  // SM clocks (about a second)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -52,7 +53,8 @@ struct AttnLayout {
   static constexpr int kBars = kP + kBlk * kBlk * 2;   // P is 128 x 128 bf16
   static constexpr int kNumBars = 16;
   static constexpr int kMisc = kBars + kNumBars * 8;
-  static constexpr int kTotal = kMisc + 64;
+  static constexpr int kRed = kMisc + 64;  // float [3 slots][2 halves][128 rows]
+  static constexpr int kTotal = kRed + 3 * 2 * kBlk * 4;
   static constexpr int kAlloc = kTotal + 1024;         // room to align to 1024
 };
 
@@ -132,7 +134,7 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i) {
       uint32_t count = 1;
-      if (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL) count = 128;
+      if (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL) count = kSoftmaxThreads;
       mbar_init(&bars[i], count);
     }
     *s_abort = 0;
@@ -254,11 +256,21 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_wait_bounded(&bars[B_MMA_DONE], 0, nullptr, kWaitLimit);
     }
   } else {
-    // ---------------- softmax / epilogue (warps 2..5) ----------------
+    // ---------------- softmax / epilogue (warps 2..9) ----------------
+    // Two warpgroups split every row: half 0 owns S/P columns 0-63 and O
+    // columns [0, D/2), half 1 the rest.  The row maximum is exchanged through
+    // shared memory once per tile; the running sums stay per half (both halves
+    // use the same reference maximum) and are added in the epilogue.
+    const int half = (warp - 2) >> 2;        // 0 or 1
     const int wq = warp & 3;                 // TMEM lane window of this warp
     const int r = wq * 32 + lane;            // query row owned by this thread
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    uint8_t* p_tile = sm + L::kP;
+    constexpr int kHalfCols = kBlk / 2;      // S / P columns per thread
+    constexpr int kHalfD = D / 2;            // O columns per thread
+    const int c0 = half * kHalfCols;
+    const uint32_t o_col = 256 + half * kHalfD;
+    float* red = reinterpret_cast<float*>(sm + L::kRed);  // [2][2][128]
+    uint8_t* p_box = sm + L::kP + half * (kBlk * 128);
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     int valid_next = n > 0 ? block_rows(a, route_block(a, item, 0)) : kBlk;
@@ -270,29 +282,36 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                       mbar_wait_bounded(&bars[B_S_FULL + st], (i / kStages) & 1, s_abort, kWaitLimit));
       if (!ok) break;
       tc_fence_after();
-      float s[kBlk];
-      tmem_ld_cols<kBlk>(tmem + lane_base + st * 128, s);
+      float s[kHalfCols];
+      tmem_ld_cols<kHalfCols>(tmem + lane_base + st * 128 + c0, s);
       tc_fence_before();
       mbar_arrive(&bars[B_S_FREE + st]);
-      float mx = -INFINITY;
+      if (valid < kBlk) {  // tail block of a chunk: mask its pad keys
 #pragma unroll
-      for (int c = 0; c < kBlk; ++c) {
-        if (c >= valid) s[c] = -INFINITY;
-        mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < kHalfCols; ++c)
+          if (c0 + c >= valid) s[c] = -INFINITY;
       }
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < kHalfCols; ++c) mq[c & 3] = fmaxf(mq[c & 3], s[c]);
+      const float pm = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+      float* red_t = red + (i & 1) * (2 * kBlk);
+      red_t[half * kBlk + r] = pm;
+      asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+      const float mx = fmaxf(pm, red_t[(half ^ 1) * kBlk + r]);
       const float mx2 = mx * a.scale_log2;
       float m_new = m_ref;
       if (i == 0 || mx2 > m_ref + kRescaleThreshold) m_new = mx2;
-      float rs = 0.f;
+      float rq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kBlk; ++c) {
+      for (int c = 0; c < kHalfCols; ++c) {
         s[c] = ex2_approx(fmaf(s[c], a.scale_log2, -m_new));
-        rs += s[c];
+        rq[c & 3] += s[c];
       }
+      const float rs = (rq[0] + rq[1]) + (rq[2] + rq[3]);
       if (i > 0) {
-        // Every tcgen05.ld/st below is warp-collective: the branch decisions
-        // are made uniform across the warp, and a lane whose own maximum did
-        // not move scales by exactly 1.
+        // tcgen05.ld/st are warp-collective: the branch is warp-uniform and a
+        // lane whose maximum did not move scales by exactly 1.
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_O_READY], (i - 1) & 1, s_abort,
                                                        kWaitLimit));
         if (!ok) break;
@@ -302,28 +321,27 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const float alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
           l *= alpha;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < kHalfD / 32; ++c) {
             float o[32];
-            tmem_ld_cols<32>(tmem + lane_base + 256 + c * 32, o);
+            tmem_ld_cols<32>(tmem + lane_base + o_col + c * 32, o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tmem + lane_base + 256 + c * 32, o);
+            tmem_st32(tmem + lane_base + o_col + c * 32, o);
           }
           tc_wait_st();
         }
       }
       l += rs;
       m_ref = m_new;
-      // P row r -> 128B-swizzled K-major operand tile (two 64-key boxes).
+      // P row r, this half's 64 keys -> one 128B-swizzled K-major box.
 #pragma unroll
-      for (int c8 = 0; c8 < kBlk / 8; ++c8) {
+      for (int cc = 0; cc < 8; ++cc) {
         uint4 pk;
-        pk.x = pack_bf16x2(s[c8 * 8 + 0], s[c8 * 8 + 1]);
-        pk.y = pack_bf16x2(s[c8 * 8 + 2], s[c8 * 8 + 3]);
-        pk.z = pack_bf16x2(s[c8 * 8 + 4], s[c8 * 8 + 5]);
-        pk.w = pack_bf16x2(s[c8 * 8 + 6], s[c8 * 8 + 7]);
-        const int box = c8 / 8, cc = c8 % 8;
-        *reinterpret_cast<uint4*>(p_tile + box * (kBlk * 128) + r * 128 + ((cc ^ (r & 7)) * 16)) = pk;
+        pk.x = pack_bf16x2(s[cc * 8 + 0], s[cc * 8 + 1]);
+        pk.y = pack_bf16x2(s[cc * 8 + 2], s[cc * 8 + 3]);
+        pk.z = pack_bf16x2(s[cc * 8 + 4], s[cc * 8 + 5]);
+        pk.w = pack_bf16x2(s[cc * 8 + 6], s[cc * 8 + 7]);
+        *reinterpret_cast<uint4*>(p_box + r * 128 + ((cc ^ (r & 7)) * 16)) = pk;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -333,10 +351,11 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
       *s_abort = 1;
     }
-    // Epilogue.
+    // Epilogue: total row sum from both halves, then each half writes its
+    // D/2 output columns; half 0 writes the LSE.
     const int q_valid = a.q_valid != nullptr ? a.q_valid[j] : kBlk;
-    const long long grow = item * kBlk + r;
-    __nv_bfloat16* orow = a.o + grow * D;
+    const long long grow_idx = item * kBlk + r;
+    __nv_bfloat16* orow = a.o + grow_idx * D + half * kHalfD;
     bool have = ok && n > 0 && r < q_valid;
     if (ok && n > 0) {
       ok = __all_sync(0xffffffffu,
@@ -348,13 +367,19 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       tc_fence_after();
     }
-    const float inv_l = have ? 1.0f / l : 0.f;
+    // Slot 2 is never used by the per-tile exchange (slots 0 and 1), so the
+    // other half may still be reading its last tile's maximum.
+    float* red_e = red + 2 * (2 * kBlk);
+    red_e[half * kBlk + r] = l;
+    asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+    const float l_tot = red_e[r] + red_e[kBlk + r];
+    const float inv_l = have ? 1.0f / l_tot : 0.f;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < kHalfD / 32; ++c) {
       float o[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) o[e] = 0.f;
-      if (ok && n > 0) tmem_ld_cols<32>(tmem + lane_base + 256 + c * 32, o);
+      if (ok && n > 0) tmem_ld_cols<32>(tmem + lane_base + o_col + c * 32, o);
 #pragma unroll
       for (int e = 0; e < 32; e += 8) {
         uint4 pk;
@@ -365,7 +390,8 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         *reinterpret_cast<uint4*>(orow + c * 32 + e) = pk;
       }
     }
-    a.lse[grow] = have ? (m_ref + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+    if (half == 0)
+      a.lse[grow_idx] = have ? (m_ref + __log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
   }
 
   tc_fence_before();
