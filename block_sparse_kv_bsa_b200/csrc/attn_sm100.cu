@@ -7,23 +7,34 @@
 //
 // One CTA computes one (batch, head, query block) work item; CTAs are
 // numbered head-major so that the query blocks of a head run together and
-// share that head's own-chunk K/V tiles through L2.  Warp roles:
-//   warp 0      TMA producer: Q once, then the selected K and V tiles
-//               (128 rows x D bf16, 128-byte swizzled boxes of 64 columns)
-//               into two-stage rings, each stage guarded by full/empty
-//               mbarriers.  Tile row = ((b*Hh + h)*max_blocks + blk)*128.
+// share that head's own-chunk K/V tiles through L2.
+//
+// Tensor memory (512 columns x 128 lanes, lane = query row):
+//   [0,128) [128,256)  two S = Q K^T buffers (fp32)
+//   [256, 256+D)       O accumulator (fp32)
+//   [384, 384+D/2)     Q (bf16 pairs, the A operand of Q K^T)
+//   [448, 512)         P (bf16 pairs, the A operand of P V)
+// Both products take A from tensor memory and only B (a K or V tile) from
+// shared memory: with M = 128 an operand read from shared memory costs as
+// much bandwidth as the tensor core consumes, so keeping Q and P out of
+// shared memory is what leaves room for the K/V tile stream.
+//
+// Warp roles:
+//   warp 0      TMA producer: the selected K and V tiles (128 rows x D bf16,
+//               128-byte swizzled boxes of 64 columns) into three-stage K and
+//               V rings guarded by full/empty mbarriers.
+//               Tile row = ((b*Hh + h)*max_blocks + blk)*128.
 //   warp 1      allocates tensor memory; one lane issues tcgen05.mma:
-//               S_i = Q K_i^T into one of two TMEM S buffers (128 x 128
-//               fp32) and O += P_i V_i into the TMEM O tile (128 x D fp32),
-//               committing each group to an mbarrier.
-//   warps 2-5   softmax, one query row per thread (TMEM lane = row): load
-//               S_i, mask the pad keys of a tail block, online softmax in
-//               base 2 with a stale-maximum rule (O and the running sum are
-//               rescaled only when the row maximum grows by more than 2^8, so
-//               both stay referenced to the same maximum and the final O/l is
-//               exact), write P_i (bf16) to shared memory in the operand
-//               layout, and finally normalise O and write O and LSE.
-// TMEM: S buffers at columns 0 and 128, O at column 256 (512 allocated).
+//               S_i = Q K_i^T and O += P_i V_i, committing each group to an
+//               mbarrier.
+//   warps 2-9   softmax: two warpgroups split every row (half 0: S/P columns
+//               0-63 and O columns [0, D/2); half 1 the rest).  They put Q
+//               into tensor memory, then per tile load S, mask the pad keys
+//               of a tail block, exchange the row maximum through shared
+//               memory, exponentiate in base 2 with a stale-maximum rule (O
+//               and the running sums are rescaled only when the row maximum
+//               grows by more than 2^8, so O/l stays exact), store P (bf16)
+//               into tensor memory, and finally normalise O and write O, LSE.
 // Every wait is bounded; a wait that gives up records
 // BSA_DEV_WAIT_TIMEOUT, stops the other roles through a shared flag, lets
 // in-flight copies and MMAs finish (bounded) and frees tensor memory.
@@ -38,41 +49,46 @@ namespace bsa {
 
 constexpr int kSoftmaxThreads = 256;  // two warpgroups, one per 64-column half
 constexpr int kAttnThreads = 64 + kSoftmaxThreads;
-constexpr int kStages = 2;
+constexpr int kStagesK = 3;
+constexpr int kStagesV = 3;
+constexpr int kSBufs = 2;
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColO = 256;
+constexpr uint32_t kColQ = 384;
+constexpr uint32_t kColP = 448;
 constexpr long long kWaitLimit = 1LL << 31;  // SM clocks (about a second)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
-template <int D>
-struct AttnLayout {
-  static constexpr int kTileBytes = kBlk * D * 2;      // 128 rows x D bf16
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kP = kV + kStages * kTileBytes;
-  static constexpr int kBars = kP + kBlk * kBlk * 2;   // P is 128 x 128 bf16
-  static constexpr int kNumBars = 16;
-  static constexpr int kMisc = kBars + kNumBars * 8;
-  static constexpr int kRed = kMisc + 64;  // float [3 slots][2 halves][128 rows]
-  static constexpr int kTotal = kRed + 3 * 2 * kBlk * 4;
-  static constexpr int kAlloc = kTotal + 1024;         // room to align to 1024
-};
-
 // mbarrier slots
 enum {
   B_Q_FULL = 0,
-  B_K_FULL = 1,   // +stage
-  B_K_EMPTY = 3,  // +stage
-  B_V_FULL = 5,   // +stage
-  B_V_EMPTY = 7,  // +stage
-  B_S_FULL = 9,   // +buffer
-  B_S_FREE = 11,  // +buffer
-  B_P_FULL = 13,
-  B_O_READY = 14,
-  B_MMA_DONE = 15,
+  B_K_FULL = 1,                       // + stage (kStagesK)
+  B_K_EMPTY = B_K_FULL + kStagesK,    // + stage
+  B_V_FULL = B_K_EMPTY + kStagesK,    // + stage (kStagesV)
+  B_V_EMPTY = B_V_FULL + kStagesV,    // + stage
+  B_S_FULL = B_V_EMPTY + kStagesV,    // + buffer
+  B_S_FREE = B_S_FULL + kSBufs,       // + buffer
+  B_P_FULL = B_S_FREE + kSBufs,
+  B_O_READY,
+  B_MMA_DONE,
+  B_COUNT
+};
+
+template <int D>
+struct AttnLayout {
+  static constexpr int kTileBytes = kBlk * D * 2;      // 128 rows x D bf16
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kStagesK * kTileBytes;
+  static constexpr int kBars = kV + kStagesV * kTileBytes;
+  static constexpr int kMisc = kBars + B_COUNT * 8;
+  static constexpr int kRed = (kMisc + 64 + 15) & ~15;  // float [3 slots][2 halves][128 rows]
+  static constexpr int kTotal = kRed + 3 * 2 * kBlk * 4;
+  static constexpr int kAlloc = kTotal + 1024;          // room to align to 1024
 };
 
 struct AttnArgs {
+  const __nv_bfloat16* q;
   const int32_t* idx;
   const int32_t* cnt;
   const int32_t* block_valid;
@@ -111,10 +127,14 @@ __device__ __forceinline__ int block_rows(const AttnArgs& a, int blk) {
   return v;
 }
 
+__device__ __forceinline__ void named_bar_sync_softmax() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+}
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
+bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                AttnArgs a) {
   using L = AttnLayout<D>;
   constexpr int kBoxes = D / 64;
   constexpr uint32_t kTileBytes = L::kTileBytes;
@@ -132,9 +152,10 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int j = static_cast<int>(item % a.n_q_blocks);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < L::kNumBars; ++i) {
+    for (int i = 0; i < B_COUNT; ++i) {
       uint32_t count = 1;
-      if (i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL) count = kSoftmaxThreads;
+      if (i == B_Q_FULL || i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL)
+        count = kSoftmaxThreads;
       mbar_init(&bars[i], count);
     }
     *s_abort = 0;
@@ -150,33 +171,28 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      const int q_row = static_cast<int>(item * kBlk);
-      mbar_expect_tx(&bars[B_Q_FULL], kTileBytes);
-      for (int bx = 0; bx < kBoxes; ++bx)
-        tma_load_2d(sm + L::kQ + bx * (kBlk * 128), &tm_q, bx * 64, q_row, &bars[B_Q_FULL]);
       int issued_k = 0, issued_v = 0;
       for (int i = 0; i < n; ++i) {
-        const int st = i % kStages;
+        const int sk = i % kStagesK, sv = i % kStagesV;
         const int blk = route_block(a, item, i);
         const int row = static_cast<int>((bh * a.max_blocks + blk) * kBlk);
-        if (i >= kStages &&
-            !mbar_wait_bounded(&bars[B_K_EMPTY + st], ((i / kStages) - 1) & 1, s_abort, kWaitLimit))
+        if (i >= kStagesK && !mbar_wait_bounded(&bars[B_K_EMPTY + sk], ((i / kStagesK) - 1) & 1,
+                                                s_abort, kWaitLimit))
           break;
-        mbar_expect_tx(&bars[B_K_FULL + st], kTileBytes);
+        mbar_expect_tx(&bars[B_K_FULL + sk], kTileBytes);
         for (int bx = 0; bx < kBoxes; ++bx)
-          tma_load_2d(sm + L::kK + st * kTileBytes + bx * (kBlk * 128), &tm_k, bx * 64, row,
-                      &bars[B_K_FULL + st]);
+          tma_load_2d(sm + L::kK + sk * kTileBytes + bx * (kBlk * 128), &tm_k, bx * 64, row,
+                      &bars[B_K_FULL + sk]);
         issued_k = i + 1;
-        if (i >= kStages &&
-            !mbar_wait_bounded(&bars[B_V_EMPTY + st], ((i / kStages) - 1) & 1, s_abort, kWaitLimit))
+        if (i >= kStagesV && !mbar_wait_bounded(&bars[B_V_EMPTY + sv], ((i / kStagesV) - 1) & 1,
+                                                s_abort, kWaitLimit))
           break;
-        mbar_expect_tx(&bars[B_V_FULL + st], kTileBytes);
+        mbar_expect_tx(&bars[B_V_FULL + sv], kTileBytes);
         for (int bx = 0; bx < kBoxes; ++bx)
-          tma_load_2d(sm + L::kV + st * kTileBytes + bx * (kBlk * 128), &tm_v, bx * 64, row,
-                      &bars[B_V_FULL + st]);
+          tma_load_2d(sm + L::kV + sv * kTileBytes + bx * (kBlk * 128), &tm_v, bx * 64, row,
+                      &bars[B_V_FULL + sv]);
         issued_v = i + 1;
       }
       if (issued_v < n) {
@@ -184,15 +200,17 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         *s_abort = 1;
       }
       // Drain: every copy this thread issued must land before the CTA exits.
-      mbar_wait_bounded(&bars[B_Q_FULL], 0, nullptr, kWaitLimit);
-      for (int st = 0; st < kStages; ++st) {
-        int last_k = -1, last_v = -1;
-        for (int i = st; i < issued_k; i += kStages) last_k = i;
-        for (int i = st; i < issued_v; i += kStages) last_v = i;
-        if (last_k >= 0)
-          mbar_wait_bounded(&bars[B_K_FULL + st], (last_k / kStages) & 1, nullptr, kWaitLimit);
-        if (last_v >= 0)
-          mbar_wait_bounded(&bars[B_V_FULL + st], (last_v / kStages) & 1, nullptr, kWaitLimit);
+      for (int st = 0; st < kStagesK; ++st) {
+        int last = -1;
+        for (int i = st; i < issued_k; i += kStagesK) last = i;
+        if (last >= 0)
+          mbar_wait_bounded(&bars[B_K_FULL + st], (last / kStagesK) & 1, nullptr, kWaitLimit);
+      }
+      for (int st = 0; st < kStagesV; ++st) {
+        int last = -1;
+        for (int i = st; i < issued_v; i += kStagesV) last = i;
+        if (last >= 0)
+          mbar_wait_bounded(&bars[B_V_FULL + st], (last / kStagesV) & 1, nullptr, kWaitLimit);
       }
     }
   } else if (warp == 1) {
@@ -200,20 +218,18 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (lane == 0 && n > 0) {
       constexpr uint32_t kIdQK = idesc_bf16(128, 128, 0);
       constexpr uint32_t kIdPV = idesc_bf16(128, D, 1);
-      const uint32_t q_addr = smem_u32(sm + L::kQ);
-      const uint32_t p_addr = smem_u32(sm + L::kP);
       bool ok = mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit);
       auto issue_qk = [&](int t) {
-        const int st = t % kStages;
-        const uint32_t k_addr = smem_u32(sm + L::kK + st * kTileBytes);
+        const int sk = t % kStagesK, sb = t % kSBufs;
+        const uint32_t k_addr = smem_u32(sm + L::kK + sk * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kBlk * 128) + (kk % 4) * 32;
-          tc_mma_ss(tmem + st * 128, smem_desc(q_addr + off, 16, 1024),
+          tc_mma_ts(tmem + kColS + sb * 128, tmem + kColQ + kk * 8,
                     smem_desc(k_addr + off, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bars[B_S_FULL + st]);
-        tc_commit(&bars[B_K_EMPTY + st]);
+        tc_commit(&bars[B_S_FULL + sb]);
+        tc_commit(&bars[B_K_EMPTY + sk]);
       };
       if (ok) ok = mbar_wait_bounded(&bars[B_K_FULL + 0], 0, s_abort, kWaitLimit);
       if (ok) {
@@ -222,29 +238,29 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       for (int i = 0; ok && i < n; ++i) {
         if (i + 1 < n) {
-          const int t = i + 1, st = t % kStages;
-          ok = mbar_wait_bounded(&bars[B_K_FULL + st], (t / kStages) & 1, s_abort, kWaitLimit);
-          if (ok && t >= kStages)
-            ok = mbar_wait_bounded(&bars[B_S_FREE + st], ((t / kStages) - 1) & 1, s_abort,
+          const int t = i + 1;
+          ok = mbar_wait_bounded(&bars[B_K_FULL + t % kStagesK], (t / kStagesK) & 1, s_abort,
+                                 kWaitLimit);
+          if (ok && t >= kSBufs)
+            ok = mbar_wait_bounded(&bars[B_S_FREE + t % kSBufs], ((t / kSBufs) - 1) & 1, s_abort,
                                    kWaitLimit);
           if (!ok) break;
           tc_fence_after();
           issue_qk(t);
         }
-        const int st = i % kStages;
+        const int sv = i % kStagesV;
         ok = mbar_wait_bounded(&bars[B_P_FULL], i & 1, s_abort, kWaitLimit);
-        if (ok) ok = mbar_wait_bounded(&bars[B_V_FULL + st], (i / kStages) & 1, s_abort, kWaitLimit);
+        if (ok) ok = mbar_wait_bounded(&bars[B_V_FULL + sv], (i / kStagesV) & 1, s_abort, kWaitLimit);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm + L::kV + st * kTileBytes);
+        const uint32_t v_addr = smem_u32(sm + L::kV + sv * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
-          const uint32_t aoff = (kk / 4) * (kBlk * 128) + (kk % 4) * 32;
-          tc_mma_ss(tmem + 256, smem_desc(p_addr + aoff, 16, 1024),
+          tc_mma_ts(tmem + kColO, tmem + kColP + kk * 8,
                     smem_desc(v_addr + kk * 2048, kBlk * 128, 1024), kIdPV,
                     (i > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&bars[B_V_EMPTY + st]);
+        tc_commit(&bars[B_V_EMPTY + sv]);
         tc_commit(&bars[B_O_READY]);
       }
       if (!ok) {
@@ -268,24 +284,44 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     constexpr int kHalfCols = kBlk / 2;      // S / P columns per thread
     constexpr int kHalfD = D / 2;            // O columns per thread
     const int c0 = half * kHalfCols;
-    const uint32_t o_col = 256 + half * kHalfD;
-    float* red = reinterpret_cast<float*>(sm + L::kRed);  // [2][2][128]
-    uint8_t* p_box = sm + L::kP + half * (kBlk * 128);
+    const uint32_t o_col = kColO + half * kHalfD;
+    float* red = reinterpret_cast<float*>(sm + L::kRed);  // [3][2][128]
+
+    // Q row r -> tensor memory as bf16 pairs (the A operand of Q K^T).  With
+    // D = 128 each half stores its 64 elements; with D = 64 half 0 stores the
+    // whole row.
+    if (n > 0) {
+      const uint4* qrow = reinterpret_cast<const uint4*>(a.q + (item * kBlk + r) * D);
+      if (D == 128 || half == 0) {
+        const int e0 = (D == 128) ? half * 64 : 0;   // first element stored
+        uint32_t qw[32];
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          uint4 x = ld_nc_v4(qrow + e0 / 8 + v);
+          qw[4 * v + 0] = x.x; qw[4 * v + 1] = x.y; qw[4 * v + 2] = x.z; qw[4 * v + 3] = x.w;
+        }
+        tmem_st32u(tmem + lane_base + kColQ + e0 / 2, qw);
+        tc_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[B_Q_FULL]);
+    }
+
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     int valid_next = n > 0 ? block_rows(a, route_block(a, item, 0)) : kBlk;
     for (int i = 0; i < n; ++i) {
-      const int st = i % kStages;
+      const int sb = i % kSBufs;
       const int valid = valid_next;
       if (i + 1 < n) valid_next = block_rows(a, route_block(a, item, i + 1));
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait_bounded(&bars[B_S_FULL + st], (i / kStages) & 1, s_abort, kWaitLimit));
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_S_FULL + sb], (i / kSBufs) & 1,
+                                                     s_abort, kWaitLimit));
       if (!ok) break;
       tc_fence_after();
       float s[kHalfCols];
-      tmem_ld_cols<kHalfCols>(tmem + lane_base + st * 128 + c0, s);
+      tmem_ld_cols<kHalfCols>(tmem + lane_base + kColS + sb * 128 + c0, s);
       tc_fence_before();
-      mbar_arrive(&bars[B_S_FREE + st]);
+      mbar_arrive(&bars[B_S_FREE + sb]);
       if (valid < kBlk) {  // tail block of a chunk: mask its pad keys
 #pragma unroll
         for (int c = 0; c < kHalfCols; ++c)
@@ -297,7 +333,7 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float pm = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
       float* red_t = red + (i & 1) * (2 * kBlk);
       red_t[half * kBlk + r] = pm;
-      asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+      named_bar_sync_softmax();
       const float mx = fmaxf(pm, red_t[(half ^ 1) * kBlk + r]);
       const float mx2 = mx * a.scale_log2;
       float m_new = m_ref;
@@ -309,7 +345,12 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         rq[c & 3] += s[c];
       }
       const float rs = (rq[0] + rq[1]) + (rq[2] + rq[3]);
+      uint32_t pk[kHalfCols / 2];
+#pragma unroll
+      for (int c = 0; c < kHalfCols / 2; ++c) pk[c] = pack_bf16x2(s[2 * c], s[2 * c + 1]);
       if (i > 0) {
+        // P V of the previous tile must be done: it reads the P columns this
+        // tile overwrites and accumulates into the O that may be rescaled.
         // tcgen05.ld/st are warp-collective: the branch is warp-uniform and a
         // lane whose maximum did not move scales by exactly 1.
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_O_READY], (i - 1) & 1, s_abort,
@@ -328,22 +369,13 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
             tmem_st32(tmem + lane_base + o_col + c * 32, o);
           }
-          tc_wait_st();
         }
       }
       l += rs;
       m_ref = m_new;
-      // P row r, this half's 64 keys -> one 128B-swizzled K-major box.
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        uint4 pk;
-        pk.x = pack_bf16x2(s[cc * 8 + 0], s[cc * 8 + 1]);
-        pk.y = pack_bf16x2(s[cc * 8 + 2], s[cc * 8 + 3]);
-        pk.z = pack_bf16x2(s[cc * 8 + 4], s[cc * 8 + 5]);
-        pk.w = pack_bf16x2(s[cc * 8 + 6], s[cc * 8 + 7]);
-        *reinterpret_cast<uint4*>(p_box + r * 128 + ((cc ^ (r & 7)) * 16)) = pk;
-      }
-      fence_proxy_async_smem();
+      // P row r, this half's 64 keys -> 32 TMEM columns of bf16 pairs.
+      tmem_st32u(tmem + lane_base + kColP + half * (kHalfCols / 2), pk);
+      tc_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[B_P_FULL]);
     }
@@ -371,7 +403,7 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // other half may still be reading its last tile's maximum.
     float* red_e = red + 2 * (2 * kBlk);
     red_e[half * kBlk + r] = l;
-    asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+    named_bar_sync_softmax();
     const float l_tot = red_e[r] + red_e[kBlk + r];
     const float inv_l = have ? 1.0f / l_tot : 0.f;
 #pragma unroll
@@ -382,12 +414,12 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (ok && n > 0) tmem_ld_cols<32>(tmem + lane_base + o_col + c * 32, o);
 #pragma unroll
       for (int e = 0; e < 32; e += 8) {
-        uint4 pk;
-        pk.x = pack_bf16x2(have ? o[e + 0] * inv_l : 0.f, have ? o[e + 1] * inv_l : 0.f);
-        pk.y = pack_bf16x2(have ? o[e + 2] * inv_l : 0.f, have ? o[e + 3] * inv_l : 0.f);
-        pk.z = pack_bf16x2(have ? o[e + 4] * inv_l : 0.f, have ? o[e + 5] * inv_l : 0.f);
-        pk.w = pack_bf16x2(have ? o[e + 6] * inv_l : 0.f, have ? o[e + 7] * inv_l : 0.f);
-        *reinterpret_cast<uint4*>(orow + c * 32 + e) = pk;
+        uint4 v;
+        v.x = pack_bf16x2(have ? o[e + 0] * inv_l : 0.f, have ? o[e + 1] * inv_l : 0.f);
+        v.y = pack_bf16x2(have ? o[e + 2] * inv_l : 0.f, have ? o[e + 3] * inv_l : 0.f);
+        v.z = pack_bf16x2(have ? o[e + 4] * inv_l : 0.f, have ? o[e + 5] * inv_l : 0.f);
+        v.w = pack_bf16x2(have ? o[e + 6] * inv_l : 0.f, have ? o[e + 7] * inv_l : 0.f);
+        *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
       }
     }
     if (half == 0)
@@ -444,17 +476,14 @@ static bool device_is_sm100() {
 template <int D>
 static bsa_status launch_attn(const void* q, const bsa_kv_cache* c, const AttnArgs& a,
                               long long items, cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
-  const long long qrows = items * kBlk;
+  CUtensorMap tk, tv;
   const long long crows = static_cast<long long>(c->B) * c->Hh * c->max_blocks * kBlk;
-  if (!make_map(&tq, q, qrows, D) || !make_map(&tk, c->k, crows, D) ||
-      !make_map(&tv, c->v, crows, D))
-    return BSA_ERR_CUDA;
+  if (!make_map(&tk, c->k, crows, D) || !make_map(&tv, c->v, crows, D)) return BSA_ERR_CUDA;
   const int smem = AttnLayout<D>::kAlloc;
   if (cudaFuncSetAttribute(bsa_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return BSA_ERR_CUDA;
-  bsa_attn_kernel<D><<<static_cast<unsigned>(items), kAttnThreads, smem, s>>>(tq, tk, tv, a);
+  bsa_attn_kernel<D><<<static_cast<unsigned>(items), kAttnThreads, smem, s>>>(tk, tv, a);
   return launch_status();
 }
 
@@ -480,6 +509,7 @@ extern "C" bsa_status bsa_attn(const void* q_blk, const bsa_kv_cache* c, const i
   if (items * kBlk >= (1LL << 31) || crows >= (1LL << 31)) return BSA_ERR_SHAPE;
   if (!device_is_sm100()) return BSA_ERR_UNSUPPORTED;
   AttnArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q_blk);
   a.idx = idx;
   a.cnt = cnt;
   a.block_valid = c->block_valid;
