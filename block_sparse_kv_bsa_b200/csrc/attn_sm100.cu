@@ -309,11 +309,24 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    int valid_next = n > 0 ? block_rows(a, route_block(a, item, 0)) : kBlk;
+    // Route lookahead: the block index two tiles ahead and the valid-row
+    // count one tile ahead are loaded early and first used a tile later, so
+    // these dependent global loads never stall the softmax.  Indices are
+    // validated (and reported) by the producer; here they are only clamped.
+    const int32_t* route = a.idx + item * a.max_sel;
+    auto clamp_blk = [&](int b_) { return static_cast<unsigned>(b_) < static_cast<unsigned>(a.n_blocks) ? b_ : 0; };
+    int blk_ahead = n > 1 ? route[1] : 0;
+    int valid_raw = n > 0 ? a.block_valid[clamp_blk(route[0])] : kBlk;
     for (int i = 0; i < n; ++i) {
       const int sb = i % kSBufs;
-      const int valid = valid_next;
-      if (i + 1 < n) valid_next = block_rows(a, route_block(a, item, i + 1));
+      int valid = valid_raw;
+      if (valid < 1 || valid > kBlk) {
+        report(a.d_err, BSA_DEV_BAD_VALID);
+        valid = valid < 1 ? 1 : kBlk;
+      }
+      const int blk_ahead2 = (i + 2 < n) ? route[i + 2] : 0;
+      valid_raw = (i + 1 < n) ? a.block_valid[clamp_blk(blk_ahead)] : kBlk;
+      blk_ahead = blk_ahead2;
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_S_FULL + sb], (i / kSBufs) & 1,
                                                      s_abort, kWaitLimit));
       if (!ok) break;
