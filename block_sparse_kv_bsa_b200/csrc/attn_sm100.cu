@@ -20,13 +20,17 @@
 // shared memory is what leaves room for the K/V tile stream.
 //
 // Warp roles:
-//   warp 0      TMA producer: the selected K and V tiles (128 rows x D bf16,
-//               128-byte swizzled boxes of 64 columns) into three-stage K and
-//               V rings guarded by full/empty mbarriers.
-//               Tile row = ((b*Hh + h)*max_blocks + blk)*128.
+//   warp 0      TMA producer: the K and V tiles of each selected block
+//               (128 rows x D bf16, 128-byte swizzled boxes of 64 columns)
+//               into a three-stage ring; one full and one empty mbarrier per
+//               stage cover both tiles.  Tile row = ((b*Hh + h)*max_blocks +
+//               blk)*128.
 //   warp 1      allocates tensor memory; one lane issues tcgen05.mma:
 //               S_i = Q K_i^T and O += P_i V_i, committing each group to an
-//               mbarrier.
+//               mbarrier.  It waits only twice per tile (next stage loaded;
+//               this tile's P stored): a wait in the issuing thread leaves the
+//               tensor pipe without queued work, and measured ~170 SM cycles of
+//               lost tensor time per wait.
 //   warps 2-9   softmax: two warpgroups split every row (half 0: S/P columns
 //               0-63 and O columns [0, D/2); half 1 the rest).  They put Q
 //               into tensor memory, then per tile load S, mask the pad keys
@@ -49,8 +53,7 @@ namespace bsa {
 
 constexpr int kSoftmaxThreads = 256;  // two warpgroups, one per 64-column half
 constexpr int kAttnThreads = 64 + kSoftmaxThreads;
-constexpr int kStagesK = 3;
-constexpr int kStagesV = 3;
+constexpr int kStages = 3;            // K/V ring depth (one K and one V tile per stage)
 constexpr int kSBufs = 2;
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColO = 256;
@@ -63,13 +66,10 @@ constexpr float kRescaleThreshold = 8.0f;    // log2 units
 // mbarrier slots
 enum {
   B_Q_FULL = 0,
-  B_K_FULL = 1,                       // + stage (kStagesK)
-  B_K_EMPTY = B_K_FULL + kStagesK,    // + stage
-  B_V_FULL = B_K_EMPTY + kStagesK,    // + stage (kStagesV)
-  B_V_EMPTY = B_V_FULL + kStagesV,    // + stage
-  B_S_FULL = B_V_EMPTY + kStagesV,    // + buffer
-  B_S_FREE = B_S_FULL + kSBufs,       // + buffer
-  B_P_FULL = B_S_FREE + kSBufs,
+  B_KV_FULL = 1,                      // + stage: K and V tile of one route entry landed
+  B_KV_EMPTY = B_KV_FULL + kStages,   // + stage: both products that read the stage are done
+  B_S_FULL = B_KV_EMPTY + kStages,    // + buffer
+  B_P_FULL = B_S_FULL + kSBufs,
   B_O_READY,
   B_MMA_DONE,
   B_COUNT
@@ -79,8 +79,8 @@ template <int D>
 struct AttnLayout {
   static constexpr int kTileBytes = kBlk * D * 2;      // 128 rows x D bf16
   static constexpr int kK = 0;
-  static constexpr int kV = kK + kStagesK * kTileBytes;
-  static constexpr int kBars = kV + kStagesV * kTileBytes;
+  static constexpr int kV = kK + kStages * kTileBytes;
+  static constexpr int kBars = kV + kStages * kTileBytes;
   static constexpr int kMisc = kBars + B_COUNT * 8;
   static constexpr int kRed = (kMisc + 64 + 15) & ~15;  // float [3 slots][2 halves][128 rows]
   static constexpr int kTotal = kRed + 3 * 2 * kBlk * 4;
@@ -154,8 +154,7 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t count = 1;
-      if (i == B_Q_FULL || i == B_S_FREE || i == B_S_FREE + 1 || i == B_P_FULL)
-        count = kSoftmaxThreads;
+      if (i == B_Q_FULL || i == B_P_FULL) count = kSoftmaxThreads;
       mbar_init(&bars[i], count);
     }
     *s_abort = 0;
@@ -173,55 +172,49 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     if (lane == 0 && n > 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int issued_k = 0, issued_v = 0;
+      int issued = 0;
       for (int i = 0; i < n; ++i) {
-        const int sk = i % kStagesK, sv = i % kStagesV;
+        const int st = i % kStages;
         const int blk = route_block(a, item, i);
         const int row = static_cast<int>((bh * a.max_blocks + blk) * kBlk);
-        if (i >= kStagesK && !mbar_wait_bounded(&bars[B_K_EMPTY + sk], ((i / kStagesK) - 1) & 1,
-                                                s_abort, kWaitLimit))
+        if (i >= kStages && !mbar_wait_bounded(&bars[B_KV_EMPTY + st], ((i / kStages) - 1) & 1,
+                                               s_abort, kWaitLimit))
           break;
-        mbar_expect_tx(&bars[B_K_FULL + sk], kTileBytes);
-        for (int bx = 0; bx < kBoxes; ++bx)
-          tma_load_2d(sm + L::kK + sk * kTileBytes + bx * (kBlk * 128), &tm_k, bx * 64, row,
-                      &bars[B_K_FULL + sk]);
-        issued_k = i + 1;
-        if (i >= kStagesV && !mbar_wait_bounded(&bars[B_V_EMPTY + sv], ((i / kStagesV) - 1) & 1,
-                                                s_abort, kWaitLimit))
-          break;
-        mbar_expect_tx(&bars[B_V_FULL + sv], kTileBytes);
-        for (int bx = 0; bx < kBoxes; ++bx)
-          tma_load_2d(sm + L::kV + sv * kTileBytes + bx * (kBlk * 128), &tm_v, bx * 64, row,
-                      &bars[B_V_FULL + sv]);
-        issued_v = i + 1;
+        mbar_expect_tx(&bars[B_KV_FULL + st], 2 * kTileBytes);
+        for (int bx = 0; bx < kBoxes; ++bx) {
+          tma_load_2d(sm + L::kK + st * kTileBytes + bx * (kBlk * 128), &tm_k, bx * 64, row,
+                      &bars[B_KV_FULL + st]);
+          tma_load_2d(sm + L::kV + st * kTileBytes + bx * (kBlk * 128), &tm_v, bx * 64, row,
+                      &bars[B_KV_FULL + st]);
+        }
+        issued = i + 1;
       }
-      if (issued_v < n) {
+      if (issued < n) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
         *s_abort = 1;
       }
       // Drain: every copy this thread issued must land before the CTA exits.
-      for (int st = 0; st < kStagesK; ++st) {
+      for (int st = 0; st < kStages; ++st) {
         int last = -1;
-        for (int i = st; i < issued_k; i += kStagesK) last = i;
+        for (int i = st; i < issued; i += kStages) last = i;
         if (last >= 0)
-          mbar_wait_bounded(&bars[B_K_FULL + st], (last / kStagesK) & 1, nullptr, kWaitLimit);
-      }
-      for (int st = 0; st < kStagesV; ++st) {
-        int last = -1;
-        for (int i = st; i < issued_v; i += kStagesV) last = i;
-        if (last >= 0)
-          mbar_wait_bounded(&bars[B_V_FULL + st], (last / kStagesV) & 1, nullptr, kWaitLimit);
+          mbar_wait_bounded(&bars[B_KV_FULL + st], (last / kStages) & 1, nullptr, kWaitLimit);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // Every mbarrier wait of this thread leaves the tensor pipe without new
+    // work for a while, so there are only two per tile: the K/V stage of the
+    // next tile (before its Q K^T) and this tile's P (before its P V).  The S
+    // buffer that Q K^T_{t} overwrites held S_{t-2}; the softmax read it
+    // before storing P_{t-2}, which this thread already waited for.
     if (lane == 0 && n > 0) {
       constexpr uint32_t kIdQK = idesc_bf16(128, 128, 0);
       constexpr uint32_t kIdPV = idesc_bf16(128, D, 1);
       bool ok = mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit);
       auto issue_qk = [&](int t) {
-        const int sk = t % kStagesK, sb = t % kSBufs;
-        const uint32_t k_addr = smem_u32(sm + L::kK + sk * kTileBytes);
+        const int st = t % kStages, sb = t % kSBufs;
+        const uint32_t k_addr = smem_u32(sm + L::kK + st * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kBlk * 128) + (kk % 4) * 32;
@@ -229,9 +222,8 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     smem_desc(k_addr + off, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
         }
         tc_commit(&bars[B_S_FULL + sb]);
-        tc_commit(&bars[B_K_EMPTY + sk]);
       };
-      if (ok) ok = mbar_wait_bounded(&bars[B_K_FULL + 0], 0, s_abort, kWaitLimit);
+      if (ok) ok = mbar_wait_bounded(&bars[B_KV_FULL + 0], 0, s_abort, kWaitLimit);
       if (ok) {
         tc_fence_after();
         issue_qk(0);
@@ -239,28 +231,24 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
       for (int i = 0; ok && i < n; ++i) {
         if (i + 1 < n) {
           const int t = i + 1;
-          ok = mbar_wait_bounded(&bars[B_K_FULL + t % kStagesK], (t / kStagesK) & 1, s_abort,
+          ok = mbar_wait_bounded(&bars[B_KV_FULL + t % kStages], (t / kStages) & 1, s_abort,
                                  kWaitLimit);
-          if (ok && t >= kSBufs)
-            ok = mbar_wait_bounded(&bars[B_S_FREE + t % kSBufs], ((t / kSBufs) - 1) & 1, s_abort,
-                                   kWaitLimit);
           if (!ok) break;
           tc_fence_after();
           issue_qk(t);
         }
-        const int sv = i % kStagesV;
+        const int st = i % kStages;
         ok = mbar_wait_bounded(&bars[B_P_FULL], i & 1, s_abort, kWaitLimit);
-        if (ok) ok = mbar_wait_bounded(&bars[B_V_FULL + sv], (i / kStagesV) & 1, s_abort, kWaitLimit);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm + L::kV + sv * kTileBytes);
+        const uint32_t v_addr = smem_u32(sm + L::kV + st * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
           tc_mma_ts(tmem + kColO, tmem + kColP + kk * 8,
                     smem_desc(v_addr + kk * 2048, kBlk * 128, 1024), kIdPV,
                     (i > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&bars[B_V_EMPTY + sv]);
+        tc_commit(&bars[B_KV_EMPTY + st]);
         tc_commit(&bars[B_O_READY]);
       }
       if (!ok) {
@@ -333,8 +321,6 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
       tc_fence_after();
       float s[kHalfCols];
       tmem_ld_cols<kHalfCols>(tmem + lane_base + kColS + sb * 128 + c0, s);
-      tc_fence_before();
-      mbar_arrive(&bars[B_S_FREE + sb]);
       if (valid < kBlk) {  // tail block of a chunk: mask its pad keys
 #pragma unroll
         for (int c = 0; c < kHalfCols; ++c)
