@@ -210,31 +210,60 @@ class State:
         self.o_blk = torch.empty_like(self.q_blk)
         self.lse = torch.empty((w.B, w.Hh, nbc * BLK), dtype=torch.float32, device=device)
         self.o_tok = torch.empty_like(self.q_tok)
-        self.attn_events = []
+        self.events = []
         bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W)
         torch.cuda.synchronize(device)
         self.q_valid = self.cache.block_valid[self.own_first:self.own_first + nbc].clone()
 
     def step(self, time_attn=False):
+        """One pass of the whole path; with ``time_attn`` every call is
+        bracketed by CUDA events on the current stream (kept in self.events)."""
         bsa, w = self.bsa, self.w
         T, H, W = self.grid
-        self.cache.n_blocks = self.own_first
-        bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W)
-        bsa.bsa_tokens_to_blocks(self.q_tok, T, H, W, out=self.q_blk)
-        bsa.bsa_route(self.q_blk, self.cache, self.n_hist, self.own_first, self.n_own,
-                      w.top_k[0], g=self.g, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale,
-                      q_valid=self.q_valid, max_sel=self.max_sel, idx=self.idx, cnt=self.cnt,
-                      workspace=self.ws)
-        if time_attn:
+        ev = []
+
+        def mark(name, fn):
+            if not time_attn:
+                fn()
+                return
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
-        bsa.bsa_attn(self.q_blk, self.cache, self.idx, self.cnt, q_valid=self.q_valid,
-                     sm_scale=w.sm_scale, o=self.o_blk, lse=self.lse)
-        if time_attn:
+            fn()
             e1.record()
-            self.attn_events.append((e0, e1))
-        bsa.bsa_blocks_to_tokens(self.o_blk, T, H, W, out=self.o_tok)
+            ev.append((name, e0, e1))
+
+        self.cache.n_blocks = self.own_first
+        mark("append", lambda: bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W))
+        mark("q_to_blocks", lambda: bsa.bsa_tokens_to_blocks(self.q_tok, T, H, W, out=self.q_blk))
+        mark("route", lambda: bsa.bsa_route(
+            self.q_blk, self.cache, self.n_hist, self.own_first, self.n_own, w.top_k[0], g=self.g,
+            lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale, q_valid=self.q_valid,
+            max_sel=self.max_sel, idx=self.idx, cnt=self.cnt, workspace=self.ws))
+        mark("attn", lambda: bsa.bsa_attn(self.q_blk, self.cache, self.idx, self.cnt,
+                                          q_valid=self.q_valid, sm_scale=w.sm_scale,
+                                          o=self.o_blk, lse=self.lse))
+        mark("o_to_tokens", lambda: bsa.bsa_blocks_to_tokens(self.o_blk, T, H, W, out=self.o_tok))
+        if time_attn:
+            self.events.append(ev)
+
+    def route_bytes(self) -> float:
+        """Algorithmic bytes of bsa_route: Q read, history K read, g read,
+        scores written and read back by top-K, idx/cnt written."""
+        w = self.w
+        q = w.B * w.Hh * self.n_own * BLK * w.D * 2
+        k = w.B * w.Hh * self.n_hist * BLK * w.D * 2
+        g = 0 if self.g is None else self.g.numel() * 4
+        s = 2 * w.B * w.Hh * self.n_own * self.n_hist * 4
+        idx = (self.idx.numel() + self.cnt.numel()) * 4
+        return float(q + k + g + s + idx)
+
+    def append_bytes(self) -> float:
+        """K and V tokens read plus the chunk's cache blocks written."""
+        w = self.w
+        tok = w.B * w.tokens * w.Hh * w.D * 2
+        blk = w.B * w.Hh * self.n_own * BLK * w.D * 2
+        return float(2 * (tok + blk))
 
     def selected_flops(self) -> float:
         c = self.cnt.to(torch.float64).sum().item()
@@ -260,7 +289,7 @@ def run_ours(args, rank, world, local, pg):
     t_wall0 = time.time()
     torch.cuda.nvtx.range_push("timed")
     step_ms = []
-    st.attn_events = []
+    st.events = []
     for _ in range(args.steps):
         flush.zero_()  # L2 flush between steps, outside the timed events
         e0 = torch.cuda.Event(enable_timing=True)
@@ -275,9 +304,13 @@ def run_ours(args, rank, world, local, pg):
     t_wall1 = time.time()
     st.bsa.raise_on_device_error(device)
     total_ms = sum(a.elapsed_time(b) for a, b in step_ms)
-    attn_ms = [a.elapsed_time(b) for a, b in st.attn_events]
+    phase_ms = {}
+    for ev in st.events:
+        for name, a, b in ev:
+            phase_ms[name] = phase_ms.get(name, 0.0) + a.elapsed_time(b)
+    phase_ms = {k: max_over_ranks(v / len(st.events), pg, device) for k, v in phase_ms.items()}
     total_ms = max_over_ranks(total_ms, pg, device)
-    attn_avg = max_over_ranks(sum(attn_ms) / len(attn_ms), pg, device)
+    attn_avg = phase_ms["attn"]
     clock_info = None
     if clocks is not None:
         time.sleep(0.3)
@@ -314,11 +347,23 @@ def run_ours(args, rank, world, local, pg):
                    "l2": "flushed between steps (256 MB write outside the timed events); "
                          "step inputs also exceed L2"},
         "attn": {"ms_per_call": round(attn_avg, 4), "tflops": round(attn_tflops, 2),
-                 "selected_gflop_per_call": round(flops / 1e9, 3)},
+                 "selected_tflop_per_call": round(flops / 1e12, 4)},
+        "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()},
+        "route": {"ms_per_call": round(phase_ms["route"], 4),
+                  "gbs": round(st.route_bytes() / (phase_ms["route"] * 1e-3) / 1e9, 1),
+                  "frac_of_hbm": round(st.route_bytes() / (phase_ms["route"] * 1e-3) / 1e9
+                                       / peaks["hbm_gbs"], 4),
+                  "bytes_per_call": int(st.route_bytes())},
+        "append": {"ms_per_call": round(phase_ms["append"], 4),
+                   "gbs": round(st.append_bytes() / (phase_ms["append"] * 1e-3) / 1e9, 1),
+                   "frac_of_hbm": round(st.append_bytes() / (phase_ms["append"] * 1e-3) / 1e9
+                                        / peaks["hbm_gbs"], 4),
+                   "bytes_per_call": int(st.append_bytes())},
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} burst dense bf16 (cuBLAS)",
+                     "kernel": "bsa_attn_kernel<128>",
                      "traffic": None},
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * args.steps,

@@ -44,7 +44,8 @@ DEV_CODES = {0: "BSA_DEV_OK", 1: "BSA_DEV_BAD_INDEX", 2: "BSA_DEV_BAD_COUNT",
 # Every symbol include/bsa.h declares (checked by the tests).
 EXPORTS = ("bsa_abi_version", "bsa_status_string", "bsa_gilbert_perm", "bsa_kv_append",
            "bsa_tokens_to_blocks", "bsa_blocks_to_tokens", "bsa_route_workspace_size",
-           "bsa_route", "bsa_route_noalloc", "bsa_attn", "bsa_check_device_error")
+           "bsa_route", "bsa_route_noalloc", "bsa_attn", "bsa_check_device_error",
+           "bsa_selftest_bounded_wait")
 
 
 class BsaError(RuntimeError):
@@ -87,6 +88,7 @@ _sig = {
                                _p, _p, _i, _p, _p]),
     "bsa_attn": (_i, [_p, ctypes.POINTER(CCache), _p, _p, _p, _i, _i, _f, _p, _p, _p, _p]),
     "bsa_check_device_error": (_i, [_p, _p, ctypes.POINTER(ctypes.c_int32)]),
+    "bsa_selftest_bounded_wait": (_i, [_p, ctypes.c_longlong, _p]),
 }
 for _name, (_res, _args) in _sig.items():
     _fn = getattr(_lib, _name)
@@ -358,6 +360,15 @@ def bsa_check_device_error(device="cuda", d_err: Optional[torch.Tensor] = None) 
     code = ctypes.c_int32(0)
     st = _lib.bsa_check_device_error(_ptr(err), _stream(dev), ctypes.byref(code))
     return int(st), int(code.value)
+
+
+def bsa_selftest_bounded_wait(device="cuda", limit_cycles: int = 2_000_000) -> Tuple[int, int]:
+    """Run the bounded-wait self-test; returns bsa_check_device_error's
+    (status, code), which should be (BSA_ERR_TIMEOUT, BSA_DEV_WAIT_TIMEOUT)."""
+    dev = _dev(device)
+    _check("bsa_selftest_bounded_wait", _lib.bsa_selftest_bounded_wait(
+        _ptr(error_word(dev)), int(limit_cycles), _stream(dev)))
+    return bsa_check_device_error(dev)
 
 
 def raise_on_device_error(device="cuda"):

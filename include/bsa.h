@@ -193,6 +193,17 @@ bsa_status bsa_attn(const void *q_blk, const bsa_kv_cache *cache, const int32_t 
                     float sm_scale, void *o_blk, float *lse, int32_t *d_err, void *stream);
 
 /*
+ * Self-test of the bounded-wait failure path used by every pipeline wait in
+ * the library (there is no counterpart in the Velox page).  Launches one
+ * thread that waits on an mbarrier nobody arrives on; after limit_cycles SM
+ * clocks (1 .. 2^34) the wait gives up, BSA_DEV_WAIT_TIMEOUT is written to
+ * d_err, and the kernel returns normally: bsa_check_device_error then
+ * reports BSA_ERR_TIMEOUT and the CUDA context stays usable.
+ * Errors: BSA_ERR_INVALID_ARG (null d_err, limit out of range), BSA_ERR_CUDA.
+ */
+bsa_status bsa_selftest_bounded_wait(int32_t *d_err, long long limit_cycles, void *stream);
+
+/*
  * bsa_route without a workspace argument, for callers that cannot allocate
  * device memory themselves: for example code running inside another
  * runtime's plugin or enqueue hook, where the host framework owns every
