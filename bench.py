@@ -65,6 +65,10 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--chunk", type=int, default=CHUNK)
+    ap.add_argument("--sweep", default="1,2,4,8,12,16,24,32,40,47",
+                    help="chunks of the 48-chunk sweep at which sparse and dense bsa_attn are "
+                         "timed while the cache is built ('' to skip); chunk 48 itself is the "
+                         "timed workload")
     return ap.parse_args()
 
 
@@ -177,10 +181,52 @@ class ClockSampler:
 # our arm
 # ---------------------------------------------------------------------------
 
+def _time_call(fn, reps=3):
+    """Median CUDA-event time (ms) of fn() over `reps` calls after one warm-up."""
+    fn()
+    ts = []
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return sorted(ts)[len(ts) // 2]
+
+
+def sweep_point(bsa, w, cache, q_tok, c, own_first, nbc, device):
+    """bsa_attn of chunk c with its routed top-K and with every cache block
+    selected (dense): the per-chunk comparison of the 48-chunk sweep."""
+    T, H, W = w.grid
+    n_hist = own_first
+    q_blk = bsa.bsa_tokens_to_blocks(q_tok, T, H, W)
+    g = synth.prior(w, c, nbc, n_hist) if n_hist > 0 else None
+    g = torch.from_numpy(g).to(device) if g is not None else None
+    q_valid = cache.block_valid[own_first:own_first + nbc].clone()
+    idx, cnt = bsa.bsa_route(q_blk, cache, n_hist, own_first, nbc, w.top_k[0], g=g, lam=w.lam,
+                             g_ref=w.g_ref, sm_scale=w.sm_scale, q_valid=q_valid)
+    n_all = cache.n_blocks
+    idx_d = torch.arange(n_all, dtype=torch.int32, device=device).expand(
+        w.B, w.Hh, nbc, n_all).contiguous()
+    cnt_d = torch.full((w.B, w.Hh, nbc), n_all, dtype=torch.int32, device=device)
+    o = torch.empty_like(q_blk)
+    lse = torch.empty((w.B, w.Hh, nbc * BLK), dtype=torch.float32, device=device)
+    sp = _time_call(lambda: bsa.bsa_attn(q_blk, cache, idx, cnt, q_valid=q_valid,
+                                         sm_scale=w.sm_scale, o=o, lse=lse))
+    dn = _time_call(lambda: bsa.bsa_attn(q_blk, cache, idx_d, cnt_d, q_valid=q_valid,
+                                         sm_scale=w.sm_scale, o=o, lse=lse))
+    bsa.raise_on_device_error(device)
+    sel = int(cnt[0, 0, 0].item())
+    return {"chunk": c, "selected_blocks": sel, "all_blocks": n_all,
+            "sparse_ms": round(sp, 4), "dense_ms": round(dn, 4), "speedup": round(dn / sp, 2)}
+
+
 class State:
     """Device-resident inputs and preallocated outputs of one rank's problem."""
 
-    def __init__(self, w, chunk, device, seed_rank=0):
+    def __init__(self, w, chunk, device, seed_rank=0, sweep_chunks=()):
         import block_sparse_kv_bsa_b200 as bsa
         self.bsa = bsa
         self.w = w
@@ -193,9 +239,14 @@ class State:
         self.cache = bsa.KVCache(w.B, w.Hh, w.D, self.n_hist + nbc, device=device)
         # A different rank solves a different, equally sized problem.
         wr = w if seed_rank == 0 else synth.Workload(**{**w.__dict__, "key": w.key + 100 * seed_rank})
+        self.sweep = []
         for c in range(1, chunk):
-            t = synth.chunk_tokens(wr, c, device=device, want=("k", "v"))
+            t = synth.chunk_tokens(wr, c, device=device,
+                                   want=("q", "k", "v") if c in sweep_chunks else ("k", "v"))
+            first = self.cache.n_blocks
             bsa.bsa_kv_append(self.cache, t["k"], t["v"], T, H, W)
+            if c in sweep_chunks:
+                self.sweep.append(sweep_point(bsa, wr, self.cache, t["q"], c, first, nbc, device))
         self.own_first = self.cache.n_blocks
         t = synth.chunk_tokens(wr, chunk, device=device)
         self.k_tok, self.v_tok, self.q_tok = t["k"], t["v"], t["q"]
@@ -274,7 +325,8 @@ def run_ours(args, rank, world, local, pg):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = synth.CONFIGS[CONFIG_KEY]
-    st = State(w, args.chunk, device, seed_rank=rank)
+    sweep = {int(x) for x in args.sweep.split(",") if x.strip()} if rank == 0 else set()
+    st = State(w, args.chunk, device, seed_rank=rank, sweep_chunks=sweep)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     for _ in range(max(args.warmup, 3)):
@@ -317,6 +369,9 @@ def run_ours(args, rank, world, local, pg):
         clocks.stop()
         clock_info = clocks.summary(t_wall0, t_wall1)
 
+    if rank == 0 and st.sweep is not None and args.sweep:
+        st.sweep.append(sweep_point(st.bsa, w, st.cache, st.q_tok, args.chunk, st.own_first,
+                                    st.n_own, device))
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(st, args, device, pg, flops)
@@ -367,6 +422,7 @@ def run_ours(args, rank, world, local, pg):
                      "traffic": None},
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "sweep": st.sweep,
         "clocks": clock_info,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

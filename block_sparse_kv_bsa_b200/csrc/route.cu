@@ -9,12 +9,13 @@
 //
 // Three launches, all stream-ordered, no host round trip:
 //   1. pool_q      mean of each query block's valid rows -> qm (workspace)
-//   2. pool_score  stream every history K block once, pool it in registers,
-//                  and score it against all query means of its head at once;
-//                  only the scores s' go to the workspace (the K stream is the
-//                  HBM-bound part of routing)
-//   3. topk        exact top-K per row by radix select on order-preserving
-//                  score keys, ties to the lower index, emitted in ascending
+//   2. pool_score  stream every history K block once (one warp per block),
+//                  pool it in registers, and score it against all query means
+//                  of its head at once; only the model scores go to the
+//                  workspace (the K stream is the HBM-bound part of routing)
+//   3. topk        add the prior (g read row by row), then an exact top-K per
+//                  row by radix select on order-preserving score keys held in
+//                  shared memory, ties to the lower index, emitted in ascending
 //                  index order by a block-wide ordered compaction, followed by
 //                  the own-chunk blocks.
 // All sums run in fp32 in a fixed order, so results are deterministic.
@@ -25,7 +26,6 @@
 namespace bsa {
 
 constexpr int kPoolThreads = 256;
-constexpr int kHistPerCta = 16;
 constexpr int kTopkThreads = 256;
 
 struct RouteArgs {
@@ -51,33 +51,51 @@ __device__ __forceinline__ int clamp_valid(int v, int32_t* d_err) {
   return v;
 }
 
-// Column sums of the first `valid` rows of one 128 x D bf16 block held as
-// VPR 16-byte vectors per row.  Thread t owns vector column t % VPR and rows
-// t / VPR + RG*i.  Partial sums go to `red` [RG][D]; the caller reduces.
+// One 128 x D bf16 block is read as VPR 16-byte vectors per row: thread t
+// owns vector column t % VPR and rows t / VPR + RG*i (RG = 256 / VPR).
 template <int VPR>
-__device__ __forceinline__ void block_colsum_partial(const uint4* blk, int valid, float* red) {
-  constexpr int RG = kPoolThreads / VPR;
-  constexpr int RPT = kBlk / RG;
+struct BlockRegs {
+  static constexpr int RG = kPoolThreads / VPR;
+  static constexpr int RPT = kBlk / RG;
+  uint4 x[RPT];
+};
+
+// Issue the loads of the first `valid` rows of a block (rows past it read 0).
+template <int VPR>
+__device__ __forceinline__ void block_load(const uint4* blk, int valid, BlockRegs<VPR>& r) {
   const int vc = threadIdx.x % VPR;
   const int rg = threadIdx.x / VPR;
-  uint4 x[RPT];
 #pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    int row = rg + RG * i;
-    x[i] = row < valid ? ld_nc_v4(blk + row * VPR + vc) : make_uint4(0, 0, 0, 0);
+  for (int i = 0; i < BlockRegs<VPR>::RPT; ++i) {
+    int row = rg + BlockRegs<VPR>::RG * i;
+    r.x[i] = row < valid ? ld_nc_v4(blk + row * VPR + vc) : make_uint4(0, 0, 0, 0);
   }
+}
+
+// Column sums of this thread's rows -> red [RG][D]; the caller reduces.
+template <int VPR>
+__device__ __forceinline__ void block_colsum_store(const BlockRegs<VPR>& r, float* red) {
+  const int vc = threadIdx.x % VPR;
+  const int rg = threadIdx.x / VPR;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
-  for (int i = 0; i < RPT; ++i) {
-    acc[0] += bf16lo(x[i].x); acc[1] += bf16hi(x[i].x);
-    acc[2] += bf16lo(x[i].y); acc[3] += bf16hi(x[i].y);
-    acc[4] += bf16lo(x[i].z); acc[5] += bf16hi(x[i].z);
-    acc[6] += bf16lo(x[i].w); acc[7] += bf16hi(x[i].w);
+  for (int i = 0; i < BlockRegs<VPR>::RPT; ++i) {
+    acc[0] += bf16lo(r.x[i].x); acc[1] += bf16hi(r.x[i].x);
+    acc[2] += bf16lo(r.x[i].y); acc[3] += bf16hi(r.x[i].y);
+    acc[4] += bf16lo(r.x[i].z); acc[5] += bf16hi(r.x[i].z);
+    acc[6] += bf16lo(r.x[i].w); acc[7] += bf16hi(r.x[i].w);
   }
 #pragma unroll
   for (int e = 0; e < 8; ++e) red[rg * (VPR * 8) + vc * 8 + e] = acc[e];
+}
+
+template <int VPR>
+__device__ __forceinline__ void block_colsum_partial(const uint4* blk, int valid, float* red) {
+  BlockRegs<VPR> r;
+  block_load<VPR>(blk, valid, r);
+  block_colsum_store<VPR>(r, red);
 }
 
 // Finish the mean: out[d] = sum_rg red[rg][d] / valid (threads d < D).
@@ -107,47 +125,99 @@ __global__ void __launch_bounds__(kPoolThreads) pool_q_kernel(RouteArgs a) {
   block_mean_finish<VPR>(red, valid, a.qm + (bh * a.n_own + j) * D);
 }
 
+// K-stream kernel: one warp reduces one history block at a time.  A CTA of
+// 8 warps covers kScoreBlocksPerWarp consecutive blocks per warp of one
+// (b, h), with that head's query means in shared memory (the only CTA-wide
+// barrier).  Per block, each lane issues 16 independent 16-byte loads per
+// batch (rows past the valid count read as 0), accumulates 8 fp32 column sums,
+// the lanes holding the same columns are combined by shuffles, and the block
+// mean is scored against every query mean (four independent shuffle chains
+// per pass).  Many warps per SM and no per-block barrier keep HBM busy.
+// The prior is added by the top-K kernel, which reads g row by row.
+constexpr int kScoreWarps = 8;
+constexpr int kScoreBlocksPerWarp = 8;
+
 template <int VPR>
-__global__ void __launch_bounds__(kPoolThreads) pool_score_kernel(RouteArgs a) {
+__global__ void __launch_bounds__(kScoreWarps * 32)
+pool_score_kernel(RouteArgs a) {
   constexpr int D = VPR * 8;
-  constexpr int EPL = D / 32;  // elements of a mean per lane
-  extern __shared__ float sm[];
-  float* qm = sm;                                  // [n_own][D]
-  float* red = qm + a.n_own * D;                   // [RG][D]
-  float* km = red + (kPoolThreads / VPR) * D;      // [D]
+  constexpr int LPR = VPR;              // lanes per row (one 16-byte chunk each)
+  constexpr int RPI = 32 / LPR;         // rows per warp-wide load (2 or 4)
+  constexpr int NB = 16;                // loads in flight per lane per batch
+  constexpr int kBatches = kBlk / (RPI * NB);
+  extern __shared__ float qm[];         // [n_own][D] of this head
   const int h = blockIdx.y, b = blockIdx.z;
   const long long bh = static_cast<long long>(b) * a.Hh + h;
-  const int n_first = blockIdx.x * kHistPerCta;
-
-  for (int i = threadIdx.x; i < a.n_own * D; i += kPoolThreads) qm[i] = a.qm[bh * a.n_own * D + i];
-
+  for (int i = threadIdx.x; i < a.n_own * D; i += kScoreWarps * 32) qm[i] = a.qm[bh * a.n_own * D + i];
+  __syncthreads();
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  for (int nn = 0; nn < kHistPerCta; ++nn) {
-    const int n = n_first + nn;
+  const int c = lane % LPR;             // 16-byte column chunk of this lane
+  const int g = lane / LPR;             // row phase within a load / query-block phase
+  const int n_base = (blockIdx.x * kScoreWarps + warp) * kScoreBlocksPerWarp;
+  for (int u = 0; u < kScoreBlocksPerWarp; ++u) {
+    const int n = n_base + u;
     if (n >= a.n_hist) break;
     const int valid = clamp_valid(a.block_valid[n], a.d_err);
     const uint4* blk = a.kc + (bh * a.max_blocks + n) * kBlk * VPR;
-    __syncthreads();  // previous block's km / red are consumed
-    block_colsum_partial<VPR>(blk, valid, red);
-    __syncthreads();
-    block_mean_finish<VPR>(red, valid, km);
-    __syncthreads();
-    float kr[EPL];
+    float acc[8];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) kr[e] = km[lane + 32 * e];
-    for (int j = warp; j < a.n_own; j += kPoolThreads / 32) {
-      float d = 0.f;
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) d = fmaf(qm[j * D + lane + 32 * e], kr[e], d);
+    for (int bt = 0; bt < kBatches; ++bt) {
+      uint4 x[NB];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-      if (lane == 0) {
-        float sc = a.sm_scale * d;
-        if (a.g != nullptr) {
-          float gv = a.g[(static_cast<long long>(b) * a.n_own + j) * a.n_hist + n];
-          sc += a.lam * fminf(gv / a.g_ref, 1.0f);
+      for (int i = 0; i < NB; ++i) {
+        const int row = (bt * NB + i) * RPI + g;
+        x[i] = row < valid ? ld_nc_v4(blk + row * VPR + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int i = 0; i < NB; ++i) {
+        acc[0] += bf16lo(x[i].x); acc[1] += bf16hi(x[i].x);
+        acc[2] += bf16lo(x[i].y); acc[3] += bf16hi(x[i].y);
+        acc[4] += bf16lo(x[i].z); acc[5] += bf16hi(x[i].z);
+        acc[6] += bf16lo(x[i].w); acc[7] += bf16hi(x[i].w);
+      }
+    }
+    // Combine the RPI lanes that hold the same columns (fixed order).
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    }
+    float km[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) km[e] = acc[e] / static_cast<float>(valid);
+    // Scores: lane group g takes query blocks j = g, g + RPI, ...; the LPR
+    // lanes of a group each hold 8 columns and are reduced by shuffles.  The
+    // loop bound is the same for every lane (the shuffles are warp-wide);
+    // out-of-range query blocks only skip their arithmetic.
+    for (int jb = 0; jb < a.n_own; jb += 4 * RPI) {
+      const int j0 = jb + g;
+      float d[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        d[t] = 0.f;
+        const int j = j0 + t * RPI;
+        if (j < a.n_own) {
+          const float4* q4 = reinterpret_cast<const float4*>(qm + j * D + c * 8);
+          const float4 q0 = q4[0], q1 = q4[1];
+          d[t] = fmaf(q0.x, km[0], d[t]); d[t] = fmaf(q0.y, km[1], d[t]);
+          d[t] = fmaf(q0.z, km[2], d[t]); d[t] = fmaf(q0.w, km[3], d[t]);
+          d[t] = fmaf(q1.x, km[4], d[t]); d[t] = fmaf(q1.y, km[5], d[t]);
+          d[t] = fmaf(q1.z, km[6], d[t]); d[t] = fmaf(q1.w, km[7], d[t]);
         }
-        a.s[(bh * a.n_own + j) * a.n_hist + n] = sc;
+      }
+#pragma unroll
+      for (int off = 1; off < LPR; off <<= 1) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) d[t] += __shfl_xor_sync(0xffffffffu, d[t], off);
+      }
+      if (c < 4) {
+        float dv = d[0];
+#pragma unroll
+        for (int t = 1; t < 4; ++t) dv = c == t ? d[t] : dv;
+        const int j = j0 + c * RPI;
+        if (j < a.n_own) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * dv;
       }
     }
   }
@@ -179,7 +249,20 @@ __device__ __forceinline__ int block_excl_count(bool flag, int* warp_tot, int* t
   return before + in_warp;
 }
 
+// Keys of a row at most this long are staged in shared memory.
+constexpr int kTopkSmemKeys = 40960;
+
+// Fused score of history block n of row (b, j): the model score plus the
+// prior boost lam * min(g / g_ref, 1) (g shared by all heads).
+__device__ __forceinline__ float fused_score(const RouteArgs& a, const float* sr, const float* gr,
+                                             int n) {
+  float sc = sr[n];
+  if (gr != nullptr) sc += a.lam * fminf(gr[n] / a.g_ref, 1.0f);
+  return sc;
+}
+
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(RouteArgs a) {
+  extern __shared__ uint32_t keys[];   // [n_hist] when staged
   __shared__ int hist[256];
   __shared__ int warp_tot[kTopkThreads / 32];
   __shared__ uint32_t s_prefix;
@@ -188,18 +271,29 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(RouteArgs a) {
   const long long row = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
   int32_t* out = a.idx + row * a.max_sel;
   const float* sr = a.s + row * a.n_hist;
+  const float* gr = a.g != nullptr ? a.g + (static_cast<long long>(b) * a.n_own + j) * a.n_hist
+                                   : nullptr;
   const int K = a.top_k < a.n_hist ? a.top_k : a.n_hist;
+  const bool staged = a.n_hist <= kTopkSmemKeys;
+  auto key_at = [&](int n) -> uint32_t {
+    return staged ? keys[n] : score_key(fused_score(a, sr, gr, n));
+  };
 
   if (K == a.n_hist) {
     for (int n = threadIdx.x; n < a.n_hist; n += kTopkThreads) out[n] = n;
   } else if (K > 0) {
+    if (staged) {
+      for (int n = threadIdx.x; n < a.n_hist; n += kTopkThreads)
+        keys[n] = score_key(fused_score(a, sr, gr, n));
+      __syncthreads();
+    }
     uint32_t prefix = 0, pmask = 0;
     int remaining = K;
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = threadIdx.x; i < 256; i += kTopkThreads) hist[i] = 0;
       __syncthreads();
       for (int n = threadIdx.x; n < a.n_hist; n += kTopkThreads) {
-        uint32_t k = score_key(sr[n]);
+        uint32_t k = key_at(n);
         if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
       }
       __syncthreads();
@@ -224,7 +318,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(RouteArgs a) {
     int pos = 0, eq_seen = 0;
     for (int base = 0; base < a.n_hist; base += kTopkThreads) {
       const int n = base + threadIdx.x;
-      uint32_t k = n < a.n_hist ? score_key(sr[n]) : 0u;
+      uint32_t k = n < a.n_hist ? key_at(n) : 0u;
       bool gt = n < a.n_hist && k > thr;
       bool eq = n < a.n_hist && k == thr;
       int eq_tot, sel_tot;
@@ -248,11 +342,6 @@ static void route_ws_layout(int B, int Hh, int D, int n_own, int n_hist, size_t*
   *qm_bytes = align256(sizeof(float) * static_cast<size_t>(B) * Hh * n_own * D);
   *s_bytes = align256(sizeof(float) * static_cast<size_t>(B) * Hh * n_own *
                       static_cast<size_t>(n_hist > 0 ? n_hist : 0));
-}
-
-static size_t pool_score_smem(int D, int n_own) {
-  int vpr = D / 8;
-  return sizeof(float) * (static_cast<size_t>(n_own) * D + (kPoolThreads / vpr) * D + D);
 }
 
 }  // namespace bsa
@@ -293,8 +382,10 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   size_t qm_b, s_b;
   route_ws_layout(c->B, c->Hh, c->D, n_own, n_hist, &qm_b, &s_b);
   if (ws_bytes < qm_b + s_b) return BSA_ERR_CAPACITY;
-  const size_t smem = pool_score_smem(c->D, n_own);
-  if (smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
+  const size_t qm_smem = sizeof(float) * static_cast<size_t>(n_own) * c->D;
+  if (qm_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
+  const size_t topk_smem =
+      n_hist <= kTopkSmemKeys ? sizeof(uint32_t) * static_cast<size_t>(n_hist > 0 ? n_hist : 1) : 0;
 
   RouteArgs a{};
   a.q = static_cast<const uint4*>(q_blk);
@@ -321,25 +412,29 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
 
   cudaStream_t s = as_stream(stream);
   dim3 qgrid(n_own, c->Hh, c->B);
-  dim3 sgrid((n_hist + kHistPerCta - 1) / kHistPerCta, c->Hh, c->B);
+  const int per_cta = kScoreWarps * kScoreBlocksPerWarp;
+  dim3 sgrid((n_hist + per_cta - 1) / per_cta, c->Hh, c->B);
   if (c->D == 128) {
+    pool_q_kernel<16><<<qgrid, kPoolThreads, 0, s>>>(a);
     if (n_hist > 0) {
       if (cudaFuncSetAttribute(pool_score_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
+                               static_cast<int>(qm_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
+      pool_score_kernel<16><<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
     }
-    pool_q_kernel<16><<<qgrid, kPoolThreads, 0, s>>>(a);
-    if (n_hist > 0) pool_score_kernel<16><<<sgrid, kPoolThreads, smem, s>>>(a);
   } else {
+    pool_q_kernel<8><<<qgrid, kPoolThreads, 0, s>>>(a);
     if (n_hist > 0) {
       if (cudaFuncSetAttribute(pool_score_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem)) != cudaSuccess)
+                               static_cast<int>(qm_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
+      pool_score_kernel<8><<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
     }
-    pool_q_kernel<8><<<qgrid, kPoolThreads, 0, s>>>(a);
-    if (n_hist > 0) pool_score_kernel<8><<<sgrid, kPoolThreads, smem, s>>>(a);
   }
-  topk_kernel<<<qgrid, kTopkThreads, 0, s>>>(a);
+  if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(topk_smem)) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  topk_kernel<<<qgrid, kTopkThreads, topk_smem, s>>>(a);
   return launch_status();
 }
 
