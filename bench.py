@@ -72,6 +72,26 @@ def parse_args():
     return ap.parse_args()
 
 
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from profiles/traffic.json (one ncu
+    capture of this workload), or None when the kernel's sources changed
+    since the capture or there is no capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            entry = json.load(f)[kernel]
+        h = hashlib.sha256()
+        for rel in entry["files"]:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != entry["sources"]:
+            return None
+        return int(entry["read"]) + int(entry["write"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -408,18 +428,23 @@ def run_ours(args, rank, world, local, pg):
                   "gbs": round(st.route_bytes() / (phase_ms["route"] * 1e-3) / 1e9, 1),
                   "frac_of_hbm": round(st.route_bytes() / (phase_ms["route"] * 1e-3) / 1e9
                                        / peaks["hbm_gbs"], 4),
-                  "bytes_per_call": int(st.route_bytes())},
+                  "bytes_per_call": int(st.route_bytes()),
+                  "pool_score_traffic": (measured_traffic("pool_score_kernel<16>")
+                                         if args.chunk == CHUNK else None)},
         "append": {"ms_per_call": round(phase_ms["append"], 4),
                    "gbs": round(st.append_bytes() / (phase_ms["append"] * 1e-3) / 1e9, 1),
                    "frac_of_hbm": round(st.append_bytes() / (phase_ms["append"] * 1e-3) / 1e9
                                         / peaks["hbm_gbs"], 4),
-                   "bytes_per_call": int(st.append_bytes())},
+                   "bytes_per_call": int(st.append_bytes()),
+                   "traffic": (measured_traffic("reorder_kernel<16,1>")
+                               if args.chunk == CHUNK else None)},
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} burst dense bf16 (cuBLAS)",
                      "kernel": "bsa_attn_kernel<128>",
-                     "traffic": None},
+                     "traffic": (measured_traffic("bsa_attn_kernel<128>")
+                                 if args.chunk == CHUNK else None)},
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "sweep": st.sweep,
