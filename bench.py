@@ -52,7 +52,8 @@ CHUNK = 48
 BLK = 128
 METRIC = "bsa_attn selected-block TFLOP/s at chunk 48 (48-chunk sweep), 1 B200"
 L2_FLUSH_BYTES = 256 << 20
-KERNELS_PER_STEP = 7  # append, tokens->blocks, pool_q, pool_score, topk, attn, blocks->tokens
+# append (scatter + key means), tokens->blocks, pool_q, pool_score, topk, attn, blocks->tokens
+KERNELS_PER_STEP = 8
 
 
 def parse_args():
@@ -256,7 +257,10 @@ class State:
         self.n_own = nbc
         self.n_hist = nbc * (chunk - 1)
         self.device = device
-        self.cache = bsa.KVCache(w.B, w.Hh, w.D, self.n_hist + nbc, device=device)
+        # The pooled-key cache: bsa_kv_append writes each block's key mean, and
+        # bsa_route scores from those instead of re-reading the history keys.
+        self.cache = bsa.KVCache(w.B, w.Hh, w.D, self.n_hist + nbc, device=device,
+                                 pooled_keys=True)
         # A different rank solves a different, equally sized problem.
         wr = w if seed_rank == 0 else synth.Workload(**{**w.__dict__, "key": w.key + 100 * seed_rank})
         self.sweep = []
@@ -318,23 +322,54 @@ class State:
         if time_attn:
             self.events.append(ev)
 
-    def route_bytes(self) -> float:
-        """Algorithmic bytes of bsa_route: Q read, history K read, g read,
-        scores written and read back by top-K, idx/cnt written."""
+    def route_bytes(self, from_means: bool = True) -> float:
+        """Algorithmic bytes of bsa_route: Q read, the history key means (or the
+        history keys themselves when streaming), g read, model scores written
+        and read back by top-K, idx/cnt written."""
         w = self.w
         q = w.B * w.Hh * self.n_own * BLK * w.D * 2
-        k = w.B * w.Hh * self.n_hist * BLK * w.D * 2
+        if from_means:
+            k = w.B * w.Hh * self.n_hist * w.D * 4
+        else:
+            k = w.B * w.Hh * self.n_hist * BLK * w.D * 2
         g = 0 if self.g is None else self.g.numel() * 4
         s = 2 * w.B * w.Hh * self.n_own * self.n_hist * 4
         idx = (self.idx.numel() + self.cnt.numel()) * 4
         return float(q + k + g + s + idx)
 
     def append_bytes(self) -> float:
-        """K and V tokens read plus the chunk's cache blocks written."""
+        """K and V tokens read, the chunk's cache blocks written, and the
+        chunk's key means written."""
         w = self.w
         tok = w.B * w.tokens * w.Hh * w.D * 2
         blk = w.B * w.Hh * self.n_own * BLK * w.D * 2
-        return float(2 * (tok + blk))
+        means = w.B * w.Hh * self.n_own * w.D * 4
+        return float(2 * (tok + blk) + means)
+
+    def route_stream_ms(self, flush, reps: int = 20) -> float:
+        """bsa_route timed without the pooled-key cache, i.e. streaming every
+        history key block (L2 flushed before each call)."""
+        w, bsa = self.w, self.bsa
+        saved = self.cache.kmean
+        self.cache.kmean = None
+        ts = []
+        try:
+            for i in range(reps + 2):
+                flush.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                bsa.bsa_route(self.q_blk, self.cache, self.n_hist, self.own_first, self.n_own,
+                              w.top_k[0], g=self.g, lam=w.lam, g_ref=w.g_ref,
+                              sm_scale=w.sm_scale, q_valid=self.q_valid, max_sel=self.max_sel,
+                              idx=self.idx, cnt=self.cnt, workspace=self.ws)
+                e1.record()
+                torch.cuda.synchronize()
+                if i >= 2:
+                    ts.append(e0.elapsed_time(e1))
+        finally:
+            self.cache.kmean = saved
+        return sorted(ts)[len(ts) // 2]
 
     def selected_flops(self) -> float:
         c = self.cnt.to(torch.float64).sum().item()
@@ -389,6 +424,7 @@ def run_ours(args, rank, world, local, pg):
         clocks.stop()
         clock_info = clocks.summary(t_wall0, t_wall1)
 
+    route_stream = st.route_stream_ms(flush)
     if rank == 0 and st.sweep is not None and args.sweep:
         st.sweep.append(sweep_point(st.bsa, w, st.cache, st.q_tok, args.chunk, st.own_first,
                                     st.n_own, device))
@@ -425,12 +461,17 @@ def run_ours(args, rank, world, local, pg):
                  "selected_tflop_per_call": round(flops / 1e12, 4)},
         "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()},
         "route": {"ms_per_call": round(phase_ms["route"], 4),
+                  "keys": "pooled-key cache (means written by bsa_kv_append)",
                   "gbs": round(st.route_bytes() / (phase_ms["route"] * 1e-3) / 1e9, 1),
-                  "frac_of_hbm": round(st.route_bytes() / (phase_ms["route"] * 1e-3) / 1e9
-                                       / peaks["hbm_gbs"], 4),
-                  "bytes_per_call": int(st.route_bytes()),
-                  "pool_score_traffic": (measured_traffic("pool_score_kernel<16>")
-                                         if args.chunk == CHUNK else None)},
+                  "bytes_per_call": int(st.route_bytes())},
+        "route_stream": {"ms_per_call": round(route_stream, 4),
+                         "keys": "history keys streamed from the cache (no pooled-key cache)",
+                         "gbs": round(st.route_bytes(False) / (route_stream * 1e-3) / 1e9, 1),
+                         "frac_of_hbm": round(st.route_bytes(False) / (route_stream * 1e-3) / 1e9
+                                              / peaks["hbm_gbs"], 4),
+                         "bytes_per_call": int(st.route_bytes(False)),
+                         "pool_score_traffic": (measured_traffic("pool_score_kernel<16>")
+                                                if args.chunk == CHUNK else None)},
         "append": {"ms_per_call": round(phase_ms["append"], 4),
                    "gbs": round(st.append_bytes() / (phase_ms["append"] * 1e-3) / 1e9, 1),
                    "frac_of_hbm": round(st.append_bytes() / (phase_ms["append"] * 1e-3) / 1e9

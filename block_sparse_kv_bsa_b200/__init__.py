@@ -43,6 +43,7 @@ DEV_CODES = {0: "BSA_DEV_OK", 1: "BSA_DEV_BAD_INDEX", 2: "BSA_DEV_BAD_COUNT",
 
 # Every symbol include/bsa.h declares (checked by the tests).
 EXPORTS = ("bsa_abi_version", "bsa_status_string", "bsa_gilbert_perm", "bsa_kv_append",
+           "bsa_kv_pool_means",
            "bsa_tokens_to_blocks", "bsa_blocks_to_tokens", "bsa_route_workspace_size",
            "bsa_route", "bsa_route_noalloc", "bsa_attn", "bsa_check_device_error",
            "bsa_selftest_bounded_wait")
@@ -70,7 +71,8 @@ class CCache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("block_valid", ctypes.c_void_p),
                 ("B", ctypes.c_int32), ("Hh", ctypes.c_int32), ("D", ctypes.c_int32),
-                ("max_blocks", ctypes.c_int32), ("n_blocks", ctypes.c_int32)]
+                ("max_blocks", ctypes.c_int32), ("n_blocks", ctypes.c_int32),
+                ("kmean", ctypes.c_void_p)]
 
 
 _i, _p, _f, _sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
@@ -79,6 +81,7 @@ _sig = {
     "bsa_status_string": (ctypes.c_char_p, [_i]),
     "bsa_gilbert_perm": (_i, [_i, _i, _i, _p]),
     "bsa_kv_append": (_i, [ctypes.POINTER(CCache), _p, _p, _i, _i, _i, _p, _p, _p]),
+    "bsa_kv_pool_means": (_i, [ctypes.POINTER(CCache), _i, _i, _p, _p]),
     "bsa_tokens_to_blocks": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "bsa_blocks_to_tokens": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "bsa_route_workspace_size": (_i, [_i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
@@ -200,18 +203,24 @@ class KVCache:
     """A caller-owned block KV cache: K, V bf16 [B, Hh, max_blocks, 128, D] and
     the valid-row count of every block."""
 
-    def __init__(self, B: int, Hh: int, D: int, max_blocks: int, device="cuda"):
+    def __init__(self, B: int, Hh: int, D: int, max_blocks: int, device="cuda",
+                 pooled_keys: bool = False):
         self.B, self.Hh, self.D, self.max_blocks = int(B), int(Hh), int(D), int(max_blocks)
         self.device = _dev(device)
         shape = (self.B, self.Hh, self.max_blocks, BLK, self.D)
         self.k = torch.zeros(shape, dtype=torch.bfloat16, device=self.device)
         self.v = torch.zeros(shape, dtype=torch.bfloat16, device=self.device)
         self.block_valid = torch.zeros(self.max_blocks, dtype=torch.int32, device=self.device)
+        # Optional pooled-key cache: block means of K, written at append time
+        # and read by bsa_route instead of the history keys.
+        self.kmean = (torch.zeros((self.B, self.Hh, self.max_blocks, self.D), dtype=torch.float32,
+                                  device=self.device) if pooled_keys else None)
         self.n_blocks = 0
 
     def c_struct(self) -> CCache:
         return CCache(self.k.data_ptr(), self.v.data_ptr(), self.block_valid.data_ptr(),
-                      self.B, self.Hh, self.D, self.max_blocks, self.n_blocks)
+                      self.B, self.Hh, self.D, self.max_blocks, self.n_blocks,
+                      None if self.kmean is None else self.kmean.data_ptr())
 
 
 def bsa_kv_append(cache: KVCache, k_tok: torch.Tensor, v_tok: torch.Tensor,
@@ -229,6 +238,18 @@ def bsa_kv_append(cache: KVCache, k_tok: torch.Tensor, v_tok: torch.Tensor,
                                                 _stream(cache.device)))
     cache.n_blocks = int(cs.n_blocks)
     return first
+
+
+def bsa_kv_pool_means(cache: KVCache, first: int = 0, count: Optional[int] = None):
+    """(Re)compute the pooled-key cache for blocks [first, first + count)."""
+    if cache.kmean is None:
+        raise ValueError("the cache was created without pooled_keys")
+    if count is None:
+        count = cache.n_blocks - first
+    cs = cache.c_struct()
+    _check("bsa_kv_pool_means", _lib.bsa_kv_pool_means(
+        ctypes.byref(cs), int(first), int(count), _ptr(error_word(cache.device)),
+        _stream(cache.device)))
 
 
 def bsa_tokens_to_blocks(x_tok: torch.Tensor, T: int, H: int, W: int,

@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "gilbert.cuh"
+#include "pool.cuh"
 
 namespace bsa {
 
@@ -134,6 +135,49 @@ static bsa_status launch_reorder(const ReorderArgs& a, int D, cudaStream_t s) {
   return launch_status();
 }
 
+// Pooled-key cache: one warp per (b, h, block) writes the fp32 mean of the
+// block's valid key rows (the router's own pooling code, pool.cuh).
+constexpr int kMeanWarps = 8;
+
+template <int VPR>
+__global__ void __launch_bounds__(kMeanWarps * 32)
+block_mean_kernel(const uint4* kc, const int32_t* block_valid, float* kmean, int Hh,
+                  int max_blocks, int first, int count, int32_t* d_err) {
+  constexpr int D = VPR * 8;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int i = blockIdx.x * kMeanWarps + warp;
+  if (i >= count) return;
+  const int n = first + i;
+  const long long bh = static_cast<long long>(blockIdx.z) * Hh + blockIdx.y;
+  int valid = block_valid[n];
+  if (valid < 1 || valid > kBlk) {
+    report(d_err, BSA_DEV_BAD_VALID);
+    valid = valid < 1 ? 1 : kBlk;
+  }
+  const int c = lane % VPR, g = lane / VPR;
+  float km[8];
+  warp_block_mean<VPR>(kc + (bh * max_blocks + n) * kBlk * VPR, valid, c, g, km);
+  if (g == 0) {
+    float4* out = reinterpret_cast<float4*>(kmean + (bh * max_blocks + n) * D + c * 8);
+    out[0] = make_float4(km[0], km[1], km[2], km[3]);
+    out[1] = make_float4(km[4], km[5], km[6], km[7]);
+  }
+}
+
+static bsa_status launch_block_means(const bsa_kv_cache* c, int first, int count, int32_t* d_err,
+                                     cudaStream_t s) {
+  if (count <= 0) return BSA_OK;
+  dim3 grid((count + kMeanWarps - 1) / kMeanWarps, c->Hh, c->B);
+  const uint4* kc = static_cast<const uint4*>(c->k);
+  if (c->D == 128)
+    block_mean_kernel<16><<<grid, kMeanWarps * 32, 0, s>>>(kc, c->block_valid, c->kmean, c->Hh,
+                                                           c->max_blocks, first, count, d_err);
+  else
+    block_mean_kernel<8><<<grid, kMeanWarps * 32, 0, s>>>(kc, c->block_valid, c->kmean, c->Hh,
+                                                          c->max_blocks, first, count, d_err);
+  return launch_status();
+}
+
 static bsa_status check_chunk(int B, int Hh, int D, int T, int H, int W) {
   if (B <= 0 || Hh <= 0 || T <= 0 || H <= 0 || W <= 0) return BSA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return BSA_ERR_UNSUPPORTED;
@@ -190,6 +234,7 @@ extern "C" bsa_status bsa_kv_append(bsa_kv_cache* c, const void* k_tok, const vo
   const int n = T * H * W;
   const int nb = (n + kBlk - 1) / kBlk;
   if (c->n_blocks + nb > c->max_blocks) return BSA_ERR_CAPACITY;
+  if (c->kmean != nullptr && !aligned16(c->kmean)) return BSA_ERR_INVALID_ARG;
   ReorderArgs a{};
   a.src0 = static_cast<const uint4*>(k_tok);
   a.dst0 = static_cast<uint4*>(c->k);
@@ -205,8 +250,21 @@ extern "C" bsa_status bsa_kv_append(bsa_kv_cache* c, const void* k_tok, const vo
   a.blk_stride = c->max_blocks;
   a.base_block = c->n_blocks;
   st = launch_reorder<true>(a, c->D, as_stream(stream));
+  if (st == BSA_OK && c->kmean != nullptr)
+    st = launch_block_means(c, c->n_blocks, nb, d_err, as_stream(stream));
   if (st == BSA_OK) c->n_blocks += nb;
   return st;
+}
+
+extern "C" bsa_status bsa_kv_pool_means(const bsa_kv_cache* c, int first, int count,
+                                        int32_t* d_err, void* stream) {
+  if (c == nullptr || c->k == nullptr || c->kmean == nullptr || c->block_valid == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (c->D != 64 && c->D != 128) return BSA_ERR_UNSUPPORTED;
+  if (c->B <= 0 || c->Hh <= 0 || c->B > 65535 || c->Hh > 65535 || first < 0 || count < 0 ||
+      first + count > c->max_blocks || !aligned16(c->k) || !aligned16(c->kmean))
+    return BSA_ERR_INVALID_ARG;
+  return launch_block_means(c, first, count, d_err, as_stream(stream));
 }
 
 extern "C" bsa_status bsa_tokens_to_blocks(const void* x_tok, void* x_blk, int B, int Hh, int D,

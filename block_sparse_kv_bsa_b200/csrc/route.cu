@@ -22,6 +22,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "pool.cuh"
 
 namespace bsa {
 
@@ -34,6 +35,7 @@ struct RouteArgs {
   const int32_t* block_valid;
   const int32_t* q_valid;  // [n_own] or null
   const float* g;          // [B, n_own, n_hist] or null
+  const float* kmean;      // [B, Hh, max_blocks, D] pooled keys, or null
   float* qm;               // [B, Hh, n_own, D]
   float* s;                // [B, Hh, n_own, n_hist]
   int32_t* idx;
@@ -137,14 +139,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_q_kernel(RouteArgs a) {
 constexpr int kScoreWarps = 8;
 constexpr int kScoreBlocksPerWarp = 8;
 
-template <int VPR>
+template <int VPR, bool kFromMeans>
 __global__ void __launch_bounds__(kScoreWarps * 32)
 pool_score_kernel(RouteArgs a) {
   constexpr int D = VPR * 8;
   constexpr int LPR = VPR;              // lanes per row (one 16-byte chunk each)
   constexpr int RPI = 32 / LPR;         // rows per warp-wide load (2 or 4)
-  constexpr int NB = 16;                // loads in flight per lane per batch
-  constexpr int kBatches = kBlk / (RPI * NB);
   extern __shared__ float qm[];         // [n_own][D] of this head
   const int h = blockIdx.y, b = blockIdx.z;
   const long long bh = static_cast<long long>(b) * a.Hh + h;
@@ -157,36 +157,18 @@ pool_score_kernel(RouteArgs a) {
   for (int u = 0; u < kScoreBlocksPerWarp; ++u) {
     const int n = n_base + u;
     if (n >= a.n_hist) break;
-    const int valid = clamp_valid(a.block_valid[n], a.d_err);
-    const uint4* blk = a.kc + (bh * a.max_blocks + n) * kBlk * VPR;
-    float acc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-    for (int bt = 0; bt < kBatches; ++bt) {
-      uint4 x[NB];
-#pragma unroll
-      for (int i = 0; i < NB; ++i) {
-        const int row = (bt * NB + i) * RPI + g;
-        x[i] = row < valid ? ld_nc_v4(blk + row * VPR + c) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int i = 0; i < NB; ++i) {
-        acc[0] += bf16lo(x[i].x); acc[1] += bf16hi(x[i].x);
-        acc[2] += bf16lo(x[i].y); acc[3] += bf16hi(x[i].y);
-        acc[4] += bf16lo(x[i].z); acc[5] += bf16hi(x[i].z);
-        acc[6] += bf16lo(x[i].w); acc[7] += bf16hi(x[i].w);
-      }
-    }
-    // Combine the RPI lanes that hold the same columns (fixed order).
-#pragma unroll
-    for (int off = LPR; off < 32; off <<= 1) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
-    }
     float km[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) km[e] = acc[e] / static_cast<float>(valid);
+    if (kFromMeans) {
+      // The block mean was written when the block was appended (same code).
+      const float4* m4 =
+          reinterpret_cast<const float4*>(a.kmean + ((bh * a.max_blocks + n) * D + c * 8));
+      const float4 m0 = m4[0], m1 = m4[1];
+      km[0] = m0.x; km[1] = m0.y; km[2] = m0.z; km[3] = m0.w;
+      km[4] = m1.x; km[5] = m1.y; km[6] = m1.z; km[7] = m1.w;
+    } else {
+      const int valid = clamp_valid(a.block_valid[n], a.d_err);
+      warp_block_mean<VPR>(a.kc + (bh * a.max_blocks + n) * kBlk * VPR, valid, c, g, km);
+    }
     // Scores: lane group g takes query blocks j = g, g + RPI, ...; the LPR
     // lanes of a group each hold 8 columns and are reduced by shuffles.  The
     // loop bound is the same for every lane (the shuffles are warp-wide);
@@ -372,7 +354,8 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   if (c->D != 64 && c->D != 128) return BSA_ERR_UNSUPPORTED;
   if (!(sm_scale == sm_scale) || (g != nullptr && !(g_ref > 0.f)) || !(lambda == lambda))
     return BSA_ERR_INVALID_ARG;
-  if (!aligned16(q_blk) || !aligned16(c->k) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  if (!aligned16(q_blk) || !aligned16(c->k) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (c->kmean != nullptr && !aligned16(c->kmean)))
     return BSA_ERR_INVALID_ARG;
   if (own_first < n_hist || own_first < 0 || own_first + n_own > c->n_blocks ||
       c->n_blocks > c->max_blocks || c->B > 65535 || c->Hh > 65535 || n_own > 65535)
@@ -393,6 +376,7 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   a.block_valid = c->block_valid;
   a.q_valid = q_valid;
   a.g = g;
+  a.kmean = c->kmean;
   a.qm = static_cast<float*>(workspace);
   a.s = reinterpret_cast<float*>(static_cast<char*>(workspace) + qm_b);
   a.idx = idx;
@@ -417,18 +401,20 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   if (c->D == 128) {
     pool_q_kernel<16><<<qgrid, kPoolThreads, 0, s>>>(a);
     if (n_hist > 0) {
-      if (cudaFuncSetAttribute(pool_score_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      auto k = c->kmean != nullptr ? pool_score_kernel<16, true> : pool_score_kernel<16, false>;
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(qm_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      pool_score_kernel<16><<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
+      k<<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
     }
   } else {
     pool_q_kernel<8><<<qgrid, kPoolThreads, 0, s>>>(a);
     if (n_hist > 0) {
-      if (cudaFuncSetAttribute(pool_score_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      auto k = c->kmean != nullptr ? pool_score_kernel<8, true> : pool_score_kernel<8, false>;
+      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(qm_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      pool_score_kernel<8><<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
+      k<<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
     }
   }
   if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

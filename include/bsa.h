@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define BSA_ABI_VERSION 1
+#define BSA_ABI_VERSION 2
 #define BSA_BLOCK 128 /* tokens per KV block = attention tile height */
 
 typedef enum bsa_status {
@@ -79,6 +79,14 @@ typedef enum bsa_status {
  *   n_blocks     blocks in use, [0, max_blocks]; bsa_kv_append writes at
  *                [n_blocks, n_blocks + nb) and then advances it (host side).
  *   D            64 or 128.
+ *   kmean        optional pooled-key cache, device fp32 [B, Hh, max_blocks, D]
+ *                (16-byte aligned), or NULL.  When present, bsa_kv_append
+ *                also writes the mean of the valid key rows of every block it
+ *                appends, and bsa_route reads these means instead of streaming
+ *                the history keys (Velox, Methodology Step 4: block importance
+ *                from mean key vectors; pooling once per block at append time
+ *                gives the same fp32 means as pooling during routing).  Blocks
+ *                written into k directly need bsa_kv_pool_means.
  */
 typedef struct bsa_kv_cache {
   void *k;
@@ -87,6 +95,7 @@ typedef struct bsa_kv_cache {
   int32_t B, Hh, D;
   int32_t max_blocks;
   int32_t n_blocks;
+  float *kmean;
 } bsa_kv_cache;
 
 /* Returns BSA_ABI_VERSION of the loaded library. */
@@ -123,6 +132,17 @@ bsa_status bsa_gilbert_perm(int T, int H, int W, int32_t *host_perm);
 bsa_status bsa_kv_append(bsa_kv_cache *cache, const void *k_tok, const void *v_tok,
                          int T, int H, int W, const int32_t *d_perm,
                          int32_t *d_err, void *stream);
+
+/*
+ * (Re)compute cache->kmean for blocks [first, first + count) of every
+ * (batch, head) from cache->k and cache->block_valid: the mean of each
+ * block's valid key rows in fp32, exactly as bsa_kv_append writes them.  For
+ * blocks the caller wrote into the cache directly.
+ * Errors: BSA_ERR_INVALID_ARG (kmean NULL, range outside [0, max_blocks)),
+ *         BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA; BSA_DEV_BAD_VALID on the device.
+ */
+bsa_status bsa_kv_pool_means(const bsa_kv_cache *cache, int first, int count,
+                             int32_t *d_err, void *stream);
 
 /*
  * The same scatter for a single tensor, e.g. the query chunk before routing:

@@ -37,7 +37,8 @@ class Step:
 
 
 def build_step(w: synth.Workload, device="cuda", chunk: Optional[int] = None,
-               top_k: Optional[int] = None, extra_blocks: int = 0) -> Step:
+               top_k: Optional[int] = None, extra_blocks: int = 0,
+               pooled_keys: bool = False) -> Step:
     """Fill a cache with the workload's history, append the query chunk, and
     lay out Q in block order.  ``chunk`` selects the query chunk of the
     48-chunk sweep (1-based; default: the workload's own history length)."""
@@ -47,13 +48,16 @@ def build_step(w: synth.Workload, device="cuda", chunk: Optional[int] = None,
         chunk = w.hist_chunks + 1
     hist_chunks = chunk - 1 if w.hist_direct == 0 else 0
     n_hist = w.hist_direct + hist_chunks * nbc
-    cache = bsa.KVCache(w.B, w.Hh, w.D, n_hist + nbc + extra_blocks, device=device)
+    cache = bsa.KVCache(w.B, w.Hh, w.D, n_hist + nbc + extra_blocks, device=device,
+                        pooled_keys=pooled_keys)
     if w.hist_direct:
         kd, vd = synth.direct_blocks(w, w.hist_direct, device=device)
         cache.k[:, :, :w.hist_direct] = kd
         cache.v[:, :, :w.hist_direct] = vd
         cache.block_valid[:w.hist_direct] = BLK
         cache.n_blocks = w.hist_direct
+        if pooled_keys:
+            bsa.bsa_kv_pool_means(cache, 0, w.hist_direct)
     for c in range(1, hist_chunks + 1):
         t = synth.chunk_tokens(w, c, device=device, want=("k", "v"))
         bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_abi_version_and_status_strings():
-    assert bsa.abi_version() == 1
+    assert bsa.abi_version() == 2
     for code, name in bsa.STATUS_NAMES.items():
         assert bsa.status_string(code) == name
 

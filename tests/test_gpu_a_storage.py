@@ -120,3 +120,40 @@ def test_bad_permutation_is_reported_not_faulted():
     status, code = bsa.bsa_check_device_error(DEV)
     assert status == 6 and code == 4
     assert bsa.bsa_check_device_error(DEV) == (0, 0)  # cleared
+
+
+@pytest.mark.parametrize("key", [2, 4])
+def test_pooled_key_means_written_at_append(key):
+    # The optional pooled-key cache holds the mean of every block's valid key
+    # rows (Velox, Methodology Step 4: importance from mean key vectors).
+    w = synth.CONFIGS[key]
+    T, H, W = w.grid
+    nb = w.blocks_per_chunk
+    cache = bsa.KVCache(w.B, w.Hh, w.D, 2 * nb, device=DEV, pooled_keys=True)
+    for c in (1, 2):
+        t = synth.chunk_tokens(w, c, device=DEV, want=("k", "v"))
+        bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+    bsa.raise_on_device_error(DEV)
+    valid = cache.block_valid.cpu().numpy()
+    heads = list(range(w.Hh)) if w.Hh <= 12 else [0, 9, w.Hh - 1]
+    exp = oracle.pool_blocks(cache.k[:, heads].cpu().double().numpy(), valid)
+    got = cache.kmean[:, heads].cpu().double().numpy()
+    assert np.allclose(got, exp, rtol=2e-6, atol=2e-7)
+
+
+def test_pool_means_for_directly_written_blocks():
+    w = synth.CONFIGS[3]
+    cache = bsa.KVCache(w.B, w.Hh, w.D, 20, device=DEV, pooled_keys=True)
+    kd, vd = synth.direct_blocks(w, 20, device=DEV)
+    cache.k.copy_(kd)
+    cache.v.copy_(vd)
+    cache.block_valid.fill_(128)
+    cache.block_valid[7] = 33                      # a ragged block
+    cache.n_blocks = 20
+    bsa.bsa_kv_pool_means(cache, 0, 20)
+    bsa.raise_on_device_error(DEV)
+    valid = cache.block_valid.cpu().numpy()
+    exp = oracle.pool_blocks(cache.k[:, [0, 23]].cpu().double().numpy(), valid)
+    assert np.allclose(cache.kmean[:, [0, 23]].cpu().double().numpy(), exp, rtol=2e-6, atol=2e-7)
+    with pytest.raises(bsa.BsaError):
+        bsa.bsa_kv_pool_means(cache, 15, 10)       # past max_blocks

@@ -88,3 +88,32 @@ def test_route_rejects_bad_arguments():
         bsa.bsa_route(step.q_blk, step.cache, step.n_hist + 1, step.own_first, step.n_own,
                       step.top_k)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("key,chunk", [(1, None), (2, None), (3, None), (4, 48)])
+def test_route_from_pooled_keys_is_identical(key, chunk):
+    # Routing from the pooled-key cache (means written at append time) gives
+    # exactly the routes of routing by streaming the history keys: the means
+    # are computed by the same code in the same order.
+    w = synth.CONFIGS[key]
+    a = hx.build_step(w, DEV, chunk=chunk)
+    b = hx.build_step(w, DEV, chunk=chunk, pooled_keys=True)
+    ia, ca = hx.route(a)
+    ib, cb = hx.route(b)
+    bsa.raise_on_device_error(DEV)
+    assert torch.equal(ca, cb)
+    assert torch.equal(ia, ib)
+    # and the no-allocation entry point takes the same path
+    import ctypes
+    idx = torch.full_like(ib, -7)
+    cnt = torch.full_like(cb, -7)
+    cs = b.cache.c_struct()
+    st = bsa.lib().bsa_route_noalloc(
+        ctypes.c_void_p(b.q_blk.data_ptr()), ctypes.byref(cs), ctypes.c_void_p(b.q_valid.data_ptr()),
+        b.n_hist, b.own_first, b.n_own, None if b.g is None else ctypes.c_void_p(b.g.data_ptr()),
+        w.lam, w.g_ref, w.sm_scale, b.top_k, ctypes.c_void_p(idx.data_ptr()),
+        ctypes.c_void_p(cnt.data_ptr()), ib.shape[-1], None,
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    assert torch.equal(idx, ib) and torch.equal(cnt, cb)
