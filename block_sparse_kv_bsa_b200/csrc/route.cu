@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_q_kernel(RouteArgs a) {
 constexpr int kScoreWarps = 8;
 constexpr int kScoreBlocksPerWarp = 8;
 
-template <int VPR, bool kFromMeans>
+template <int VPR>
 __global__ void __launch_bounds__(kScoreWarps * 32)
 pool_score_kernel(RouteArgs a) {
   constexpr int D = VPR * 8;
@@ -154,25 +154,12 @@ pool_score_kernel(RouteArgs a) {
   const int c = lane % LPR;             // 16-byte column chunk of this lane
   const int g = lane / LPR;             // row phase within a load / query-block phase
   const int n_base = (blockIdx.x * kScoreWarps + warp) * kScoreBlocksPerWarp;
-  for (int u = 0; u < kScoreBlocksPerWarp; ++u) {
-    const int n = n_base + u;
-    if (n >= a.n_hist) break;
-    float km[8];
-    if (kFromMeans) {
-      // The block mean was written when the block was appended (same code).
-      const float4* m4 =
-          reinterpret_cast<const float4*>(a.kmean + ((bh * a.max_blocks + n) * D + c * 8));
-      const float4 m0 = m4[0], m1 = m4[1];
-      km[0] = m0.x; km[1] = m0.y; km[2] = m0.z; km[3] = m0.w;
-      km[4] = m1.x; km[5] = m1.y; km[6] = m1.z; km[7] = m1.w;
-    } else {
-      const int valid = clamp_valid(a.block_valid[n], a.d_err);
-      warp_block_mean<VPR>(a.kc + (bh * a.max_blocks + n) * kBlk * VPR, valid, c, g, km);
-    }
-    // Scores: lane group g takes query blocks j = g, g + RPI, ...; the LPR
-    // lanes of a group each hold 8 columns and are reduced by shuffles.  The
-    // loop bound is the same for every lane (the shuffles are warp-wide);
-    // out-of-range query blocks only skip their arithmetic.
+  // Score one block mean (this lane's 8 columns in km) against every query
+  // mean: lane group g takes query blocks j = g, g + RPI, ...; the LPR lanes
+  // of a group are reduced by shuffles.  The loop bound is the same for every
+  // lane (the shuffles are warp-wide); out-of-range query blocks only skip
+  // their arithmetic.
+  auto score_block = [&](int n, const float (&km)[8]) {
     for (int jb = 0; jb < a.n_own; jb += 4 * RPI) {
       const int j0 = jb + g;
       float d[4];
@@ -200,6 +187,91 @@ pool_score_kernel(RouteArgs a) {
         for (int t = 1; t < 4; ++t) dv = c == t ? d[t] : dv;
         const int j = j0 + c * RPI;
         if (j < a.n_own) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * dv;
+      }
+    }
+  };
+  {
+    for (int u = 0; u < kScoreBlocksPerWarp; ++u) {
+      const int n = n_base + u;
+      if (n >= a.n_hist) break;
+      const int valid = clamp_valid(a.block_valid[n], a.d_err);
+      float km[8];
+      warp_block_mean<VPR>(a.kc + (bh * a.max_blocks + n) * kBlk * VPR, valid, c, g, km);
+      score_block(n, km);
+    }
+  }
+}
+
+// Scores from the pooled-key cache: s[j, n] = sm_scale * <qmean_j, kmean_n>
+// for all query blocks j of a head and a tile of 64 history blocks, as a
+// register-blocked CUDA-core product (the whole step is ~0.7 GFLOP at chunk
+// 48, far too small for the tensor cores to matter).  Both operands go to
+// shared memory with a 4-float row pad; each thread owns 4 query blocks x 4
+// history blocks and accumulates over D in order, 4 dimensions per step.
+constexpr int kMeanTileN = 64;
+constexpr int kMeanThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kMeanThreads)
+score_means_kernel(RouteArgs a) {
+  constexpr int P = D + 4;                       // padded row (floats)
+  extern __shared__ float sm[];
+  const int nq = (a.n_own + 15) & ~15;           // query rows, rounded up to 16
+  float* qs = sm;                                // [nq][P]
+  float* ks = qs + nq * P;                       // [64][P]
+  const int h = blockIdx.y, b = blockIdx.z;
+  const long long bh = static_cast<long long>(b) * a.Hh + h;
+  const int n0 = blockIdx.x * kMeanTileN;
+  for (int i = threadIdx.x; i < nq * (D / 4); i += kMeanThreads) {
+    const int r = i / (D / 4), c4 = i % (D / 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < a.n_own) v = reinterpret_cast<const float4*>(a.qm + (bh * a.n_own + r) * D)[c4];
+    *reinterpret_cast<float4*>(qs + r * P + c4 * 4) = v;
+  }
+  for (int i = threadIdx.x; i < kMeanTileN * (D / 4); i += kMeanThreads) {
+    const int r = i / (D / 4), c4 = i % (D / 4);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (n0 + r < a.n_hist)
+      v = reinterpret_cast<const float4*>(a.kmean + (bh * a.max_blocks + n0 + r) * D)[c4];
+    *reinterpret_cast<float4*>(ks + r * P + c4 * 4) = v;
+  }
+  __syncthreads();
+  const int tn = threadIdx.x % 16;               // history blocks tn*4 .. tn*4+3 of the tile
+  const int tj = threadIdx.x / 16;               // query blocks tj, tj+16, tj+32, ...
+  for (int jb = 0; jb < nq; jb += 64) {
+    float acc[4][4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
+#pragma unroll 4
+    for (int d = 0; d < D; d += 4) {
+      float4 q[4], k[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int j = jb + tj + 16 * x;
+        q[x] = j < nq ? *reinterpret_cast<const float4*>(qs + j * P + d) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int y = 0; y < 4; ++y) k[y] = *reinterpret_cast<const float4*>(ks + (tn * 4 + y) * P + d);
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          acc[x][y] = fmaf(q[x].x, k[y].x, acc[x][y]);
+          acc[x][y] = fmaf(q[x].y, k[y].y, acc[x][y]);
+          acc[x][y] = fmaf(q[x].z, k[y].z, acc[x][y]);
+          acc[x][y] = fmaf(q[x].w, k[y].w, acc[x][y]);
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int j = jb + tj + 16 * x;
+      if (j >= a.n_own) continue;
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        const int n = n0 + tn * 4 + y;
+        if (n < a.n_hist) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * acc[x][y];
       }
     }
   }
@@ -265,6 +337,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(RouteArgs a) {
     for (int n = threadIdx.x; n < a.n_hist; n += kTopkThreads) out[n] = n;
   } else if (K > 0) {
     if (staged) {
+#pragma unroll 4
       for (int n = threadIdx.x; n < a.n_hist; n += kTopkThreads)
         keys[n] = score_key(fused_score(a, sr, gr, n));
       __syncthreads();
@@ -279,15 +352,34 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(RouteArgs a) {
         if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
       }
       __syncthreads();
-      if (threadIdx.x == 0) {
-        int above = 0;
-        int d = 255;
-        for (; d > 0; --d) {
-          if (above + hist[d] >= remaining) break;
-          above += hist[d];
+      if (threadIdx.x < 32) {
+        // Lane l holds bins 255 - 8l .. 248 - 8l (highest first); a suffix
+        // count over lanes finds the bin that holds the remaining-th key.
+        const int l = threadIdx.x;
+        int cnts[8], tot = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          cnts[q] = hist[255 - (8 * l + q)];
+          tot += cnts[q];
         }
-        s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
-        s_remaining = remaining - above;
+        int incl = tot;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, off);
+          if (l >= off) incl += t;
+        }
+        const int excl = incl - tot;
+        if (excl < remaining && remaining <= incl) {
+          int above = excl, d = 255 - 8 * l;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            d = 255 - (8 * l + q);
+            if (above + cnts[q] >= remaining) break;
+            above += cnts[q];
+          }
+          s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
+          s_remaining = remaining - above;
+        }
       }
       __syncthreads();
       prefix = s_prefix;
@@ -398,23 +490,35 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   dim3 qgrid(n_own, c->Hh, c->B);
   const int per_cta = kScoreWarps * kScoreBlocksPerWarp;
   dim3 sgrid((n_hist + per_cta - 1) / per_cta, c->Hh, c->B);
+  const int nq16 = (n_own + 15) & ~15;
+  const size_t mean_smem = sizeof(float) * static_cast<size_t>(nq16 + kMeanTileN) * (c->D + 4);
+  dim3 mgrid((n_hist + kMeanTileN - 1) / kMeanTileN, c->Hh, c->B);
+  if (c->kmean != nullptr && mean_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
   if (c->D == 128) {
     pool_q_kernel<16><<<qgrid, kPoolThreads, 0, s>>>(a);
-    if (n_hist > 0) {
-      auto k = c->kmean != nullptr ? pool_score_kernel<16, true> : pool_score_kernel<16, false>;
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (n_hist > 0 && c->kmean != nullptr) {
+      if (cudaFuncSetAttribute(score_means_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(mean_smem)) != cudaSuccess)
+        return BSA_ERR_CUDA;
+      score_means_kernel<128><<<mgrid, kMeanThreads, mean_smem, s>>>(a);
+    } else if (n_hist > 0) {
+      if (cudaFuncSetAttribute(pool_score_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(qm_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      k<<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
+      pool_score_kernel<16><<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
     }
   } else {
     pool_q_kernel<8><<<qgrid, kPoolThreads, 0, s>>>(a);
-    if (n_hist > 0) {
-      auto k = c->kmean != nullptr ? pool_score_kernel<8, true> : pool_score_kernel<8, false>;
-      if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (n_hist > 0 && c->kmean != nullptr) {
+      if (cudaFuncSetAttribute(score_means_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(mean_smem)) != cudaSuccess)
+        return BSA_ERR_CUDA;
+      score_means_kernel<64><<<mgrid, kMeanThreads, mean_smem, s>>>(a);
+    } else if (n_hist > 0) {
+      if (cudaFuncSetAttribute(pool_score_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(qm_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      k<<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
+      pool_score_kernel<8><<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
     }
   }
   if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -91,19 +91,16 @@ def test_route_rejects_bad_arguments():
 
 
 @pytest.mark.parametrize("key,chunk", [(1, None), (2, None), (3, None), (4, 48)])
-def test_route_from_pooled_keys_is_identical(key, chunk):
-    # Routing from the pooled-key cache (means written at append time) gives
-    # exactly the routes of routing by streaming the history keys: the means
-    # are computed by the same code in the same order.
+def test_route_from_pooled_keys(key, chunk):
+    # Routing from the pooled-key cache (block key means written at append
+    # time, scored by a small product kernel) against the oracle, with the
+    # same near-tie rule as the streaming route; its fp32 sums run in another
+    # order than the streaming route's, so the two may differ only at
+    # near-ties.
     w = synth.CONFIGS[key]
-    a = hx.build_step(w, DEV, chunk=chunk)
     b = hx.build_step(w, DEV, chunk=chunk, pooled_keys=True)
-    ia, ca = hx.route(a)
-    ib, cb = hx.route(b)
-    bsa.raise_on_device_error(DEV)
-    assert torch.equal(ca, cb)
-    assert torch.equal(ia, ib)
-    # and the no-allocation entry point takes the same path
+    ib, cb = _check(b, heads=[5] if key == 4 else None)
+    # The no-allocation entry point takes the same path, bit for bit.
     import ctypes
     idx = torch.full_like(ib, -7)
     cnt = torch.full_like(cb, -7)
