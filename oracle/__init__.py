@@ -25,4 +25,7 @@ from .bsa import (  # noqa: F401
     route,
     tokens_to_blocks,
     top_k_with_own,
+    velox_route,
+    velox_route_row,
+    vetted_overlap,
 )

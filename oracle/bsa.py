@@ -291,3 +291,91 @@ def dense_masked_attn(q_rows, keys_all, vals_all, allowed: np.ndarray, sm_scale:
         o[r] = (e @ v) / e.sum()
         lse[r] = m + np.log(e.sum())
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# The page's full route (Methodology Steps 4-5)
+# ---------------------------------------------------------------------------
+
+def vetted_overlap(g: np.ndarray, tau: float, g_ref: float) -> np.ndarray:
+    """g_hat: overlap above the noise threshold tau, rescaled by g_ref and
+    clipped to 1; overlap at or below tau counts as none."""
+    g = _f64(g)
+    return np.where(g > tau, np.minimum(g / g_ref, 1.0), 0.0)
+
+
+def velox_route_row(s_row: np.ndarray, g_row: Optional[np.ndarray], covered: bool,
+                    j: int, lam: float, g_ref: float, tau: float, k_cov: int, k_unc: int,
+                    mass: float, prev_first: int, n_prev: int, window_half: int,
+                    ref_first: int, n_ref: int, own_first: int, n_own: int) -> np.ndarray:
+    """Route of one query block j over history blocks [0, len(s_row)).
+
+    Covered query block: the importance distribution softmax(s) is multiplied
+    by (1 + lam * g_hat) and renormalised, which ranks blocks exactly like
+    s + log(1 + lam * g_hat); the previous chunk's blocks are reserved first,
+    then the best remaining blocks fill the budget up to k_cov in total.
+    Uncovered query block: the unfused distribution softmax(s) is taken in
+    decreasing order (ties to the lower index) up to the smallest prefix whose
+    mass reaches `mass`, at most k_unc blocks.
+    Both are joined with the window of previous-chunk blocks at Gilbert
+    positions j - window_half .. j + window_half, the reference blocks and the
+    query block's own chunk; the result is sorted ascending without repeats.
+    """
+    n_hist = s_row.shape[0]
+    chosen = set()
+    prev = [prev_first + p for p in range(n_prev) if 0 <= prev_first + p < n_hist]
+    if covered:
+        f = s_row.copy()
+        if g_row is not None:
+            f = f + np.log1p(lam * vetted_overlap(g_row, tau, g_ref))
+        reserved = set(prev)
+        chosen |= reserved
+        budget = max(k_cov - len(reserved), 0)
+        rest = sorted((n for n in range(n_hist) if n not in reserved), key=lambda n: (-f[n], n))
+        chosen |= set(rest[:budget])
+    elif n_hist > 0:
+        m = s_row.max()
+        p = np.exp(s_row - m)
+        p = p / p.sum()
+        order = sorted(range(n_hist), key=lambda n: (-s_row[n], n))
+        acc = 0.0
+        for r, n in enumerate(order[:k_unc]):
+            chosen.add(n)
+            acc += p[n]
+            if acc >= mass:
+                break
+    for pos in range(j - window_half, j + window_half + 1):
+        if 0 <= pos < n_prev and 0 <= prev_first + pos < n_hist:
+            chosen.add(prev_first + pos)
+    for r in range(n_ref):
+        if 0 <= ref_first + r < n_hist:
+            chosen.add(ref_first + r)
+    return np.array(sorted(chosen) + list(range(own_first, own_first + n_own)), dtype=np.int64)
+
+
+def velox_route(q_blk, k_cache, valid, n_hist: int, own_first: int, n_own: int, g,
+                coverage, lam: float, g_ref: float, sm_scale: float, tau: float,
+                eta_cov: float, k_cov: int, k_unc: int, mass: float, prev_first: int,
+                n_prev: int, window_half: int, ref_first: int = 0, n_ref: int = 0,
+                q_valid: Optional[Sequence[int]] = None):
+    """The page's route for every (b, h, query block); returns (idx lists, model scores).
+
+    ``coverage`` is [B, n_own] (fraction of a query block's tokens inside a
+    valid historical slab) or None (no query block is covered).
+    """
+    q = _f64(q_blk)
+    B, Hh, nq_rows, D = q.shape
+    if q_valid is None:
+        q_valid = [int(valid[own_first + j]) for j in range(n_own)]
+    q_mean = pool_blocks(q.reshape(B, Hh, n_own, BLK, D), q_valid)
+    kc = _f64(k_cache)[:, :, :n_hist]
+    k_mean = pool_blocks(kc, valid[:n_hist]) if n_hist > 0 else np.zeros((B, Hh, 0, D))
+    s = block_scores(q_mean, k_mean, sm_scale)
+    g = None if g is None else _f64(g)
+    cov = None if coverage is None else _f64(coverage)
+    idx = [[[velox_route_row(s[b, h, j], None if g is None else g[b, j],
+                             cov is not None and cov[b, j] >= eta_cov, j, lam, g_ref, tau,
+                             k_cov, k_unc, mass, prev_first, n_prev, window_half, ref_first,
+                             n_ref, own_first, n_own)
+             for j in range(n_own)] for h in range(Hh)] for b in range(B)]
+    return idx, s
