@@ -45,7 +45,8 @@ DEV_CODES = {0: "BSA_DEV_OK", 1: "BSA_DEV_BAD_INDEX", 2: "BSA_DEV_BAD_COUNT",
 EXPORTS = ("bsa_abi_version", "bsa_status_string", "bsa_gilbert_perm", "bsa_kv_append",
            "bsa_kv_pool_means",
            "bsa_tokens_to_blocks", "bsa_blocks_to_tokens", "bsa_route_workspace_size",
-           "bsa_route", "bsa_route_noalloc", "bsa_attn", "bsa_check_device_error",
+           "bsa_route", "bsa_route_velox", "bsa_route_noalloc", "bsa_attn",
+           "bsa_check_device_error",
            "bsa_selftest_bounded_wait")
 
 
@@ -75,6 +76,15 @@ class CCache(ctypes.Structure):
                 ("kmean", ctypes.c_void_p)]
 
 
+class CVeloxRoute(ctypes.Structure):
+    """ctypes mirror of ``bsa_velox_route``."""
+    _fields_ = [("coverage", ctypes.c_void_p), ("eta_cov", ctypes.c_float),
+                ("tau", ctypes.c_float), ("k_cov", ctypes.c_int32), ("k_unc", ctypes.c_int32),
+                ("mass", ctypes.c_float), ("prev_first", ctypes.c_int32),
+                ("n_prev", ctypes.c_int32), ("window_half", ctypes.c_int32),
+                ("ref_first", ctypes.c_int32), ("n_ref", ctypes.c_int32)]
+
+
 _i, _p, _f, _sz = ctypes.c_int, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
 _sig = {
     "bsa_abi_version": (ctypes.c_int, []),
@@ -87,6 +97,8 @@ _sig = {
     "bsa_route_workspace_size": (_i, [_i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "bsa_route": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f, _i,
                        _p, _p, _i, _p, _sz, _p, _p]),
+    "bsa_route_velox": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f,
+                             ctypes.POINTER(CVeloxRoute), _p, _p, _i, _p, _sz, _p, _p]),
     "bsa_route_noalloc": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f, _i,
                                _p, _p, _i, _p, _p]),
     "bsa_attn": (_i, [_p, ctypes.POINTER(CCache), _p, _p, _p, _i, _i, _f, _p, _p, _p, _p]),
@@ -336,6 +348,57 @@ def bsa_route(q_blk: torch.Tensor, cache: KVCache, n_hist: int, own_first: int, 
         _ptr(q_blk), ctypes.byref(cs), _ptr(q_valid), int(n_hist), int(own_first), int(n_own),
         _ptr(g), float(lam), float(g_ref), float(sm_scale), int(top_k), _ptr(idx), _ptr(cnt),
         int(max_sel), _ptr(workspace), workspace.numel(), _ptr(error_word(dev)), _stream(dev)))
+    return idx, cnt
+
+
+def velox_max_sel(n_hist: int, n_own: int, k_cov: int = 80, k_unc: int = 150, n_prev: int = 0,
+                  window_half: int = 13, n_ref: int = 0) -> int:
+    """Smallest max_sel bsa_route_velox accepts."""
+    budget = max(k_cov, n_prev, k_unc)
+    return min(n_hist, budget + 2 * window_half + 1 + n_ref) + n_own
+
+
+def bsa_route_velox(q_blk: torch.Tensor, cache: KVCache, n_hist: int, own_first: int,
+                    n_own: int, g: Optional[torch.Tensor] = None,
+                    coverage: Optional[torch.Tensor] = None, lam: float = 2.0,
+                    g_ref: float = 0.2, sm_scale: Optional[float] = None, tau: float = 0.1,
+                    eta_cov: float = 0.9, k_cov: int = 80, k_unc: int = 150, mass: float = 0.9,
+                    prev_first: int = 0, n_prev: int = 0, window_half: int = 13,
+                    ref_first: int = 0, n_ref: int = 0, q_valid: Optional[torch.Tensor] = None,
+                    max_sel: Optional[int] = None, idx: Optional[torch.Tensor] = None,
+                    cnt: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The page's full route; returns (idx [B,Hh,n_own,max_sel] padded with -1, cnt)."""
+    dev = cache.device
+    _need(q_blk, "q_blk", torch.bfloat16, dev, (cache.B, cache.Hh, n_own * BLK, cache.D))
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(cache.D)
+    if max_sel is None:
+        max_sel = velox_max_sel(n_hist, n_own, k_cov, k_unc, n_prev, window_half, n_ref)
+    if idx is None:
+        idx = torch.empty((cache.B, cache.Hh, n_own, max_sel), dtype=torch.int32, device=dev)
+    if cnt is None:
+        cnt = torch.empty((cache.B, cache.Hh, n_own), dtype=torch.int32, device=dev)
+    _need(idx, "idx", torch.int32, dev, (cache.B, cache.Hh, n_own, max_sel))
+    _need(cnt, "cnt", torch.int32, dev, (cache.B, cache.Hh, n_own))
+    if g is not None:
+        _need(g, "g", torch.float32, dev, (cache.B, n_own, n_hist))
+    if coverage is not None:
+        _need(coverage, "coverage", torch.float32, dev, (cache.B, n_own))
+    if q_valid is not None:
+        _need(q_valid, "q_valid", torch.int32, dev, (n_own,))
+    ws_bytes = bsa_route_workspace_size(cache.B, cache.Hh, cache.D, n_own, n_hist)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    opts = CVeloxRoute(None if coverage is None else coverage.data_ptr(), float(eta_cov),
+                       float(tau), int(k_cov), int(k_unc), float(mass), int(prev_first),
+                       int(n_prev), int(window_half), int(ref_first), int(n_ref))
+    cs = cache.c_struct()
+    _check("bsa_route_velox", _lib.bsa_route_velox(
+        _ptr(q_blk), ctypes.byref(cs), _ptr(q_valid), int(n_hist), int(own_first), int(n_own),
+        _ptr(g), float(lam), float(g_ref), float(sm_scale), ctypes.byref(opts), _ptr(idx),
+        _ptr(cnt), int(max_sel), _ptr(workspace), workspace.numel(), _ptr(error_word(dev)),
+        _stream(dev)))
     return idx, cnt
 
 

@@ -19,6 +19,7 @@
 //                  index order by a block-wide ordered compaction, followed by
 //                  the own-chunk blocks.
 // All sums run in fp32 in a fixed order, so results are deterministic.
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -409,6 +410,238 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(RouteArgs a) {
   if (threadIdx.x == 0) a.cnt[row] = K + a.n_own;
 }
 
+// ---------------------------------------------------------------------------
+// The page's full route (Methodology Steps 4-5): coverage split, tau-gated
+// multiplicative fusion, previous-chunk reservation, mass prefix, window.
+// ---------------------------------------------------------------------------
+constexpr int kVeloxMaxHist = 32768;   // keys + flags staged in shared memory
+constexpr int kVeloxSortMax = 1024;    // largest uncovered budget (K_unc)
+
+struct VeloxArgs {
+  const float* coverage;  // [B, n_own] or null
+  float eta_cov, tau, mass;
+  int k_cov, k_unc, prev_first, n_prev, window_half, ref_first, n_ref;
+};
+
+// Radix select over keys[0..n) staged in shared memory: after it, keys above
+// *thr are taken, plus the *need_eq lowest-index keys equal to *thr (K total).
+__device__ void radix_threshold(const uint32_t* keys, int n, int K, int* hist, uint32_t* s_prefix,
+                                int* s_remaining, uint32_t* thr, int* need_eq) {
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = K;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t k = keys[i];
+      if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      const int l = threadIdx.x;
+      int cnts[8], tot = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        cnts[q] = hist[255 - (8 * l + q)];
+        tot += cnts[q];
+      }
+      int incl = tot;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (l >= off) incl += t;
+      }
+      const int excl = incl - tot;
+      if (excl < remaining && remaining <= incl) {
+        int above = excl, d = 255 - 8 * l;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          d = 255 - (8 * l + q);
+          if (above + cnts[q] >= remaining) break;
+          above += cnts[q];
+        }
+        *s_prefix = prefix | (static_cast<uint32_t>(d) << shift);
+        *s_remaining = remaining - above;
+      }
+    }
+    __syncthreads();
+    prefix = *s_prefix;
+    remaining = *s_remaining;
+    pmask |= 255u << shift;
+    __syncthreads();
+  }
+  *thr = prefix;
+  *need_eq = remaining;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a, VeloxArgs v) {
+  extern __shared__ __align__(16) uint8_t vsm[];
+  const int nh = a.n_hist;
+  uint64_t* sortbuf = reinterpret_cast<uint64_t*>(vsm);                 // [kVeloxSortMax]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sortbuf + kVeloxSortMax); // [nh]
+  uint8_t* flag = reinterpret_cast<uint8_t*>(keys + nh);                // [nh]
+  __shared__ int hist[256];
+  __shared__ int warp_tot[kTopkThreads / 32];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_remaining, s_m;
+  __shared__ float red[kTopkThreads];
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const long long row = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
+  int32_t* out = a.idx + row * a.max_sel;
+  const float* sr = a.s + row * nh;
+  const float* gr = a.g != nullptr ? a.g + (static_cast<long long>(b) * a.n_own + j) * nh : nullptr;
+  const bool covered = v.coverage != nullptr && v.coverage[b * a.n_own + j] >= v.eta_cov;
+  const int p0 = min(max(v.prev_first, 0), nh);
+  const int p1 = min(max(v.prev_first + v.n_prev, p0), nh);
+
+  if (covered) {
+    // s + log(1 + lam * g_hat) ranks like the renormalised product of the
+    // importance distribution and 1 + lam * g_hat; the previous chunk is
+    // reserved (key 0 keeps it out of the selection).
+    for (int n = threadIdx.x; n < nh; n += kTopkThreads) {
+      const bool res = n >= p0 && n < p1;
+      float f = sr[n];
+      if (gr != nullptr) {
+        const float gv = gr[n];
+        const float gh = gv > v.tau ? fminf(gv / a.g_ref, 1.0f) : 0.0f;
+        f += log1pf(a.lam * gh);
+      }
+      keys[n] = res ? 0u : score_key(f);
+      flag[n] = res ? 1 : 0;
+    }
+    __syncthreads();
+    const int n_res = p1 - p0;
+    const int K = max(0, min(v.k_cov - n_res, nh - n_res));
+    if (K > 0) {
+      uint32_t thr;
+      int need_eq;
+      radix_threshold(keys, nh, K, hist, &s_prefix, &s_remaining, &thr, &need_eq);
+      int eq_seen = 0;
+      for (int base = 0; base < nh; base += kTopkThreads) {
+        const int n = base + threadIdx.x;
+        const uint32_t k = n < nh ? keys[n] : 0u;
+        const bool eq = n < nh && k == thr && k != 0u;
+        int eq_tot;
+        const int eq_rank = eq_seen + block_excl_count(eq, warp_tot, &eq_tot);
+        if (n < nh && k != 0u && (k > thr || (eq && eq_rank < need_eq))) flag[n] = 1;
+        eq_seen += eq_tot;
+      }
+    }
+  } else {
+    for (int n = threadIdx.x; n < nh; n += kTopkThreads) {
+      keys[n] = score_key(sr[n]);
+      flag[n] = 0;
+    }
+    __syncthreads();
+    const int K = min(v.k_unc, nh);
+    if (K > 0) {
+      // Row maximum and normaliser of softmax(s), in a fixed order.
+      float mx = -INFINITY;
+      for (int n = threadIdx.x; n < nh; n += kTopkThreads) mx = fmaxf(mx, sr[n]);
+      red[threadIdx.x] = mx;
+      __syncthreads();
+      for (int w = kTopkThreads / 2; w > 0; w >>= 1) {
+        if (threadIdx.x < w) red[threadIdx.x] = fmaxf(red[threadIdx.x], red[threadIdx.x + w]);
+        __syncthreads();
+      }
+      const float smax = red[0];
+      __syncthreads();
+      float z = 0.f;
+      for (int n = threadIdx.x; n < nh; n += kTopkThreads) z += expf(sr[n] - smax);
+      red[threadIdx.x] = z;
+      __syncthreads();
+      for (int w = kTopkThreads / 2; w > 0; w >>= 1) {
+        if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+        __syncthreads();
+      }
+      const float zsum = red[0];
+      // The K best blocks, listed in index order, then sorted by (score
+      // descending, index ascending) so the mass prefix can be walked.
+      uint32_t thr;
+      int need_eq;
+      radix_threshold(keys, nh, K, hist, &s_prefix, &s_remaining, &thr, &need_eq);
+      int pos = 0, eq_seen = 0;
+      for (int base = 0; base < nh; base += kTopkThreads) {
+        const int n = base + threadIdx.x;
+        const uint32_t k = n < nh ? keys[n] : 0u;
+        const bool gt = n < nh && k > thr;
+        const bool eq = n < nh && k == thr;
+        int eq_tot, sel_tot;
+        const int eq_rank = eq_seen + block_excl_count(eq, warp_tot, &eq_tot);
+        const bool sel = gt || (eq && eq_rank < need_eq);
+        const int at = pos + block_excl_count(sel, warp_tot, &sel_tot);
+        // ascending order of ~((key << 32) | ~n) = descending key, ascending n
+        if (sel) sortbuf[at] = ~((static_cast<uint64_t>(k) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(n)));
+        pos += sel_tot;
+        eq_seen += eq_tot;
+      }
+      int P = 2;
+      while (P < K) P <<= 1;
+      for (int i = K + threadIdx.x; i < P; i += kTopkThreads) sortbuf[i] = ~0ull;
+      __syncthreads();
+      for (int kk = 2; kk <= P; kk <<= 1) {
+        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+          for (int i = threadIdx.x; i < P; i += kTopkThreads) {
+            const int ixj = i ^ jj;
+            if (ixj > i) {
+              const uint64_t x = sortbuf[i], y = sortbuf[ixj];
+              const bool up = (i & kk) == 0;
+              if (up ? (x > y) : (x < y)) {
+                sortbuf[i] = y;
+                sortbuf[ixj] = x;
+              }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      if (threadIdx.x == 0) {
+        float acc = 0.f;
+        int m = K;
+        for (int r = 0; r < K; ++r) {
+          const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]));
+          acc += expf(sr[n] - smax) / zsum;
+          if (acc >= v.mass) {
+            m = r + 1;
+            break;
+          }
+        }
+        s_m = m;
+      }
+      __syncthreads();
+      for (int r = threadIdx.x; r < s_m; r += kTopkThreads)
+        flag[static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]))] = 1;
+    }
+  }
+  __syncthreads();
+  // Window of previous-chunk blocks around this query block's position, and
+  // the reference blocks, outside the budget.
+  for (int pos = j - v.window_half + static_cast<int>(threadIdx.x); pos <= j + v.window_half;
+       pos += kTopkThreads) {
+    const int n = v.prev_first + pos;
+    if (pos >= 0 && pos < v.n_prev && n >= 0 && n < nh) flag[n] = 1;
+  }
+  for (int r = threadIdx.x; r < v.n_ref; r += kTopkThreads) {
+    const int n = v.ref_first + r;
+    if (n >= 0 && n < nh) flag[n] = 1;
+  }
+  __syncthreads();
+  int pos = 0;
+  for (int base = 0; base < nh; base += kTopkThreads) {
+    const int n = base + threadIdx.x;
+    const bool sel = n < nh && flag[n];
+    int tot;
+    const int at = pos + block_excl_count(sel, warp_tot, &tot);
+    if (sel && at < a.max_sel) out[at] = n;
+    pos += tot;
+  }
+  const int c = min(pos, a.max_sel - a.n_own);
+  if (pos + a.n_own > a.max_sel && threadIdx.x == 0) report(a.d_err, BSA_DEV_BAD_COUNT);
+  for (int i = threadIdx.x; i < a.n_own; i += kTopkThreads) out[c + i] = a.own_first + i;
+  for (int i = c + a.n_own + threadIdx.x; i < a.max_sel; i += kTopkThreads) out[i] = -1;
+  if (threadIdx.x == 0) a.cnt[row] = c + a.n_own;
+}
+
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 static void route_ws_layout(int B, int Hh, int D, int n_own, int n_hist, size_t* qm_bytes,
@@ -433,15 +666,20 @@ extern "C" bsa_status bsa_route_workspace_size(int B, int Hh, int D, int n_q_blo
   return BSA_OK;
 }
 
-extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
-                                int n_hist, int own_first, int n_own, const float* g,
-                                float lambda, float g_ref, float sm_scale, int top_k, int32_t* idx,
-                                int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
-                                int32_t* d_err, void* stream) {
+namespace bsa {
+
+// Validation shared by both routes, the query means and the model scores
+// (from the pooled-key cache or by streaming the history keys).  Fills `a`
+// for the selection kernel the caller launches next.
+static bsa_status route_scores(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
+                               int n_hist, int own_first, int n_own, const float* g,
+                               float lambda, float g_ref, float sm_scale, int32_t* idx,
+                               int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
+                               int32_t* d_err, cudaStream_t s, RouteArgs* out) {
   if (q_blk == nullptr || c == nullptr || idx == nullptr || cnt == nullptr ||
       workspace == nullptr || c->k == nullptr || c->block_valid == nullptr)
     return BSA_ERR_INVALID_ARG;
-  if (c->B <= 0 || c->Hh <= 0 || n_own <= 0 || n_hist < 0 || top_k < 0 || max_sel <= 0)
+  if (c->B <= 0 || c->Hh <= 0 || n_own <= 0 || n_hist < 0 || max_sel <= 0)
     return BSA_ERR_INVALID_ARG;
   if (c->D != 64 && c->D != 128) return BSA_ERR_UNSUPPORTED;
   if (!(sm_scale == sm_scale) || (g != nullptr && !(g_ref > 0.f)) || !(lambda == lambda))
@@ -452,17 +690,17 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   if (own_first < n_hist || own_first < 0 || own_first + n_own > c->n_blocks ||
       c->n_blocks > c->max_blocks || c->B > 65535 || c->Hh > 65535 || n_own > 65535)
     return BSA_ERR_SHAPE;
-  const int K = top_k < n_hist ? top_k : n_hist;
-  if (max_sel < K + n_own) return BSA_ERR_CAPACITY;
   size_t qm_b, s_b;
   route_ws_layout(c->B, c->Hh, c->D, n_own, n_hist, &qm_b, &s_b);
   if (ws_bytes < qm_b + s_b) return BSA_ERR_CAPACITY;
   const size_t qm_smem = sizeof(float) * static_cast<size_t>(n_own) * c->D;
   if (qm_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
-  const size_t topk_smem =
-      n_hist <= kTopkSmemKeys ? sizeof(uint32_t) * static_cast<size_t>(n_hist > 0 ? n_hist : 1) : 0;
+  const int nq16 = (n_own + 15) & ~15;
+  const size_t mean_smem = sizeof(float) * static_cast<size_t>(nq16 + kMeanTileN) * (c->D + 4);
+  if (c->kmean != nullptr && mean_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
 
-  RouteArgs a{};
+  RouteArgs& a = *out;
+  a = RouteArgs{};
   a.q = static_cast<const uint4*>(q_blk);
   a.kc = static_cast<const uint4*>(c->k);
   a.block_valid = c->block_valid;
@@ -480,20 +718,15 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   a.n_hist = n_hist;
   a.own_first = own_first;
   a.max_blocks = c->max_blocks;
-  a.top_k = top_k;
   a.max_sel = max_sel;
   a.sm_scale = sm_scale;
   a.lam = lambda;
   a.g_ref = g_ref;
 
-  cudaStream_t s = as_stream(stream);
   dim3 qgrid(n_own, c->Hh, c->B);
   const int per_cta = kScoreWarps * kScoreBlocksPerWarp;
   dim3 sgrid((n_hist + per_cta - 1) / per_cta, c->Hh, c->B);
-  const int nq16 = (n_own + 15) & ~15;
-  const size_t mean_smem = sizeof(float) * static_cast<size_t>(nq16 + kMeanTileN) * (c->D + 4);
   dim3 mgrid((n_hist + kMeanTileN - 1) / kMeanTileN, c->Hh, c->B);
-  if (c->kmean != nullptr && mean_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
   if (c->D == 128) {
     pool_q_kernel<16><<<qgrid, kPoolThreads, 0, s>>>(a);
     if (n_hist > 0 && c->kmean != nullptr) {
@@ -521,10 +754,71 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
       pool_score_kernel<8><<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
     }
   }
+  return launch_status();
+}
+
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
+                                int n_hist, int own_first, int n_own, const float* g,
+                                float lambda, float g_ref, float sm_scale, int top_k, int32_t* idx,
+                                int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
+                                int32_t* d_err, void* stream) {
+  if (top_k < 0) return BSA_ERR_INVALID_ARG;
+  const int K = top_k < n_hist ? top_k : n_hist;
+  if (n_hist >= 0 && n_own > 0 && max_sel > 0 && max_sel < K + n_own) return BSA_ERR_CAPACITY;
+  cudaStream_t s = as_stream(stream);
+  RouteArgs a;
+  bsa_status st = route_scores(q_blk, c, q_valid, n_hist, own_first, n_own, g, lambda, g_ref,
+                               sm_scale, idx, cnt, max_sel, workspace, ws_bytes, d_err, s, &a);
+  if (st != BSA_OK) return st;
+  a.top_k = top_k;
+  const size_t topk_smem =
+      n_hist <= kTopkSmemKeys ? sizeof(uint32_t) * static_cast<size_t>(n_hist > 0 ? n_hist : 1) : 0;
   if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(topk_smem)) != cudaSuccess)
     return BSA_ERR_CUDA;
+  dim3 qgrid(n_own, c->Hh, c->B);
   topk_kernel<<<qgrid, kTopkThreads, topk_smem, s>>>(a);
+  return launch_status();
+}
+
+extern "C" bsa_status bsa_route_velox(const void* q_blk, const bsa_kv_cache* c,
+                                      const int32_t* q_valid, int n_hist, int own_first,
+                                      int n_own, const float* g, float lambda, float g_ref,
+                                      float sm_scale, const bsa_velox_route* opts, int32_t* idx,
+                                      int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
+                                      int32_t* d_err, void* stream) {
+  if (opts == nullptr) return BSA_ERR_INVALID_ARG;
+  const bsa_velox_route& o = *opts;
+  if (o.k_cov < 0 || o.k_unc < 0 || o.n_prev < 0 || o.window_half < 0 || o.n_ref < 0 ||
+      !(o.mass == o.mass) || !(o.tau == o.tau) || !(o.eta_cov == o.eta_cov))
+    return BSA_ERR_INVALID_ARG;
+  if (o.k_unc > kVeloxSortMax || n_hist > kVeloxMaxHist) return BSA_ERR_UNSUPPORTED;
+  // Largest route a query block can get: its budgeted part, the window and
+  // the reference blocks (all history), then its own chunk.
+  const int p0 = std::min(std::max(o.prev_first, 0), std::max(n_hist, 0));
+  const int p1 = std::min(std::max(o.prev_first + o.n_prev, p0), std::max(n_hist, 0));
+  const long long budget = std::max<long long>(std::max(o.k_cov, p1 - p0), o.k_unc);
+  const long long bound =
+      std::min<long long>(n_hist, budget + 2LL * o.window_half + 1 + o.n_ref) + n_own;
+  if (max_sel < bound) return BSA_ERR_CAPACITY;
+  cudaStream_t s = as_stream(stream);
+  RouteArgs a;
+  bsa_status st = route_scores(q_blk, c, q_valid, n_hist, own_first, n_own, g, lambda, g_ref,
+                               sm_scale, idx, cnt, max_sel, workspace, ws_bytes, d_err, s, &a);
+  if (st != BSA_OK) return st;
+  VeloxArgs v{o.coverage, o.eta_cov, o.tau, o.mass, o.k_cov, o.k_unc, o.prev_first, o.n_prev,
+              o.window_half, o.ref_first, o.n_ref};
+  const size_t smem = sizeof(uint64_t) * kVeloxSortMax +
+                      static_cast<size_t>(std::max(n_hist, 1)) * (sizeof(uint32_t) + 1) + 16;
+  if (cudaFuncSetAttribute(velox_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  dim3 qgrid(n_own, c->Hh, c->B);
+  velox_select_kernel<<<qgrid, kTopkThreads, smem, s>>>(a, v);
   return launch_status();
 }
 

@@ -224,6 +224,58 @@ bsa_status bsa_attn(const void *q_blk, const bsa_kv_cache *cache, const int32_t 
 bsa_status bsa_selftest_bounded_wait(int32_t *d_err, long long limit_cycles, void *stream);
 
 /*
+ * Options of the page's own route (Velox, Methodology Steps 4-5).
+ *   coverage     device fp32 [B, n_own]: fraction of each query block's
+ *                tokens inside a valid historical slab, or NULL (no query
+ *                block is well covered)
+ *   eta_cov      a query block is well covered when coverage >= eta_cov (0.9)
+ *   tau          overlap at or below tau counts as none (0.1)
+ *   k_cov        covered route size: the previous chunk is reserved first,
+ *                then the best other history blocks up to k_cov in all (80)
+ *   k_unc        cap of the uncovered route (150, at most 1024)
+ *   mass         uncovered route: smallest prefix of softmax(s), in order of
+ *                decreasing s (ties to the lower index), whose mass reaches
+ *                this value (the page does not state it; 0.9 is a choice)
+ *   prev_first, n_prev   the previous chunk's blocks [prev_first, +n_prev)
+ *   window_half  window of previous-chunk blocks at Gilbert positions
+ *                j - window_half .. j + window_half around query block j,
+ *                added outside the budget (13)
+ *   ref_first, n_ref     reference blocks always added (n_ref may be 0)
+ */
+typedef struct bsa_velox_route {
+  const float *coverage;
+  float eta_cov, tau;
+  int32_t k_cov, k_unc;
+  float mass;
+  int32_t prev_first, n_prev;
+  int32_t window_half;
+  int32_t ref_first, n_ref;
+} bsa_velox_route;
+
+/*
+ * The page's full route for every (batch, head, query block).  Scores s are
+ * those of bsa_route (sm_scale * <mean q, mean k>, from the pooled-key cache
+ * when present).  A well-covered query block ranks history blocks by
+ * s + log(1 + lambda * g_hat), g_hat = min(g / g_ref, 1) where g > tau and 0
+ * elsewhere, which is the order of the importance distribution multiplied by
+ * (1 + lambda * g_hat) and renormalised; it takes the previous chunk, then
+ * the best remaining blocks up to k_cov.  Other query blocks take the
+ * smallest mass prefix of the unfused distribution, at most k_unc blocks.
+ * Every route is joined with the window and reference blocks, sorted
+ * ascending without repeats, and followed by the own chunk; cnt varies per
+ * query block and unused idx entries are -1.
+ *   max_sel   at least min(n_hist, max(k_cov, n_prev, k_unc) + 2 *
+ *             window_half + 1 + n_ref) + n_own, else BSA_ERR_CAPACITY
+ * Errors: those of bsa_route; BSA_ERR_UNSUPPORTED when n_hist > 32768 or
+ *         k_unc > 1024.
+ */
+bsa_status bsa_route_velox(const void *q_blk, const bsa_kv_cache *cache, const int32_t *q_valid,
+                           int n_hist, int own_first, int n_own, const float *g,
+                           float lambda, float g_ref, float sm_scale,
+                           const bsa_velox_route *opts, int32_t *idx, int32_t *cnt, int max_sel,
+                           void *workspace, size_t ws_bytes, int32_t *d_err, void *stream);
+
+/*
  * bsa_route without a workspace argument, for callers that cannot allocate
  * device memory themselves: for example code running inside another
  * runtime's plugin or enqueue hook, where the host framework owns every

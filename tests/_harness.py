@@ -92,6 +92,19 @@ def oracle_scores(step: Step, heads) -> np.ndarray:
     return oracle.fuse_prior(s, step.g_np, step.w.lam, step.w.g_ref)
 
 
+def oracle_scores_model(step: Step, heads) -> np.ndarray:
+    """Oracle model scores s = sm_scale * <qmean, kmean> (no prior) [B, len(heads), n_own, n_hist]."""
+    import oracle
+    q = f64(step.q_blk[:, heads])
+    kc = f64(step.cache.k[:, heads, :step.n_hist])
+    valid = step.cache.block_valid.cpu().numpy()
+    B, Hs, R, D = q.shape
+    qm = oracle.pool_blocks(q.reshape(B, Hs, step.n_own, BLK, D),
+                            [int(v) for v in valid[step.own_first:step.own_first + step.n_own]])
+    km = oracle.pool_blocks(kc, valid[:step.n_hist])
+    return oracle.block_scores(qm, km, step.w.sm_scale)
+
+
 def check_route_rows(idx: np.ndarray, cnt: np.ndarray, scores: np.ndarray, top_k: int,
                      own_first: int, n_own: int, rel_tol: float = 1e-5) -> int:
     """Compare GPU routes with the oracle's, row by row.
