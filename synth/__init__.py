@@ -8,6 +8,7 @@ from .workloads import (  # noqa: F401
     Workload,
     chunk_seed,
     chunk_tokens,
+    coverage,
     direct_blocks,
     prior,
     random_bf16,

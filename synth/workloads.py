@@ -169,6 +169,14 @@ def prior(w: Workload, c: int, n_q_blocks: int, n_hist: int) -> Optional[np.ndar
     return g.astype(np.float32)
 
 
+def coverage(w: Workload, c: int, n_q_blocks: int) -> np.ndarray:
+    """Synthetic coverage of each query block (fraction of its tokens inside a
+    valid historical slab): float32 [B, n_q_blocks] ~ U(0.5, 1), so that about
+    one query block in five is well covered at eta_cov = 0.9."""
+    rng = np.random.Generator(np.random.PCG64(1000 * w.key + 700 + c))
+    return rng.uniform(0.5, 1.0, size=(w.B, n_q_blocks)).astype(np.float32)
+
+
 def random_bf16(shape, seed: int, device="cpu", scale: float = 1.0) -> torch.Tensor:
     """Plain N(0, scale^2) bf16 tensor for edge-case tests."""
     gen = _gen(seed, device)
