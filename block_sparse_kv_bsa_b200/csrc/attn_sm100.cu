@@ -10,38 +10,46 @@
 // share that head's own-chunk K/V tiles through L2.
 //
 // Tensor memory (512 columns x 128 lanes, lane = query row):
-//   [0,128) [128,256)  two S = Q K^T buffers (fp32)
-//   [256, 256+D)       O accumulator (fp32)
-//   [384, 384+D/2)     Q (bf16 pairs, the A operand of Q K^T)
-//   [448, 512)         P (bf16 pairs, the A operand of P V)
-// Both products take A from tensor memory and only B (a K or V tile) from
-// shared memory: with M = 128 an operand read from shared memory costs as
-// much bandwidth as the tensor core consumes, so keeping Q and P out of
-// shared memory is what leaves room for the K/V tile stream.
+//   [0,128) [128,256) [256,384)  three S = Q K^T buffers (fp32); tile t uses
+//                                buffer t % 3, and P_t (bf16 pairs, the A
+//                                operand of P V) is written over columns
+//                                [0, 64) of that buffer
+//   [384, 384+D)                 O accumulator (fp32)
+// Q (128 x D bf16) stays in shared memory for the whole work item and is the
+// A operand of Q K^T; V is the B operand of P V (A from tensor memory).
+// Three S buffers let the Q K^T of tile t + 3 follow the P V of tile t, so
+// S_t is ready two product groups before the tensor core needs P_t, and the
+// softmax of one tile overlaps the products of the next two.  Writing P
+// over its own S buffer relies on the tcgen05.mma operations of one thread
+// executing in issue order: the P V of tile t reads the buffer before the
+// Q K^T of tile t + 3, issued after it, overwrites it.
 //
 // Warp roles:
-//   warp 0      TMA producer: the K and V tiles of each selected block
-//               (128 rows x D bf16, 128-byte swizzled boxes of 64 columns)
-//               into a three-stage ring; one full and one empty mbarrier per
-//               stage cover both tiles.  Tile row = ((b*Hh + h)*max_blocks +
-//               blk)*128.
-//   warp 1      allocates tensor memory; one lane issues tcgen05.mma:
-//               S_i = Q K_i^T and O += P_i V_i, committing each group to an
-//               mbarrier.  It waits only twice per tile (next stage loaded;
-//               this tile's P stored): a wait in the issuing thread leaves the
-//               tensor pipe without queued work, and measured ~170 SM cycles of
-//               lost tensor time per wait.
-//   warps 2-9   softmax: two warpgroups split every row (half 0: S/P columns
-//               0-63 and O columns [0, D/2); half 1 the rest).  They put Q
-//               into tensor memory, then per tile load S, mask the pad keys
-//               of a tail block, exchange the row maximum through shared
-//               memory, exponentiate in base 2 with a stale-maximum rule (O
-//               and the running sums are rescaled only when the row maximum
-//               grows by more than 2^8, so O/l stays exact), store P (bf16)
-//               into tensor memory, and finally normalise O and write O, LSE.
+//   warp 0      TMA producer: Q once, then the K tile (three-slot K ring) and
+//               the V tile (three-slot V ring) of each selected block, 128
+//               rows x D bf16 in 128-byte swizzled boxes of 64 columns; K runs
+//               two tiles ahead of V, the order in which the products consume
+//               them.  Tile row = ((b*Hh + h)*max_blocks + blk)*128.
+//   warp 1      allocates tensor memory; one lane issues tcgen05.mma.  Per
+//               tile it waits twice: for P_t stored and V_t landed (one
+//               barrier), then issues O += P_t V_t; for K_{t+3} landed, then
+//               issues S_{t+3} = Q K_{t+3}^T.  A wait in the issuing thread
+//               leaves the tensor pipe without queued work, and measured ~170
+//               SM cycles of lost tensor time per wait.
+//   warps 2-9   softmax: warpgroup g (warps 2-5, 6-9) takes every other tile
+//               t = g, g + 2, ...; a thread owns one query row.  Per tile it
+//               loads S, masks the pad keys of a tail block, takes the row
+//               maximum, receives the reference maximum of tile t - 1 from
+//               the other warpgroup and passes on its own (stale-maximum
+//               rule: the reference moves only when the row maximum exceeds
+//               it by more than 2^8, and O is then rescaled, so O/l stays
+//               exact), exponentiates in base 2 and stores P.  Finally the
+//               two warpgroups merge their running sums and write O and LSE.
 // Every wait is bounded; a wait that gives up records
 // BSA_DEV_WAIT_TIMEOUT, stops the other roles through a shared flag, lets
-// in-flight copies and MMAs finish (bounded) and frees tensor memory.
+// in-flight copies and MMAs finish (bounded) and frees tensor memory.  Every
+// warp runs the same sequence of named-barrier operations whether or not a
+// wait gave up, so an abort never leaves a partner waiting at a barrier.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -51,44 +59,49 @@
 
 namespace bsa {
 
-constexpr int kSoftmaxThreads = 256;  // two warpgroups, one per 64-column half
+constexpr int kSoftmaxThreads = 256;  // two warpgroups, one per tile parity
 constexpr int kAttnThreads = 64 + kSoftmaxThreads;
-constexpr int kStages = 3;            // K/V ring depth (one K and one V tile per stage)
-constexpr int kSBufs = 2;
-constexpr uint32_t kColS = 0;
-constexpr uint32_t kColO = 256;
-constexpr uint32_t kColQ = 384;
-constexpr uint32_t kColP = 448;
+constexpr int kKSlots = 3;            // K ring
+constexpr int kVSlots = 3;            // V ring
+constexpr int kSBufs = 3;             // S / P buffers in tensor memory
+constexpr int kKLead = 2;             // K tiles issued ahead of the V tile
+constexpr uint32_t kColO = 384;
 constexpr long long kWaitLimit = 1LL << 31;  // SM clocks (about a second)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
 // mbarrier slots
 enum {
-  B_Q_FULL = 0,
-  B_KV_FULL = 1,                      // + stage: K and V tile of one route entry landed
-  B_KV_EMPTY = B_KV_FULL + kStages,   // + stage: both products that read the stage are done
-  B_S_FULL = B_KV_EMPTY + kStages,    // + buffer
-  B_P_FULL = B_S_FULL + kSBufs,
-  B_O_READY,
-  B_MMA_DONE,
+  B_Q_FULL = 0,                       // Q landed (producer arrive + bytes)
+  B_K_FULL = 1,                       // + K slot: K tile landed
+  B_K_EMPTY = B_K_FULL + kKSlots,     // + K slot: its Q K^T is done
+  B_PV_READY = B_K_EMPTY + kKSlots,   // + V slot: V tile landed and P stored
+  B_V_EMPTY = B_PV_READY + kVSlots,   // + V slot: its P V is done
+  B_S_FULL = B_V_EMPTY + kVSlots,     // + warpgroup: S of its next tile ready
+  B_O_READY = B_S_FULL + 2,           // + tile parity: the P V of that tile is done
+  B_MMA_DONE = B_O_READY + 2,
   B_COUNT
 };
 
 template <int D>
 struct AttnLayout {
   static constexpr int kTileBytes = kBlk * D * 2;      // 128 rows x D bf16
-  static constexpr int kK = 0;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBars = kV + kStages * kTileBytes;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kV = kK + kKSlots * kTileBytes;
+  static constexpr int kBars = kV + kVSlots * kTileBytes;
   static constexpr int kMisc = kBars + B_COUNT * 8;
-  static constexpr int kRed = (kMisc + 64 + 15) & ~15;  // float [3 slots][2 halves][128 rows]
-  static constexpr int kTotal = kRed + 3 * 2 * kBlk * 4;
+  static constexpr int kTok = (kMisc + 64 + 15) & ~15;  // float [2 warpgroups][128 rows]
+  static constexpr int kTotal = kTok + 2 * kBlk * 4;
   static constexpr int kAlloc = kTotal + 1024;          // room to align to 1024
+  // The epilogue's [2][2][128] floats reuse K slot 0: by then every Q K^T
+  // has completed and no K copy is in flight.
+  static constexpr int kFin = kK;
+  static_assert(kAlloc <= 227 * 1024, "shared memory per CTA");
+  static_assert(kTileBytes >= 4 * kBlk * 4, "epilogue scratch fits in one K slot");
 };
 
 struct AttnArgs {
-  const __nv_bfloat16* q;
   const int32_t* idx;
   const int32_t* cnt;
   const int32_t* block_valid;
@@ -118,23 +131,27 @@ __device__ __forceinline__ int route_block(const AttnArgs& a, long long item, in
   return blk;
 }
 
-__device__ __forceinline__ int block_rows(const AttnArgs& a, int blk) {
-  int v = a.block_valid[blk];
-  if (v < 1 || v > kBlk) {
-    report(a.d_err, BSA_DEV_BAD_VALID);
-    v = v < 1 ? 1 : kBlk;
-  }
-  return v;
+// Named barriers 1-8 carry the row-maximum tokens between the two softmax
+// warpgroups (one per direction and TMEM lane window, 64 threads each);
+// barrier 9 joins all softmax threads in the epilogue.
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ void named_bar_sync_softmax() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxThreads) : "memory");
+// Maximum of three floats in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float x, float y, float z) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(x), "f"(y), "f"(z));
+  return d;
 }
 
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                AttnArgs a) {
+bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
   using L = AttnLayout<D>;
   constexpr int kBoxes = D / 64;
   constexpr uint32_t kTileBytes = L::kTileBytes;
@@ -154,7 +171,9 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t count = 1;
-      if (i == B_Q_FULL || i == B_P_FULL) count = kSoftmaxThreads;
+      // V landed (the producer's arrive with its byte count) + P stored by
+      // the 128 threads of one warpgroup.
+      if (i >= B_PV_READY && i < B_PV_READY + kVSlots) count = 1 + kSoftmaxThreads / 2;
       mbar_init(&bars[i], count);
     }
     *s_abort = 0;
@@ -170,86 +189,107 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int issued = 0;
-      for (int i = 0; i < n; ++i) {
-        const int st = i % kStages;
-        const int blk = route_block(a, item, i);
-        const int row = static_cast<int>((bh * a.max_blocks + blk) * kBlk);
-        if (i >= kStages && !mbar_wait_bounded(&bars[B_KV_EMPTY + st], ((i / kStages) - 1) & 1,
-                                               s_abort, kWaitLimit))
-          break;
-        mbar_expect_tx(&bars[B_KV_FULL + st], 2 * kTileBytes);
-        for (int bx = 0; bx < kBoxes; ++bx) {
-          tma_load_2d(sm + L::kK + st * kTileBytes + bx * (kBlk * 128), &tm_k, bx * 64, row,
-                      &bars[B_KV_FULL + st]);
-          tma_load_2d(sm + L::kV + st * kTileBytes + bx * (kBlk * 128), &tm_v, bx * 64, row,
-                      &bars[B_KV_FULL + st]);
+      mbar_expect_tx(&bars[B_Q_FULL], kTileBytes);
+      for (int bx = 0; bx < kBoxes; ++bx)
+        tma_load_2d(sm + L::kQ + bx * (kBlk * 128), &tm_q, bx * 64, static_cast<int>(item * kBlk),
+                    &bars[B_Q_FULL]);
+      int k_issued = 0, v_issued = 0;
+      bool ok = true;
+      // Step s issues K_s (while s < n), then V_{s - kKLead}.
+      for (int step = 0; ok && step < n + kKLead; ++step) {
+        if (step < n) {
+          const int t = step, sl = t % kKSlots;
+          const int row = static_cast<int>((bh * a.max_blocks + route_block(a, item, t)) * kBlk);
+          if (t >= kKSlots)
+            ok = mbar_wait_bounded(&bars[B_K_EMPTY + sl], ((t / kKSlots) - 1) & 1, s_abort,
+                                   kWaitLimit);
+          if (!ok) break;
+          mbar_expect_tx(&bars[B_K_FULL + sl], kTileBytes);
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_2d(sm + L::kK + sl * kTileBytes + bx * (kBlk * 128), &tm_k, bx * 64, row,
+                        &bars[B_K_FULL + sl]);
+          k_issued = t + 1;
         }
-        issued = i + 1;
+        const int t = step - kKLead;
+        if (t >= 0 && t < n) {
+          const int sl = t % kVSlots;
+          const int row = static_cast<int>((bh * a.max_blocks + route_block(a, item, t)) * kBlk);
+          if (t >= kVSlots)
+            ok = mbar_wait_bounded(&bars[B_V_EMPTY + sl], ((t / kVSlots) - 1) & 1, s_abort,
+                                   kWaitLimit);
+          if (!ok) break;
+          mbar_expect_tx(&bars[B_PV_READY + sl], kTileBytes);
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_2d(sm + L::kV + sl * kTileBytes + bx * (kBlk * 128), &tm_v, bx * 64, row,
+                        &bars[B_PV_READY + sl]);
+          v_issued = t + 1;
+        }
       }
-      if (issued < n) {
+      if (!ok) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
         *s_abort = 1;
       }
       // Drain: every copy this thread issued must land before the CTA exits.
-      for (int st = 0; st < kStages; ++st) {
+      // (A V slot's barrier also counts the P arrivals of its tile, which
+      // every softmax warpgroup makes for each of its tiles.)
+      mbar_wait_bounded(&bars[B_Q_FULL], 0, nullptr, kWaitLimit);
+      for (int sl = 0; sl < kKSlots; ++sl) {
         int last = -1;
-        for (int i = st; i < issued; i += kStages) last = i;
+        for (int t = sl; t < k_issued; t += kKSlots) last = t;
         if (last >= 0)
-          mbar_wait_bounded(&bars[B_KV_FULL + st], (last / kStages) & 1, nullptr, kWaitLimit);
+          mbar_wait_bounded(&bars[B_K_FULL + sl], (last / kKSlots) & 1, nullptr, kWaitLimit);
+      }
+      for (int sl = 0; sl < kVSlots; ++sl) {
+        int last = -1;
+        for (int t = sl; t < v_issued; t += kVSlots) last = t;
+        if (last >= 0)
+          mbar_wait_bounded(&bars[B_PV_READY + sl], (last / kVSlots) & 1, nullptr, kWaitLimit);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    // Every mbarrier wait of this thread leaves the tensor pipe without new
-    // work for a while, so there are only two per tile: the K/V stage of the
-    // next tile (before its Q K^T) and this tile's P (before its P V).  The S
-    // buffer that Q K^T_{t} overwrites held S_{t-2}; the softmax read it
-    // before storing P_{t-2}, which this thread already waited for.
     if (lane == 0 && n > 0) {
       constexpr uint32_t kIdQK = idesc_bf16(128, 128, 0);
       constexpr uint32_t kIdPV = idesc_bf16(128, D, 1);
-      bool ok = mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit);
-      auto issue_qk = [&](int t) {
-        const int st = t % kStages, sb = t % kSBufs;
-        const uint32_t k_addr = smem_u32(sm + L::kK + st * kTileBytes);
+      const uint32_t q_addr = smem_u32(sm + L::kQ);
+      // S_t = Q K_t^T into buffer t % 3 (K slot t % 3), once K_t landed.
+      auto issue_qk = [&](int t) -> bool {
+        const int sl = t % kKSlots;
+        if (!mbar_wait_bounded(&bars[B_K_FULL + sl], (t / kKSlots) & 1, s_abort, kWaitLimit))
+          return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sm + L::kK + sl * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * (kBlk * 128) + (kk % 4) * 32;
-          tc_mma_ts(tmem + kColS + sb * 128, tmem + kColQ + kk * 8,
+          tc_mma_ss(tmem + (t % kSBufs) * 128, smem_desc(q_addr + off, 16, 1024),
                     smem_desc(k_addr + off, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bars[B_S_FULL + sb]);
+        tc_commit(&bars[B_K_EMPTY + sl]);
+        tc_commit(&bars[B_S_FULL + (t & 1)]);
+        return true;
       };
-      if (ok) ok = mbar_wait_bounded(&bars[B_KV_FULL + 0], 0, s_abort, kWaitLimit);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0);
-      }
+      bool ok = mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit);
+      for (int t = 0; ok && t < kSBufs && t < n; ++t) ok = issue_qk(t);
       for (int i = 0; ok && i < n; ++i) {
-        if (i + 1 < n) {
-          const int t = i + 1;
-          ok = mbar_wait_bounded(&bars[B_KV_FULL + t % kStages], (t / kStages) & 1, s_abort,
-                                 kWaitLimit);
-          if (!ok) break;
-          tc_fence_after();
-          issue_qk(t);
-        }
-        const int st = i % kStages;
-        ok = mbar_wait_bounded(&bars[B_P_FULL], i & 1, s_abort, kWaitLimit);
+        // O += P_i V_i once P_i is stored and V_i landed.
+        const int sl = i % kVSlots;
+        ok = mbar_wait_bounded(&bars[B_PV_READY + sl], (i / kVSlots) & 1, s_abort, kWaitLimit);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm + L::kV + st * kTileBytes);
+        const uint32_t v_addr = smem_u32(sm + L::kV + sl * kTileBytes);
+        const uint32_t p_col = tmem + (i % kSBufs) * 128;
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
-          tc_mma_ts(tmem + kColO, tmem + kColP + kk * 8,
-                    smem_desc(v_addr + kk * 2048, kBlk * 128, 1024), kIdPV,
-                    (i > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + kColO, p_col + kk * 8, smem_desc(v_addr + kk * 2048, kBlk * 128, 1024),
+                    kIdPV, (i > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&bars[B_KV_EMPTY + st]);
-        tc_commit(&bars[B_O_READY]);
+        tc_commit(&bars[B_V_EMPTY + sl]);
+        tc_commit(&bars[B_O_READY + (i & 1)]);
+        if (i + kSBufs < n) ok = issue_qk(i + kSBufs);
       }
       if (!ok) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
@@ -261,156 +301,187 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
   } else {
     // ---------------- softmax / epilogue (warps 2..9) ----------------
-    // Two warpgroups split every row: half 0 owns S/P columns 0-63 and O
-    // columns [0, D/2), half 1 the rest.  The row maximum is exchanged through
-    // shared memory once per tile; the running sums stay per half (both halves
-    // use the same reference maximum) and are added in the epilogue.
-    const int half = (warp - 2) >> 2;        // 0 or 1
+    // The reference maximum m_t of tile t is decided in tile order: the
+    // thread of row r in the warpgroup of tile t - 1 hands m_{t-1} to the
+    // thread of row r in the other warpgroup through shared memory and a
+    // named barrier per TMEM lane window (producer bar.arrive, consumer
+    // bar.sync).  Both warpgroups thus exponentiate against the same
+    // reference as O.  Each keeps its own running sum, expressed in the last
+    // reference it used; the two are merged in the epilogue.
+    const int g = (warp - 2) >> 2;           // warpgroup: 0 or 1
     const int wq = warp & 3;                 // TMEM lane window of this warp
     const int r = wq * 32 + lane;            // query row owned by this thread
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    constexpr int kHalfCols = kBlk / 2;      // S / P columns per thread
-    constexpr int kHalfD = D / 2;            // O columns per thread
-    const int c0 = half * kHalfCols;
-    const uint32_t o_col = kColO + half * kHalfD;
-    float* red = reinterpret_cast<float*>(sm + L::kRed);  // [3][2][128]
+    float* tok = reinterpret_cast<float*>(sm + L::kTok);  // [2 warpgroups][128 rows]
+    const int bar_in = 1 + (g ^ 1) * 4 + wq;              // token from the other warpgroup
+    const int bar_out = 1 + g * 4 + wq;                   // token to the other warpgroup
 
-    // Q row r -> tensor memory as bf16 pairs (the A operand of Q K^T).  With
-    // D = 128 each half stores its 64 elements; with D = 64 half 0 stores the
-    // whole row.
-    if (n > 0) {
-      const uint4* qrow = reinterpret_cast<const uint4*>(a.q + (item * kBlk + r) * D);
-      if (D == 128 || half == 0) {
-        const int e0 = (D == 128) ? half * 64 : 0;   // first element stored
-        uint32_t qw[32];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          uint4 x = ld_nc_v4(qrow + e0 / 8 + v);
-          qw[4 * v + 0] = x.x; qw[4 * v + 1] = x.y; qw[4 * v + 2] = x.z; qw[4 * v + 3] = x.w;
-        }
-        tmem_st32u(tmem + lane_base + kColQ + e0 / 2, qw);
-        tc_wait_st();
-      }
-      tc_fence_before();
-      mbar_arrive(&bars[B_Q_FULL]);
-    }
-
-    float m_ref = -INFINITY, l = 0.f;
+    float m_last = -INFINITY;  // reference of this warpgroup's running sum
+    float l = 0.f;
     bool ok = true;
-    // Route lookahead: the block index two tiles ahead and the valid-row
-    // count one tile ahead are loaded early and first used a tile later, so
-    // these dependent global loads never stall the softmax.  Indices are
-    // validated (and reported) by the producer; here they are only clamped.
+    // Route lookahead: the valid-row count of this warpgroup's next tile and
+    // the block index of the one after it are loaded a tile early, so these
+    // dependent global loads never stall the softmax.  Indices are validated
+    // (and reported) by the producer; here they are only clamped.
     const int32_t* route = a.idx + item * a.max_sel;
-    auto clamp_blk = [&](int b_) { return static_cast<unsigned>(b_) < static_cast<unsigned>(a.n_blocks) ? b_ : 0; };
-    int blk_ahead = n > 1 ? route[1] : 0;
-    int valid_raw = n > 0 ? a.block_valid[clamp_blk(route[0])] : kBlk;
-    for (int i = 0; i < n; ++i) {
-      const int sb = i % kSBufs;
+    auto clamp_blk = [&](int b_) {
+      return static_cast<unsigned>(b_) < static_cast<unsigned>(a.n_blocks) ? b_ : 0;
+    };
+    int blk_ahead = (g + 2 < n) ? route[g + 2] : 0;
+    int valid_raw = (g < n) ? a.block_valid[clamp_blk(route[g])] : kBlk;
+    for (int t = g; t < n; t += 2) {
       int valid = valid_raw;
       if (valid < 1 || valid > kBlk) {
         report(a.d_err, BSA_DEV_BAD_VALID);
         valid = valid < 1 ? 1 : kBlk;
       }
-      const int blk_ahead2 = (i + 2 < n) ? route[i + 2] : 0;
-      valid_raw = (i + 1 < n) ? a.block_valid[clamp_blk(blk_ahead)] : kBlk;
+      const int blk_ahead2 = (t + 4 < n) ? route[t + 4] : 0;
+      valid_raw = (t + 2 < n) ? a.block_valid[clamp_blk(blk_ahead)] : kBlk;
       blk_ahead = blk_ahead2;
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_S_FULL + sb], (i / kSBufs) & 1,
-                                                     s_abort, kWaitLimit));
-      if (!ok) break;
-      tc_fence_after();
-      float s[kHalfCols];
-      tmem_ld_cols<kHalfCols>(tmem + lane_base + kColS + sb * 128 + c0, s);
+      const uint32_t s_col = static_cast<uint32_t>(t % kSBufs) * 128;
+
+      // Warpgroup g is the only waiter on S_FULL + g and waits for each of
+      // its completions in turn, so the parity is exact.
+      float s[kBlk];
+      if (ok)
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_S_FULL + g], (t >> 1) & 1, s_abort,
+                                                       kWaitLimit));
+      if (ok) {
+        tc_fence_after();
+        tmem_ld_cols<kBlk>(tmem + lane_base + s_col, s);
+      } else {
+#pragma unroll
+        for (int c = 0; c < kBlk; ++c) s[c] = 0.f;
+      }
       if (valid < kBlk) {  // tail block of a chunk: mask its pad keys
 #pragma unroll
-        for (int c = 0; c < kHalfCols; ++c)
-          if (c0 + c >= valid) s[c] = -INFINITY;
+        for (int c = 0; c < kBlk; ++c)
+          if (c >= valid) s[c] = -INFINITY;
       }
-      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      // Row maximum: four chains over columns 0-11, 12-123 (pairs), 124-127.
+      static_assert(kBlk == 128, "the maximum below covers exactly 128 columns");
+      float mq[4];
 #pragma unroll
-      for (int c = 0; c < kHalfCols; ++c) mq[c & 3] = fmaxf(mq[c & 3], s[c]);
-      const float pm = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-      float* red_t = red + (i & 1) * (2 * kBlk);
-      red_t[half * kBlk + r] = pm;
-      named_bar_sync_softmax();
-      const float mx = fmaxf(pm, red_t[(half ^ 1) * kBlk + r]);
-      const float mx2 = mx * a.scale_log2;
-      float m_new = m_ref;
-      if (i == 0 || mx2 > m_ref + kRescaleThreshold) m_new = mx2;
+      for (int k = 0; k < 4; ++k) mq[k] = fmax3(s[k], s[k + 4], s[k + 8]);
+#pragma unroll
+      for (int c = 12; c + 4 < kBlk; c += 8) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mq[k] = fmax3(mq[k], s[c + k], s[c + 4 + k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mq[k] = fmaxf(mq[k], s[kBlk - 4 + k]);
+      const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * a.scale_log2;
+
+      // Reference maximum of tile t, decided in tile order.
+      float m_prev = -INFINITY;
+      if (t > 0) {
+        named_bar_sync(bar_in, 64);
+        m_prev = tok[(g ^ 1) * kBlk + r];
+      }
+      const float m_t = (t == 0 || mx > m_prev + kRescaleThreshold) ? mx : m_prev;
+      if (t + 1 < n) {
+        tok[g * kBlk + r] = m_t;
+        named_bar_arrive(bar_out, 64);
+      }
+
+      // P (bf16 pairs) overwrites the S buffer it was computed from, 32 keys
+      // at a time: TMEM columns s_col + [0, 64) then hold P row r.
       float rq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kHalfCols; ++c) {
-        s[c] = ex2_approx(fmaf(s[c], a.scale_log2, -m_new));
-        rq[c & 3] += s[c];
+      for (int q = 0; q < kBlk / 32; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float e0 = ex2_approx(fmaf(s[32 * q + 2 * c], a.scale_log2, -m_t));
+          const float e1 = ex2_approx(fmaf(s[32 * q + 2 * c + 1], a.scale_log2, -m_t));
+          rq[(2 * c) & 3] += e0;
+          rq[(2 * c + 1) & 3] += e1;
+          pk[c] = pack_bf16x2(e0, e1);
+        }
+        if (ok) tmem_st16u(tmem + lane_base + s_col + 16 * q, pk);
       }
       const float rs = (rq[0] + rq[1]) + (rq[2] + rq[3]);
-      uint32_t pk[kHalfCols / 2];
+      if (m_t != m_last) {  // m_last = -inf scales the empty sum 0 by 0
+        l *= ex2_approx(m_last - m_t);
+        m_last = m_t;
+      }
+      l += rs;
+
+      // The P V of the previous tile (accumulated against m_prev) completes
+      // before this tile's P is released, so that a larger reference can
+      // rescale O in between; this also keeps the arrivals of consecutive
+      // tiles on the PV_READY barriers apart.  It costs the tensor pipe
+      // nothing: this tile's P V queues behind Q K^T of tile t + 2 anyway.
+      // Warpgroup g is the only waiter on O_READY + (g ^ 1) here and waits
+      // for each of its completions in turn, so the parity is exact.
+      // tcgen05.ld/st are warp-collective: the branch is warp-uniform and a
+      // lane whose reference did not move scales by exactly 1.
+      if (ok && t > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_O_READY + (g ^ 1)],
+                                                       ((t - 1) >> 1) & 1, s_abort, kWaitLimit));
+        const bool grow = m_t != m_prev;
+        if (ok && __any_sync(0xffffffffu, grow)) {
+          tc_fence_after();
+          const float alpha = grow ? ex2_approx(m_prev - m_t) : 1.0f;
 #pragma unroll
-      for (int c = 0; c < kHalfCols / 2; ++c) pk[c] = pack_bf16x2(s[2 * c], s[2 * c + 1]);
-      if (i > 0) {
-        // P V of the previous tile must be done: it reads the P columns this
-        // tile overwrites and accumulates into the O that may be rescaled.
-        // tcgen05.ld/st are warp-collective: the branch is warp-uniform and a
-        // lane whose maximum did not move scales by exactly 1.
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_O_READY], (i - 1) & 1, s_abort,
-                                                       kWaitLimit));
-        if (!ok) break;
-        tc_fence_after();
-        const bool grow = m_new != m_ref;
-        if (__any_sync(0xffffffffu, grow)) {
-          const float alpha = grow ? ex2_approx(m_ref - m_new) : 1.0f;
-          l *= alpha;
-#pragma unroll
-          for (int c = 0; c < kHalfD / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             float o[32];
-            tmem_ld_cols<32>(tmem + lane_base + o_col + c * 32, o);
+            tmem_ld_cols<32>(tmem + lane_base + kColO + c * 32, o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] *= alpha;
-            tmem_st32(tmem + lane_base + o_col + c * 32, o);
+            tmem_st32(tmem + lane_base + kColO + c * 32, o);
           }
         }
       }
-      l += rs;
-      m_ref = m_new;
-      // P row r, this half's 64 keys -> 32 TMEM columns of bf16 pairs.
-      tmem_st32u(tmem + lane_base + kColP + half * (kHalfCols / 2), pk);
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars[B_P_FULL]);
+      mbar_arrive(&bars[B_PV_READY + t % kVSlots]);
     }
     if (!ok) {
       report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
       *s_abort = 1;
     }
-    // Epilogue: total row sum from both halves, then each half writes its
-    // D/2 output columns; half 0 writes the LSE.
+    // Epilogue: merge the two running sums against the final reference (the
+    // larger of the two: references never decrease), then each warpgroup
+    // normalises D/2 output columns; warpgroup 0 writes the LSE.
     const int q_valid = a.q_valid != nullptr ? a.q_valid[j] : kBlk;
     const long long grow_idx = item * kBlk + r;
-    __nv_bfloat16* orow = a.o + grow_idx * D + half * kHalfD;
-    bool have = ok && n > 0 && r < q_valid;
-    if (ok && n > 0) {
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait_bounded(&bars[B_O_READY], (n - 1) & 1, s_abort, kWaitLimit));
+    __nv_bfloat16* orow = a.o + grow_idx * D + g * (D / 2);
+    // The last P V (tile n - 1) is awaited by the warpgroup that did not
+    // process tile n - 1: in its loop it waited for every earlier completion
+    // of that barrier, so the parity is exact.  The named barrier then
+    // releases both; that commit covers every earlier MMA of the issuer.
+    if (ok && n > 0 && g == (n & 1)) {
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_O_READY + ((n - 1) & 1)],
+                                                     ((n - 1) >> 1) & 1, s_abort, kWaitLimit));
       if (!ok) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
         *s_abort = 1;
-        have = false;
       }
-      tc_fence_after();
     }
-    // Slot 2 is never used by the per-tile exchange (slots 0 and 1), so the
-    // other half may still be reading its last tile's maximum.
-    float* red_e = red + 2 * (2 * kBlk);
-    red_e[half * kBlk + r] = l;
-    named_bar_sync_softmax();
-    const float l_tot = red_e[r] + red_e[kBlk + r];
+    // Every Q K^T has completed by now (warpgroup (n - 1) & 1 saw the last
+    // S, the other the last P V), so K slot 0 is free for the merge.
+    float* fin = reinterpret_cast<float*>(sm + L::kFin);  // [m, l][warpgroup][128 rows]
+    fin[(0 * 2 + g) * kBlk + r] = m_last;
+    fin[(1 * 2 + g) * kBlk + r] = l;
+    tc_fence_before();
+    named_bar_sync(9, kSoftmaxThreads);
+    tc_fence_after();
+    ok = __all_sync(0xffffffffu, ok && *s_abort == 0);
+    const float m0 = fin[0 * kBlk + r], m1 = fin[1 * kBlk + r];
+    const float m_fin = fmaxf(m0, m1);
+    const bool have = ok && n > 0 && r < q_valid && m_fin > -INFINITY;
+    float l_tot = 0.f;
+    if (have) {
+      l_tot = fin[2 * kBlk + r] * ex2_approx(m0 - m_fin) + fin[3 * kBlk + r] * ex2_approx(m1 - m_fin);
+    }
     const float inv_l = have ? 1.0f / l_tot : 0.f;
 #pragma unroll
-    for (int c = 0; c < kHalfD / 32; ++c) {
+    for (int c = 0; c < D / 64; ++c) {
       float o[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) o[e] = 0.f;
-      if (ok && n > 0) tmem_ld_cols<32>(tmem + lane_base + o_col + c * 32, o);
+      if (ok && n > 0) tmem_ld_cols<32>(tmem + lane_base + kColO + g * (D / 2) + c * 32, o);
 #pragma unroll
       for (int e = 0; e < 32; e += 8) {
         uint4 v;
@@ -421,8 +492,8 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
       }
     }
-    if (half == 0)
-      a.lse[grow_idx] = have ? (m_ref + __log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
+    if (g == 0)
+      a.lse[grow_idx] = have ? (m_fin + __log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
   }
 
   tc_fence_before();
@@ -475,14 +546,16 @@ static bool device_is_sm100() {
 template <int D>
 static bsa_status launch_attn(const void* q, const bsa_kv_cache* c, const AttnArgs& a,
                               long long items, cudaStream_t s) {
-  CUtensorMap tk, tv;
+  CUtensorMap tq, tk, tv;
   const long long crows = static_cast<long long>(c->B) * c->Hh * c->max_blocks * kBlk;
-  if (!make_map(&tk, c->k, crows, D) || !make_map(&tv, c->v, crows, D)) return BSA_ERR_CUDA;
+  if (!make_map(&tq, q, items * kBlk, D) || !make_map(&tk, c->k, crows, D) ||
+      !make_map(&tv, c->v, crows, D))
+    return BSA_ERR_CUDA;
   const int smem = AttnLayout<D>::kAlloc;
   if (cudaFuncSetAttribute(bsa_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return BSA_ERR_CUDA;
-  bsa_attn_kernel<D><<<static_cast<unsigned>(items), kAttnThreads, smem, s>>>(tk, tv, a);
+  bsa_attn_kernel<D><<<static_cast<unsigned>(items), kAttnThreads, smem, s>>>(tq, tk, tv, a);
   return launch_status();
 }
 
@@ -508,7 +581,6 @@ extern "C" bsa_status bsa_attn(const void* q_blk, const bsa_kv_cache* c, const i
   if (items * kBlk >= (1LL << 31) || crows >= (1LL << 31)) return BSA_ERR_SHAPE;
   if (!device_is_sm100()) return BSA_ERR_UNSUPPORTED;
   AttnArgs a{};
-  a.q = static_cast<const __nv_bfloat16*>(q_blk);
   a.idx = idx;
   a.cnt = cnt;
   a.block_valid = c->block_valid;
