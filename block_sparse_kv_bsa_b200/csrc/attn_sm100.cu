@@ -31,11 +31,15 @@
 //               two tiles ahead of V, the order in which the products consume
 //               them.  Tile row = ((b*Hh + h)*max_blocks + blk)*128.
 //   warp 1      allocates tensor memory; one lane issues tcgen05.mma.  Per
-//               tile it waits twice: for P_t stored and V_t landed (one
-//               barrier), then issues O += P_t V_t; for K_{t+3} landed, then
-//               issues S_{t+3} = Q K_{t+3}^T.  A wait in the issuing thread
-//               leaves the tensor pipe without queued work, and measured ~170
-//               SM cycles of lost tensor time per wait.
+//               tile it waits once, for one barrier that the softmax
+//               warpgroup completes after storing P_t and seeing V_t and
+//               K_{t+3} land; it then issues O += P_t V_t and S_{t+3} =
+//               Q K_{t+3}^T.  Operand descriptors are built once per CTA.
+//               The tensor pipe is fed only as fast as this one thread
+//               issues: each wait it executes, and every instruction it
+//               shares issue slots with, costs tensor time (measured: ~190
+//               SM cycles per wait per tile, and as much again from busy
+//               warps on the same SM).
 //   warps 2-9   softmax: warpgroup g (warps 2-5, 6-9) takes every other tile
 //               t = g, g + 2, ...; a thread owns one query row.  Per tile it
 //               loads S, masks the pad keys of a tail block, takes the row
@@ -75,9 +79,10 @@ enum {
   B_Q_FULL = 0,                       // Q landed (producer arrive + bytes)
   B_K_FULL = 1,                       // + K slot: K tile landed
   B_K_EMPTY = B_K_FULL + kKSlots,     // + K slot: its Q K^T is done
-  B_PV_READY = B_K_EMPTY + kKSlots,   // + V slot: V tile landed and P stored
-  B_V_EMPTY = B_PV_READY + kVSlots,   // + V slot: its P V is done
-  B_S_FULL = B_V_EMPTY + kVSlots,     // + warpgroup: S of its next tile ready
+  B_V_FULL = B_K_EMPTY + kKSlots,     // + V slot: V tile landed
+  B_V_EMPTY = B_V_FULL + kVSlots,     // + V slot: its P V is done
+  B_PV_READY = B_V_EMPTY + kVSlots,   // + slot t % 3: P_t stored, V_t and K_{t+3} landed
+  B_S_FULL = B_PV_READY + kVSlots,    // + warpgroup: S of its next tile ready
   B_O_READY = B_S_FULL + 2,           // + tile parity: the P V of that tile is done
   B_MMA_DONE = B_O_READY + 2,
   B_COUNT
@@ -141,6 +146,27 @@ __device__ __forceinline__ void named_bar_arrive(int id, int count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Two-wide fp32 arithmetic (sm_100): one instruction per pair, each lane
+// rounded exactly like its scalar counterpart.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t x, uint64_t y, uint64_t z) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(x), "l"(y), "l"(z));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t x, uint64_t y) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(y));
+  return d;
+}
+
 // Maximum of three floats in one instruction (sm_100).
 __device__ __forceinline__ float fmax3(float x, float y, float z) {
   float d;
@@ -171,9 +197,8 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int i = 0; i < B_COUNT; ++i) {
       uint32_t count = 1;
-      // V landed (the producer's arrive with its byte count) + P stored by
-      // the 128 threads of one warpgroup.
-      if (i >= B_PV_READY && i < B_PV_READY + kVSlots) count = 1 + kSoftmaxThreads / 2;
+      // The 128 threads of the warpgroup that owns the tile.
+      if (i >= B_PV_READY && i < B_PV_READY + kVSlots) count = kSoftmaxThreads / 2;
       mbar_init(&bars[i], count);
     }
     *s_abort = 0;
@@ -221,10 +246,10 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ok = mbar_wait_bounded(&bars[B_V_EMPTY + sl], ((t / kVSlots) - 1) & 1, s_abort,
                                    kWaitLimit);
           if (!ok) break;
-          mbar_expect_tx(&bars[B_PV_READY + sl], kTileBytes);
+          mbar_expect_tx(&bars[B_V_FULL + sl], kTileBytes);
           for (int bx = 0; bx < kBoxes; ++bx)
             tma_load_2d(sm + L::kV + sl * kTileBytes + bx * (kBlk * 128), &tm_v, bx * 64, row,
-                        &bars[B_PV_READY + sl]);
+                        &bars[B_V_FULL + sl]);
           v_issued = t + 1;
         }
       }
@@ -233,8 +258,6 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         *s_abort = 1;
       }
       // Drain: every copy this thread issued must land before the CTA exits.
-      // (A V slot's barrier also counts the P arrivals of its tile, which
-      // every softmax warpgroup makes for each of its tiles.)
       mbar_wait_bounded(&bars[B_Q_FULL], 0, nullptr, kWaitLimit);
       for (int sl = 0; sl < kKSlots; ++sl) {
         int last = -1;
@@ -246,7 +269,7 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int last = -1;
         for (int t = sl; t < v_issued; t += kVSlots) last = t;
         if (last >= 0)
-          mbar_wait_bounded(&bars[B_PV_READY + sl], (last / kVSlots) & 1, nullptr, kWaitLimit);
+          mbar_wait_bounded(&bars[B_V_FULL + sl], (last / kVSlots) & 1, nullptr, kWaitLimit);
       }
     }
   } else if (warp == 1) {
@@ -254,42 +277,52 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (lane == 0 && n > 0) {
       constexpr uint32_t kIdQK = idesc_bf16(128, 128, 0);
       constexpr uint32_t kIdPV = idesc_bf16(128, D, 1);
-      const uint32_t q_addr = smem_u32(sm + L::kQ);
-      // S_t = Q K_t^T into buffer t % 3 (K slot t % 3), once K_t landed.
-      auto issue_qk = [&](int t) -> bool {
+      // Descriptors of every operand tile, built once; a k-step only adds
+      // its byte offset / 16 to the start-address field.
+      // Slots are kTileBytes apart, so slot sl adds sl * kTileBytes / 16.
+      const uint64_t q_desc = smem_desc(smem_u32(sm + L::kQ), 16, 1024);
+      const uint64_t k_desc0 = smem_desc(smem_u32(sm + L::kK), 16, 1024);
+      const uint64_t v_desc0 = smem_desc(smem_u32(sm + L::kV), kBlk * 128, 1024);
+      constexpr uint32_t kSlot16 = kTileBytes >> 4;
+      // S_t = Q K_t^T into buffer t % 3 from K slot t % 3.
+      auto issue_qk = [&](int t) {
         const int sl = t % kKSlots;
-        if (!mbar_wait_bounded(&bars[B_K_FULL + sl], (t / kKSlots) & 1, s_abort, kWaitLimit))
-          return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm + L::kK + sl * kTileBytes);
+        const uint64_t k_desc = desc_add(k_desc0, sl * kSlot16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * (kBlk * 128) + (kk % 4) * 32;
-          tc_mma_ss(tmem + (t % kSBufs) * 128, smem_desc(q_addr + off, 16, 1024),
-                    smem_desc(k_addr + off, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * (kBlk * 128) + (kk % 4) * 32) >> 4;
+          tc_mma_ss(tmem + (t % kSBufs) * 128, desc_add(q_desc, off), desc_add(k_desc, off),
+                    kIdQK, kk > 0 ? 1u : 0u);
         }
         tc_commit(&bars[B_K_EMPTY + sl]);
         tc_commit(&bars[B_S_FULL + (t & 1)]);
-        return true;
       };
       bool ok = mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit);
-      for (int t = 0; ok && t < kSBufs && t < n; ++t) ok = issue_qk(t);
+      for (int t = 0; ok && t < kSBufs && t < n; ++t) {
+        ok = mbar_wait_bounded(&bars[B_K_FULL + t], 0, s_abort, kWaitLimit);
+        if (!ok) break;
+        tc_fence_after();
+        issue_qk(t);
+      }
+      // One wait per tile: PV_READY_i completes once P_i is stored and V_i
+      // and K_{i+3} have landed (the softmax warpgroup checks the copies
+      // before it arrives).  Then O += P_i V_i, and S_{i+3} = Q K_{i+3}^T
+      // into the buffer P_i V_i has just read.
       for (int i = 0; ok && i < n; ++i) {
-        // O += P_i V_i once P_i is stored and V_i landed.
         const int sl = i % kVSlots;
         ok = mbar_wait_bounded(&bars[B_PV_READY + sl], (i / kVSlots) & 1, s_abort, kWaitLimit);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm + L::kV + sl * kTileBytes);
         const uint32_t p_col = tmem + (i % kSBufs) * 128;
+        const uint64_t v_desc = desc_add(v_desc0, sl * kSlot16);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
-          tc_mma_ts(tmem + kColO, p_col + kk * 8, smem_desc(v_addr + kk * 2048, kBlk * 128, 1024),
-                    kIdPV, (i > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + kColO, p_col + kk * 8, desc_add(v_desc, (kk * 2048) >> 4), kIdPV,
+                    (i > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&bars[B_V_EMPTY + sl]);
         tc_commit(&bars[B_O_READY + (i & 1)]);
-        if (i + kSBufs < n) ok = issue_qk(i + kSBufs);
+        if (i + kSBufs < n) issue_qk(i + kSBufs);
       }
       if (!ok) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
@@ -386,20 +419,28 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
       // P (bf16 pairs) overwrites the S buffer it was computed from, 32 keys
       // at a time: TMEM columns s_col + [0, 64) then hold P row r.
-      float rq[4] = {0.f, 0.f, 0.f, 0.f};
+      // Pairs of columns go through two-wide FMA / add; the running sums
+      // are the four partial sums of columns = 0, 1, 2, 3 (mod 4).
+      const uint64_t scale2 = f2_pack(a.scale_log2, a.scale_log2);
+      const uint64_t neg_m2 = f2_pack(-m_t, -m_t);
+      uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
       for (int q = 0; q < kBlk / 32; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float e0 = ex2_approx(fmaf(s[32 * q + 2 * c], a.scale_log2, -m_t));
-          const float e1 = ex2_approx(fmaf(s[32 * q + 2 * c + 1], a.scale_log2, -m_t));
-          rq[(2 * c) & 3] += e0;
-          rq[(2 * c + 1) & 3] += e1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[32 * q + 2 * c], s[32 * q + 2 * c + 1]), scale2, neg_m2), x0,
+                    x1);
+          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+          acc2[c & 1] = f2_add(acc2[c & 1], f2_pack(e0, e1));
           pk[c] = pack_bf16x2(e0, e1);
         }
         if (ok) tmem_st16u(tmem + lane_base + s_col + 16 * q, pk);
       }
+      float rq[4];
+      f2_unpack(acc2[0], rq[0], rq[1]);
+      f2_unpack(acc2[1], rq[2], rq[3]);
       const float rs = (rq[0] + rq[1]) + (rq[2] + rq[3]);
       if (m_t != m_last) {  // m_last = -inf scales the empty sum 0 by 0
         l *= ex2_approx(m_last - m_t);
@@ -432,6 +473,19 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tmem_st32(tmem + lane_base + kColO + c * 32, o);
           }
         }
+      }
+      // Before releasing the tile to the MMA thread: V_t and K_{t+3} (the
+      // next product into this S buffer) have landed.  This warpgroup waits
+      // for K slot t % 3 and V slot t % 3 only at tiles t, t + 6, ..., and the
+      // tile three earlier on the same slots was released (by the other
+      // warpgroup) only after its own copies landed, so each parity is exact.
+      if (ok) {
+        bool landed = mbar_wait_bounded(&bars[B_V_FULL + t % kVSlots], (t / kVSlots) & 1, s_abort,
+                                        kWaitLimit);
+        if (landed && t + kSBufs < n)
+          landed = mbar_wait_bounded(&bars[B_K_FULL + t % kKSlots], ((t / kKSlots) + 1) & 1,
+                                     s_abort, kWaitLimit);
+        ok = __all_sync(0xffffffffu, landed);
       }
       tc_wait_st();
       tc_fence_before();

@@ -288,6 +288,14 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
+// Advance a shared-memory descriptor by `units16` 16-byte units.  The start
+// address field (bits 0-13) holds address / 16 of a shared-memory address
+// below 256 KB, so the sum never carries out of the low word.
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t units16) {
+  const uint32_t lo = static_cast<uint32_t>(d) + units16;
+  return (static_cast<uint64_t>(static_cast<uint32_t>(d >> 32)) << 32) | lo;
+}
+
 // Instruction descriptor of tcgen05.mma kind::f16: bf16 x bf16 -> fp32,
 // A K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
