@@ -417,7 +417,7 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         named_bar_arrive(bar_out, 64);
       }
 
-      // P (bf16 pairs) overwrites the S buffer it was computed from, 32 keys
+      // P (bf16 pairs) overwrites the S buffer it was computed from, 64 keys
       // at a time: TMEM columns s_col + [0, 64) then hold P row r.
       // Pairs of columns go through two-wide FMA / add; the running sums
       // are the four partial sums of columns = 0, 1, 2, 3 (mod 4).
@@ -425,18 +425,18 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint64_t neg_m2 = f2_pack(-m_t, -m_t);
       uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-      for (int q = 0; q < kBlk / 32; ++q) {
-        uint32_t pk[16];
+      for (int q = 0; q < kBlk / 64; ++q) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < 32; ++c) {
           float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[32 * q + 2 * c], s[32 * q + 2 * c + 1]), scale2, neg_m2), x0,
+          f2_unpack(f2_fma(f2_pack(s[64 * q + 2 * c], s[64 * q + 2 * c + 1]), scale2, neg_m2), x0,
                     x1);
           const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
           acc2[c & 1] = f2_add(acc2[c & 1], f2_pack(e0, e1));
           pk[c] = pack_bf16x2(e0, e1);
         }
-        if (ok) tmem_st16u(tmem + lane_base + s_col + 16 * q, pk);
+        if (ok) tmem_st32u(tmem + lane_base + s_col + 32 * q, pk);
       }
       float rq[4];
       f2_unpack(acc2[0], rq[0], rq[1]);
