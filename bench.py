@@ -93,6 +93,13 @@ def measured_traffic(kernel: str):
         return None
 
 
+def append_traffic():
+    """DRAM bytes of one append: the K/V reorder launch plus the block-mean
+    launch, or None unless both captures match the current sources."""
+    parts = [measured_traffic("reorder_kernel<16,1>"), measured_traffic("block_mean_kernel<16>")]
+    return None if None in parts else sum(parts)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -509,8 +516,7 @@ def run_ours(args, rank, world, local, pg):
                    "frac_of_hbm": round(st.append_bytes() / (phase_ms["append"] * 1e-3) / 1e9
                                         / peaks["hbm_gbs"], 4),
                    "bytes_per_call": int(st.append_bytes()),
-                   "traffic": (measured_traffic("reorder_kernel<16,1>")
-                               if args.chunk == CHUNK else None)},
+                   "traffic": (append_traffic() if args.chunk == CHUNK else None)},
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
