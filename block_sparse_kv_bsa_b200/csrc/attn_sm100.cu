@@ -17,30 +17,30 @@
 //   [384, 384+D)                 O accumulator (fp32)
 // Q (128 x D bf16) stays in shared memory for the whole work item and is the
 // A operand of Q K^T; V is the B operand of P V (A from tensor memory).
-// Three S buffers let the Q K^T of tile t + 3 follow the P V of tile t, so
-// S_t is ready two product groups before the tensor core needs P_t, and the
-// softmax of one tile overlaps the products of the next two.  Writing P
-// over its own S buffer relies on the tcgen05.mma operations of one thread
-// executing in issue order: the P V of tile t reads the buffer before the
-// Q K^T of tile t + 3, issued after it, overwrites it.
+// Three S buffers let the Q K^T of tile t + 3 run as soon as the P V of
+// tile t has read P_t, so S_t is ready well before the tensor core needs
+// P_t, and the softmax of one tile overlaps the products of the next two.
 //
-// Warp roles:
+// Warp roles (384 threads):
 //   warp 0      TMA producer: Q once, then the K tile (three-slot K ring) and
 //               the V tile (three-slot V ring) of each selected block, 128
 //               rows x D bf16 in 128-byte swizzled boxes of 64 columns; K runs
 //               two tiles ahead of V, the order in which the products consume
 //               them.  Tile row = ((b*Hh + h)*max_blocks + blk)*128.
-//   warp 1      allocates tensor memory; one lane issues tcgen05.mma.  Per
-//               tile it waits once, for one barrier that the softmax
-//               warpgroup completes after storing P_t and seeing V_t and
-//               K_{t+3} land; it then issues O += P_t V_t and S_{t+3} =
-//               Q K_{t+3}^T.  Operand descriptors are built once per CTA.
-//               The tensor pipe is fed only as fast as this one thread
-//               issues: each wait it executes, and every instruction it
+//   warp 1      allocates tensor memory; one lane issues O += P_t V_t once
+//               the softmax warpgroup has stored P_t and seen V_t land (one
+//               barrier per tile).
+//   warp 2      one lane issues S_t = Q K_t^T once K_t has landed and the
+//               P V of tile t - 3 (which read P from the same buffer) is done.
+//               The tensor pipe is fed only as fast as its issuing threads
+//               issue: a wait in an issuing thread, and every instruction it
 //               shares issue slots with, costs tensor time (measured: ~190
 //               SM cycles per wait per tile, and as much again from busy
-//               warps on the same SM).
-//   warps 2-9   softmax: warpgroup g (warps 2-5, 6-9) takes every other tile
+//               warps on the same SM).  Two issuers on two SM sub-partitions
+//               keep work queued while one of them waits.  Operand
+//               descriptors are built once per CTA.
+//   warp 3      idle (keeps the softmax warpgroups aligned to lane windows).
+//   warps 4-11  softmax: warpgroup g (warps 4-7, 8-11) takes every other tile
 //               t = g, g + 2, ...; a thread owns one query row.  Per tile it
 //               loads S, masks the pad keys of a tail block, takes the row
 //               maximum, receives the reference maximum of tile t - 1 from
@@ -64,7 +64,7 @@
 namespace bsa {
 
 constexpr int kSoftmaxThreads = 256;  // two warpgroups, one per tile parity
-constexpr int kAttnThreads = 64 + kSoftmaxThreads;
+constexpr int kAttnThreads = 128 + kSoftmaxThreads;  // producer, PV issuer, QK issuer, spare
 constexpr int kKSlots = 3;            // K ring
 constexpr int kVSlots = 3;            // V ring
 constexpr int kSBufs = 3;             // S / P buffers in tensor memory
@@ -84,8 +84,9 @@ enum {
   B_PV_READY = B_V_EMPTY + kVSlots,   // + slot t % 3: P_t stored, V_t and K_{t+3} landed
   B_S_FULL = B_PV_READY + kVSlots,    // + warpgroup: S of its next tile ready
   B_O_READY = B_S_FULL + 2,           // + tile parity: the P V of that tile is done
-  B_MMA_DONE = B_O_READY + 2,
-  B_COUNT
+  B_MMA_DONE = B_O_READY + 2,         // + issuer (0: P V thread, 1: Q K^T thread)
+  B_MMA_DONE_END = B_MMA_DONE + 2,
+  B_COUNT = B_MMA_DONE_END
 };
 
 template <int D>
@@ -272,68 +273,67 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mbar_wait_bounded(&bars[B_V_FULL + sl], (last / kVSlots) & 1, nullptr, kWaitLimit);
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers ----------------
+    // Warp 1 issues O += P_t V_t, warp 2 issues S_t = Q K_t^T: two threads on
+    // two SM sub-partitions, so that one's waits do not leave the tensor pipe
+    // without queued work.  Q K^T_t overwrites the S buffer whose P the
+    // P V of tile t - 3 read, so it waits for that P V to complete.
     if (lane == 0 && n > 0) {
-      constexpr uint32_t kIdQK = idesc_bf16(128, 128, 0);
-      constexpr uint32_t kIdPV = idesc_bf16(128, D, 1);
-      // Descriptors of every operand tile, built once; a k-step only adds
-      // its byte offset / 16 to the start-address field.
-      // Slots are kTileBytes apart, so slot sl adds sl * kTileBytes / 16.
-      const uint64_t q_desc = smem_desc(smem_u32(sm + L::kQ), 16, 1024);
-      const uint64_t k_desc0 = smem_desc(smem_u32(sm + L::kK), 16, 1024);
-      const uint64_t v_desc0 = smem_desc(smem_u32(sm + L::kV), kBlk * 128, 1024);
       constexpr uint32_t kSlot16 = kTileBytes >> 4;
-      // S_t = Q K_t^T into buffer t % 3 from K slot t % 3.
-      auto issue_qk = [&](int t) {
-        const int sl = t % kKSlots;
-        const uint64_t k_desc = desc_add(k_desc0, sl * kSlot16);
+      bool ok = true;
+      if (warp == 2) {
+        constexpr uint32_t kIdQK = idesc_bf16(128, 128, 0);
+        const uint64_t q_desc = smem_desc(smem_u32(sm + L::kQ), 16, 1024);
+        const uint64_t k_desc0 = smem_desc(smem_u32(sm + L::kK), 16, 1024);
+        ok = mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit);
+        for (int t = 0; ok && t < n; ++t) {
+          const int sl = t % kKSlots;
+          ok = mbar_wait_bounded(&bars[B_K_FULL + sl], (t / kKSlots) & 1, s_abort, kWaitLimit);
+          if (ok && t >= kSBufs)
+            ok = mbar_wait_bounded(&bars[B_V_EMPTY + t % kVSlots], ((t / kVSlots) - 1) & 1,
+                                   s_abort, kWaitLimit);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t k_desc = desc_add(k_desc0, sl * kSlot16);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * (kBlk * 128) + (kk % 4) * 32) >> 4;
-          tc_mma_ss(tmem + (t % kSBufs) * 128, desc_add(q_desc, off), desc_add(k_desc, off),
-                    kIdQK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * (kBlk * 128) + (kk % 4) * 32) >> 4;
+            tc_mma_ss(tmem + (t % kSBufs) * 128, desc_add(q_desc, off), desc_add(k_desc, off),
+                      kIdQK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars[B_K_EMPTY + sl]);
+          tc_commit(&bars[B_S_FULL + (t & 1)]);
         }
-        tc_commit(&bars[B_K_EMPTY + sl]);
-        tc_commit(&bars[B_S_FULL + (t & 1)]);
-      };
-      bool ok = mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit);
-      for (int t = 0; ok && t < kSBufs && t < n; ++t) {
-        ok = mbar_wait_bounded(&bars[B_K_FULL + t], 0, s_abort, kWaitLimit);
-        if (!ok) break;
-        tc_fence_after();
-        issue_qk(t);
-      }
-      // One wait per tile: PV_READY_i completes once P_i is stored and V_i
-      // and K_{i+3} have landed (the softmax warpgroup checks the copies
-      // before it arrives).  Then O += P_i V_i, and S_{i+3} = Q K_{i+3}^T
-      // into the buffer P_i V_i has just read.
-      for (int i = 0; ok && i < n; ++i) {
-        const int sl = i % kVSlots;
-        ok = mbar_wait_bounded(&bars[B_PV_READY + sl], (i / kVSlots) & 1, s_abort, kWaitLimit);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t p_col = tmem + (i % kSBufs) * 128;
-        const uint64_t v_desc = desc_add(v_desc0, sl * kSlot16);
+      } else {
+        constexpr uint32_t kIdPV = idesc_bf16(128, D, 1);
+        const uint64_t v_desc0 = smem_desc(smem_u32(sm + L::kV), kBlk * 128, 1024);
+        for (int i = 0; ok && i < n; ++i) {
+          const int sl = i % kVSlots;
+          ok = mbar_wait_bounded(&bars[B_PV_READY + sl], (i / kVSlots) & 1, s_abort, kWaitLimit);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t p_col = tmem + (i % kSBufs) * 128;
+          const uint64_t v_desc = desc_add(v_desc0, sl * kSlot16);
 #pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk) {
-          tc_mma_ts(tmem + kColO, p_col + kk * 8, desc_add(v_desc, (kk * 2048) >> 4), kIdPV,
-                    (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBlk / 16; ++kk) {
+            tc_mma_ts(tmem + kColO, p_col + kk * 8, desc_add(v_desc, (kk * 2048) >> 4), kIdPV,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&bars[B_V_EMPTY + sl]);
+          tc_commit(&bars[B_O_READY + (i & 1)]);
         }
-        tc_commit(&bars[B_V_EMPTY + sl]);
-        tc_commit(&bars[B_O_READY + (i & 1)]);
-        if (i + kSBufs < n) issue_qk(i + kSBufs);
       }
       if (!ok) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
         *s_abort = 1;
       }
       // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      tc_commit(&bars[B_MMA_DONE]);
-      mbar_wait_bounded(&bars[B_MMA_DONE], 0, nullptr, kWaitLimit);
+      tc_commit(&bars[B_MMA_DONE + (warp - 1)]);
+      mbar_wait_bounded(&bars[B_MMA_DONE + (warp - 1)], 0, nullptr, kWaitLimit);
     }
-  } else {
-    // ---------------- softmax / epilogue (warps 2..9) ----------------
+  } else if (warp >= 4) {
+    // ---------------- softmax / epilogue (warps 4..11) ----------------
     // The reference maximum m_t of tile t is decided in tile order: the
     // thread of row r in the warpgroup of tile t - 1 hands m_{t-1} to the
     // thread of row r in the other warpgroup through shared memory and a
@@ -341,7 +341,7 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // bar.sync).  Both warpgroups thus exponentiate against the same
     // reference as O.  Each keeps its own running sum, expressed in the last
     // reference it used; the two are merged in the epilogue.
-    const int g = (warp - 2) >> 2;           // warpgroup: 0 or 1
+    const int g = (warp - 4) >> 2;           // warpgroup: 0 or 1
     const int wq = warp & 3;                 // TMEM lane window of this warp
     const int r = wq * 32 + lane;            // query row owned by this thread
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
@@ -480,12 +480,8 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // tile three earlier on the same slots was released (by the other
       // warpgroup) only after its own copies landed, so each parity is exact.
       if (ok) {
-        bool landed = mbar_wait_bounded(&bars[B_V_FULL + t % kVSlots], (t / kVSlots) & 1, s_abort,
-                                        kWaitLimit);
-        if (landed && t + kSBufs < n)
-          landed = mbar_wait_bounded(&bars[B_K_FULL + t % kKSlots], ((t / kKSlots) + 1) & 1,
-                                     s_abort, kWaitLimit);
-        ok = __all_sync(0xffffffffu, landed);
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_V_FULL + t % kVSlots],
+                                                       (t / kVSlots) & 1, s_abort, kWaitLimit));
       }
       tc_wait_st();
       tc_fence_before();
