@@ -178,6 +178,107 @@ static bsa_status launch_block_means(const bsa_kv_cache* c, int first, int count
   return launch_status();
 }
 
+// Fused append for chunks of up to kGatherMaxTokens tokens: one CTA per
+// (chunk block, group of kAppendHeads heads, batch) gathers the block's 128
+// curve slots from the token-major K and V and writes whole cache rows; each
+// K warp owns one head and pools the block's key rows with the router's
+// summation (pool.cuh) while it moves them, so the pooled-key cache costs
+// no second pass over K.  The CTA inverts the caller's permutation for its
+// own slots by scanning it (perm is small and L2-resident at these sizes).
+constexpr int kAppendHeads = 4;
+constexpr int kAppendThreads = 2 * kAppendHeads * 32;  // K warps, then V warps
+constexpr int kGatherMaxTokens = 1 << 14;
+
+struct AppendArgs {
+  const uint4* k_tok;
+  const uint4* v_tok;
+  uint4* kc;
+  uint4* vc;
+  float* kmean;         // optional
+  const int32_t* perm;
+  int32_t* block_valid;
+  int32_t* d_err;
+  int N, Hh, max_blocks, base_block;
+};
+
+template <int VPR>
+__global__ void __launch_bounds__(kAppendThreads)
+append_gather_kernel(AppendArgs a) {
+  constexpr int D = VPR * 8;
+  __shared__ int s_tok[kBlk];
+  const int j = blockIdx.x;
+  const int b = blockIdx.z;
+  const int slot0 = j * kBlk;
+  const int valid = min(kBlk, a.N - slot0);
+  const bool first_cta = blockIdx.y == 0 && b == 0;
+  if (threadIdx.x < kBlk) s_tok[threadIdx.x] = -1;
+  __syncthreads();
+  // Slot -> token for this block's slots, scanning perm in rounds of
+  // kScan independent loads per thread (one L2 round trip per round).
+  constexpr int kScan = 16;
+  for (int base = 0; base < a.N; base += kScan * kAppendThreads) {
+    int pv[kScan];
+#pragma unroll
+    for (int k = 0; k < kScan; ++k) {
+      const int r = base + threadIdx.x + k * kAppendThreads;
+      pv[k] = r < a.N ? __ldg(a.perm + r) : 0;
+    }
+#pragma unroll
+    for (int k = 0; k < kScan; ++k) {
+      const int r = base + threadIdx.x + k * kAppendThreads;
+      if (r >= a.N) break;
+      const int p = pv[k];
+      if (p < 0 || p >= a.N) {
+        if (j == 0 && first_cta) report(a.d_err, BSA_DEV_BAD_PERM);
+        continue;
+      }
+      const unsigned d = static_cast<unsigned>(p - slot0);
+      if (d < static_cast<unsigned>(kBlk)) s_tok[d] = r;
+    }
+  }
+  __syncthreads();
+  if (first_cta && threadIdx.x == 0) a.block_valid[a.base_block + j] = valid;
+  // A slot of the chunk that no token maps to: perm is not a permutation.
+  if (first_cta && threadIdx.x < valid && s_tok[threadIdx.x] < 0) report(a.d_err, BSA_DEV_BAD_PERM);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const bool is_k = warp < kAppendHeads;
+  const int h = blockIdx.y * kAppendHeads + (is_k ? warp : warp - kAppendHeads);
+  if (h >= a.Hh) return;
+  const int c = lane % VPR, g = lane / VPR;
+  const long long tok_stride = static_cast<long long>(a.Hh) * VPR;  // vectors per token
+  const long long tok_base = static_cast<long long>(b) * a.N * tok_stride +
+                             static_cast<long long>(h) * VPR + c;
+  const long long bh = static_cast<long long>(b) * a.Hh + h;
+  const long long blk = bh * a.max_blocks + a.base_block + j;
+  const uint4* src = is_k ? a.k_tok : a.v_tok;
+  uint4* dst = (is_k ? a.kc : a.vc) + blk * kBlk * VPR + c;
+  // Rows at or past `valid` are the block's zero pad rows.
+  auto load = [&](int row) {
+    const int tok = s_tok[row];
+    return tok >= 0 ? ld_nc_v4(src + tok_base + static_cast<long long>(tok) * tok_stride)
+                    : make_uint4(0, 0, 0, 0);
+  };
+  auto store = [&](int row, uint4 x) { st_v4(dst + row * VPR, x); };
+  float acc[8];
+  warp_colsum_rows<VPR>(load, store, valid, g, acc);
+  if (is_k && a.kmean != nullptr && g == 0) {
+    float4* out = reinterpret_cast<float4*>(a.kmean + blk * D + c * 8);
+    const float inv = static_cast<float>(valid);
+    out[0] = make_float4(acc[0] / inv, acc[1] / inv, acc[2] / inv, acc[3] / inv);
+    out[1] = make_float4(acc[4] / inv, acc[5] / inv, acc[6] / inv, acc[7] / inv);
+  }
+}
+
+static bsa_status launch_append_gather(const AppendArgs& a, int B, int D, int nb, cudaStream_t s) {
+  dim3 grid(nb, (a.Hh + kAppendHeads - 1) / kAppendHeads, B);
+  if (D == 128)
+    append_gather_kernel<16><<<grid, kAppendThreads, 0, s>>>(a);
+  else
+    append_gather_kernel<8><<<grid, kAppendThreads, 0, s>>>(a);
+  return launch_status();
+}
+
 static bsa_status check_chunk(int B, int Hh, int D, int T, int H, int W) {
   if (B <= 0 || Hh <= 0 || T <= 0 || H <= 0 || W <= 0) return BSA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return BSA_ERR_UNSUPPORTED;
@@ -235,23 +336,42 @@ extern "C" bsa_status bsa_kv_append(bsa_kv_cache* c, const void* k_tok, const vo
   const int nb = (n + kBlk - 1) / kBlk;
   if (c->n_blocks + nb > c->max_blocks) return BSA_ERR_CAPACITY;
   if (c->kmean != nullptr && !aligned16(c->kmean)) return BSA_ERR_INVALID_ARG;
-  ReorderArgs a{};
-  a.src0 = static_cast<const uint4*>(k_tok);
-  a.dst0 = static_cast<uint4*>(c->k);
-  a.src1 = static_cast<const uint4*>(v_tok);
-  a.dst1 = static_cast<uint4*>(c->v);
-  a.perm = d_perm;
-  a.block_valid = c->block_valid;
-  a.d_err = d_err;
-  a.N = n;
-  a.nb = nb;
-  a.B = c->B;
-  a.Hh = c->Hh;
-  a.blk_stride = c->max_blocks;
-  a.base_block = c->n_blocks;
-  st = launch_reorder<true>(a, c->D, as_stream(stream));
-  if (st == BSA_OK && c->kmean != nullptr)
-    st = launch_block_means(c, c->n_blocks, nb, d_err, as_stream(stream));
+  if (n <= kGatherMaxTokens) {
+    // One pass: gather into whole cache rows, pooling the keys on the way.
+    AppendArgs g{};
+    g.k_tok = static_cast<const uint4*>(k_tok);
+    g.v_tok = static_cast<const uint4*>(v_tok);
+    g.kc = static_cast<uint4*>(c->k);
+    g.vc = static_cast<uint4*>(c->v);
+    g.kmean = c->kmean;
+    g.perm = d_perm;
+    g.block_valid = c->block_valid;
+    g.d_err = d_err;
+    g.N = n;
+    g.Hh = c->Hh;
+    g.max_blocks = c->max_blocks;
+    g.base_block = c->n_blocks;
+    st = launch_append_gather(g, c->B, c->D, nb, as_stream(stream));
+  } else {
+    // Large chunks: scatter K and V, then pool the new blocks.
+    ReorderArgs a{};
+    a.src0 = static_cast<const uint4*>(k_tok);
+    a.dst0 = static_cast<uint4*>(c->k);
+    a.src1 = static_cast<const uint4*>(v_tok);
+    a.dst1 = static_cast<uint4*>(c->v);
+    a.perm = d_perm;
+    a.block_valid = c->block_valid;
+    a.d_err = d_err;
+    a.N = n;
+    a.nb = nb;
+    a.B = c->B;
+    a.Hh = c->Hh;
+    a.blk_stride = c->max_blocks;
+    a.base_block = c->n_blocks;
+    st = launch_reorder<true>(a, c->D, as_stream(stream));
+    if (st == BSA_OK && c->kmean != nullptr)
+      st = launch_block_means(c, c->n_blocks, nb, d_err, as_stream(stream));
+  }
   if (st == BSA_OK) c->n_blocks += nb;
   return st;
 }

@@ -157,3 +157,77 @@ def test_pool_means_for_directly_written_blocks():
     assert np.allclose(cache.kmean[:, [0, 23]].cpu().double().numpy(), exp, rtol=2e-6, atol=2e-7)
     with pytest.raises(bsa.BsaError):
         bsa.bsa_kv_pool_means(cache, 15, 10)       # past max_blocks
+
+
+def _append_raw(cache, k, v, T, H, W, perm):
+    import ctypes
+    cs = cache.c_struct()
+    st = bsa.lib().bsa_kv_append(ctypes.byref(cs), ctypes.c_void_p(k.data_ptr()),
+                                 ctypes.c_void_p(v.data_ptr()), T, H, W,
+                                 ctypes.c_void_p(perm.data_ptr()),
+                                 ctypes.c_void_p(bsa.error_word(DEV).data_ptr()),
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    cache.n_blocks = int(cs.n_blocks)
+
+
+def test_append_any_permutation():
+    # The ABI accepts any permutation of the chunk's tokens, not only the
+    # Gilbert table: token i lands in curve slot perm[i] (block perm[i] / 128,
+    # row perm[i] % 128), every head, pads zero.
+    w = synth.CONFIGS[2]
+    T, H, W = w.grid
+    N = T * H * W
+    nb = w.blocks_per_chunk
+    perm_np = np.random.default_rng(7).permutation(N).astype(np.int32)
+    perm = torch.from_numpy(perm_np).to(DEV)
+    cache = bsa.KVCache(w.B, w.Hh, w.D, nb, device=DEV, pooled_keys=True)
+    t = synth.chunk_tokens(w, 1, device=DEV, want=("k", "v"))
+    _append_raw(cache, t["k"], t["v"], T, H, W, perm)
+    bsa.raise_on_device_error(DEV)
+    for name in ("k", "v"):
+        x = t[name].cpu()                                   # [B, N, Hh, D]
+        exp = torch.zeros(w.B, w.Hh, nb * 128, w.D, dtype=torch.bfloat16)
+        exp[:, :, torch.from_numpy(perm_np).long()] = x.permute(0, 2, 1, 3)
+        got = getattr(cache, name).cpu().reshape(w.B, w.Hh, nb * 128, w.D)
+        assert torch.equal(got.view(torch.int16), exp.view(torch.int16)), name
+    valid = cache.block_valid.cpu().numpy()
+    exp_m = oracle.pool_blocks(cache.k.cpu().double().numpy(), valid)
+    assert np.allclose(cache.kmean.cpu().double().numpy(), exp_m, rtol=2e-6, atol=2e-7)
+
+
+@pytest.mark.parametrize("key", [1, 2, 4])
+def test_append_means_equal_pool_means_bitwise(key):
+    # The append pools the keys while it moves them, with the router's own
+    # summation order: recomputing the means from the cache gives the same
+    # bits (and so the pooled and the streaming route score the same means).
+    w = synth.CONFIGS[key]
+    T, H, W = w.grid
+    nb = w.blocks_per_chunk
+    cache = bsa.KVCache(w.B, w.Hh, w.D, 2 * nb, device=DEV, pooled_keys=True)
+    for c in (1, 2):
+        t = synth.chunk_tokens(w, c, device=DEV, want=("k", "v"))
+        bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+    bsa.raise_on_device_error(DEV)
+    at_append = cache.kmean.clone()
+    bsa.bsa_kv_pool_means(cache, 0, 2 * nb)
+    bsa.raise_on_device_error(DEV)
+    assert torch.equal(cache.kmean.view(torch.int32), at_append.view(torch.int32))
+
+
+def test_append_large_chunk():
+    # Chunks above 16384 tokens take the scatter kernel and a separate pooling
+    # pass; the cache and the means are the same as the oracle's.
+    w = synth.Workload(90, "large-chunk", B=1, Hh=2, D=64, grid=(2, 96, 101))
+    T, H, W = w.grid
+    nb = w.blocks_per_chunk                                # 19392 tokens: 152 blocks, tail of 64
+    cache = bsa.KVCache(w.B, w.Hh, w.D, nb + 1, device=DEV, pooled_keys=True)
+    t = synth.chunk_tokens(w, 1, device=DEV, want=("k", "v"))
+    bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+    bsa.raise_on_device_error(DEV)
+    exp_k = oracle.tokens_to_blocks(t["k"].cpu().double().numpy(), T, H, W)
+    assert np.array_equal(bits(cache.k[:, :, :nb]), bf16_of(exp_k))
+    valid = cache.block_valid.cpu().numpy()
+    assert np.array_equal(valid[:nb], oracle.block_valid_for(T, H, W))
+    exp_m = oracle.pool_blocks(cache.k[:, :, :nb].cpu().double().numpy(), valid[:nb])
+    assert np.allclose(cache.kmean[:, :, :nb].cpu().double().numpy(), exp_m, rtol=2e-6, atol=2e-7)
