@@ -53,7 +53,7 @@ BLK = 128
 METRIC = "bsa_attn selected-block TFLOP/s at chunk 48 (48-chunk sweep), 1 B200"
 L2_FLUSH_BYTES = 256 << 20
 # append (scatter + key means), tokens->blocks, pool_q, pool_score, topk, attn, blocks->tokens
-KERNELS_PER_STEP = 8
+KERNELS_PER_STEP = 7  # append (fused), Q to blocks, pool_q, score_means, topk, attn, O to tokens
 
 
 def parse_args():
@@ -94,10 +94,9 @@ def measured_traffic(kernel: str):
 
 
 def append_traffic():
-    """DRAM bytes of one append: the K/V reorder launch plus the block-mean
-    launch, or None unless both captures match the current sources."""
-    parts = [measured_traffic("reorder_kernel<16,1>"), measured_traffic("block_mean_kernel<16>")]
-    return None if None in parts else sum(parts)
+    """DRAM bytes of one append (the fused gather + pooling launch), or None
+    unless the capture matches the current sources."""
+    return measured_traffic("append_gather_kernel<16>")
 
 
 def load_peaks():
