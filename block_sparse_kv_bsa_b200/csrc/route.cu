@@ -223,21 +223,42 @@ score_means_kernel(RouteArgs a) {
   const int h = blockIdx.y, b = blockIdx.z;
   const long long bh = static_cast<long long>(b) * a.Hh + h;
   const int n0 = blockIdx.x * kMeanTileN;
-  for (int i = threadIdx.x; i < nq * (D / 4); i += kMeanThreads) {
-    const int r = i / (D / 4), c4 = i % (D / 4);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < a.n_own) v = reinterpret_cast<const float4*>(a.qm + (bh * a.n_own + r) * D)[c4];
-    *reinterpret_cast<float4*>(qs + r * P + c4 * 4) = v;
-  }
-  for (int i = threadIdx.x; i < kMeanTileN * (D / 4); i += kMeanThreads) {
-    const int r = i / (D / 4), c4 = i % (D / 4);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (n0 + r < a.n_hist)
-      v = reinterpret_cast<const float4*>(a.kmean + (bh * a.max_blocks + n0 + r) * D)[c4];
-    *reinterpret_cast<float4*>(ks + r * P + c4 * 4) = v;
+  // Stage the query means and this tile's key means, kLoads independent
+  // 16-byte loads per thread in flight before any is stored.
+  constexpr int kLoads = 8;
+  const int n_q4 = nq * (D / 4), n_k4 = kMeanTileN * (D / 4);
+  for (int base = 0; base < n_q4 + n_k4; base += kLoads * kMeanThreads) {
+    float4 v[kLoads];
+#pragma unroll
+    for (int u = 0; u < kLoads; ++u) {
+      const int i = base + u * kMeanThreads + threadIdx.x;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < n_q4) {
+        const int r = i / (D / 4), c4 = i % (D / 4);
+        if (r < a.n_own) v[u] = ld_nc_f4(a.qm + (bh * a.n_own + r) * D + c4 * 4);
+      } else if (i < n_q4 + n_k4) {
+        const int r = (i - n_q4) / (D / 4), c4 = (i - n_q4) % (D / 4);
+        if (n0 + r < a.n_hist) v[u] = ld_nc_f4(a.kmean + (bh * a.max_blocks + n0 + r) * D + c4 * 4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kLoads; ++u) {
+      const int i = base + u * kMeanThreads + threadIdx.x;
+      if (i < n_q4) {
+        const int r = i / (D / 4), c4 = i % (D / 4);
+        *reinterpret_cast<float4*>(qs + r * P + c4 * 4) = v[u];
+      } else if (i < n_q4 + n_k4) {
+        const int r = (i - n_q4) / (D / 4), c4 = (i - n_q4) % (D / 4);
+        *reinterpret_cast<float4*>(ks + r * P + c4 * 4) = v[u];
+      }
+    }
   }
   __syncthreads();
-  const int tn = threadIdx.x % 16;               // history blocks tn*4 .. tn*4+3 of the tile
+  // History blocks tn, tn+16, tn+32, tn+48 of the tile: with rows P = D+4
+  // floats apart (an odd number of 16-byte units), the 8 lanes of a
+  // 16-byte-load phase hit 8 different bank groups, and the scores of
+  // consecutive lanes are consecutive in memory.
+  const int tn = threadIdx.x % 16;
   const int tj = threadIdx.x / 16;               // query blocks tj, tj+16, tj+32, ...
   for (int jb = 0; jb < nq; jb += 64) {
     float acc[4][4];
@@ -254,7 +275,7 @@ score_means_kernel(RouteArgs a) {
         q[x] = j < nq ? *reinterpret_cast<const float4*>(qs + j * P + d) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int y = 0; y < 4; ++y) k[y] = *reinterpret_cast<const float4*>(ks + (tn * 4 + y) * P + d);
+      for (int y = 0; y < 4; ++y) k[y] = *reinterpret_cast<const float4*>(ks + (tn + 16 * y) * P + d);
 #pragma unroll
       for (int x = 0; x < 4; ++x)
 #pragma unroll
@@ -271,7 +292,7 @@ score_means_kernel(RouteArgs a) {
       if (j >= a.n_own) continue;
 #pragma unroll
       for (int y = 0; y < 4; ++y) {
-        const int n = n0 + tn * 4 + y;
+        const int n = n0 + tn + 16 * y;
         if (n < a.n_hist) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * acc[x][y];
       }
     }
