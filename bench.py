@@ -52,7 +52,6 @@ CHUNK = 48
 BLK = 128
 METRIC = "bsa_attn selected-block TFLOP/s at chunk 48 (48-chunk sweep), 1 B200"
 L2_FLUSH_BYTES = 256 << 20
-# append (scatter + key means), tokens->blocks, pool_q, pool_score, topk, attn, blocks->tokens
 KERNELS_PER_STEP = 7  # append (fused), Q to blocks, pool_q, score_means, topk, attn, O to tokens
 
 
@@ -383,6 +382,56 @@ class State:
                 "constants": "tau 0.1, g_ref 0.2, lambda 2, eta_cov 0.9, K_cov 80, "
                              "K_unc 150, mass 0.9, window +/-13 in the previous chunk"}
 
+    def geometry_point(self, reps: int = 20) -> dict:
+        """The geometric prior computed on the GPU (bsa_geometry_prior: slab
+        boxes, separating-axis test, 8^3 grid IoU, coverage) from seeded
+        synthetic slabs of this chunk's history, timed; then the page's route
+        from that g and coverage, and bsa_attn on those routes."""
+        w, bsa = self.w, self.bsa
+        sc = synth.slab_scene(w.grid, self.n_hist // self.n_own, self.n_own,
+                              seed=1000 * w.key + 800 + CHUNK)
+
+        def dev(x, dtype):
+            return torch.from_numpy(np.ascontiguousarray(x)[None]).to(self.device, dtype)
+        t = {k: dev(getattr(sc, k), torch.float32) for k in ("cams", "h_rect", "q_rect", "tok_uvd")}
+        t.update({k: dev(getattr(sc, k), torch.int32) for k in ("h_cam", "q_cam", "tok_cam")})
+
+        def call():
+            return bsa.bsa_geometry_prior(t["cams"], sc.intr, t["h_cam"], t["h_rect"], t["q_cam"],
+                                          t["q_rect"], t["tok_cam"], t["tok_uvd"],
+                                          q_valid=self.q_valid, grid_n=8)
+        g, cov = call()
+        gt = _time_call(call, reps)
+        kw = dict(g=g, coverage=cov, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale, tau=0.1,
+                  eta_cov=0.9, k_cov=80, k_unc=150, mass=0.9,
+                  prev_first=self.own_first - self.n_own, n_prev=self.n_own, window_half=13,
+                  q_valid=self.q_valid, workspace=self.ws)
+        idx, cnt = bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist, self.own_first,
+                                       self.n_own, **kw)
+        o = torch.empty_like(self.q_blk)
+        lse = torch.empty_like(self.lse)
+        rt = _time_call(lambda: bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist,
+                                                    self.own_first, self.n_own, idx=idx,
+                                                    cnt=cnt, **kw), 10)
+        at = _time_call(lambda: bsa.bsa_attn(self.q_blk, self.cache, idx, cnt,
+                                             q_valid=self.q_valid, sm_scale=w.sm_scale, o=o,
+                                             lse=lse), 10)
+        bsa.raise_on_device_error(self.device)
+        c = cnt.to(torch.float64)
+        n_slab_pairs = int((t["q_cam"] >= 0).sum().item()) * int((t["h_cam"] >= 0).sum().item())
+        return {"prior_ms": round(gt, 4),
+                "slab_box_pairs": n_slab_pairs,
+                "token_slab_tests": int((t["tok_cam"] >= 0).sum().item()) *
+                int((t["h_cam"] >= 0).sum().item()),
+                "g_nonzero_frac": round(float((g > 0).double().mean().item()), 4),
+                "coverage_mean": round(float(cov.double().mean().item()), 4),
+                "route_ms": round(rt, 4), "attn_ms": round(at, 4),
+                "blocks_per_query_block": {"mean": round(float(c.mean().item()), 1),
+                                           "min": int(c.min().item()),
+                                           "max": int(c.max().item())},
+                "scene": "seeded synthetic slabs: camera trajectory, wall at z=14, "
+                         "foreground objects; grid 8^3"}
+
     def route_stream_ms(self, flush, reps: int = 20) -> float:
         """bsa_route timed without the pooled-key cache, i.e. streaming every
         history key block (L2 flushed before each call)."""
@@ -463,6 +512,7 @@ def run_ours(args, rank, world, local, pg):
 
     route_stream = st.route_stream_ms(flush)
     velox = st.velox_point(flush) if rank == 0 else None
+    geometry = st.geometry_point() if rank == 0 else None
     if rank == 0 and st.sweep is not None and args.sweep:
         st.sweep.append(sweep_point(st.bsa, w, st.cache, st.q_tok, args.chunk, st.own_first,
                                     st.n_own, device))
@@ -527,6 +577,7 @@ def run_ours(args, rank, world, local, pg):
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "sweep": st.sweep,
         "velox_route": velox,
+        "geometry_prior": geometry,
         "clocks": clock_info,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -46,6 +46,7 @@ EXPORTS = ("bsa_abi_version", "bsa_status_string", "bsa_gilbert_perm", "bsa_kv_a
            "bsa_kv_pool_means",
            "bsa_tokens_to_blocks", "bsa_blocks_to_tokens", "bsa_route_workspace_size",
            "bsa_route", "bsa_route_velox", "bsa_route_noalloc", "bsa_attn",
+           "bsa_geometry_prior",
            "bsa_check_device_error",
            "bsa_selftest_bounded_wait")
 
@@ -97,6 +98,8 @@ _sig = {
     "bsa_route_workspace_size": (_i, [_i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "bsa_route": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f, _i,
                        _p, _p, _i, _p, _sz, _p, _p]),
+    "bsa_geometry_prior": (_i, [_p, _i, _f, _f, _f, _f, _p, _p, _i, _p, _p, _i, _i, _i, _p, _p,
+                                _p, _i, _p, _p, _p, _p]),
     "bsa_route_velox": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f,
                              ctypes.POINTER(CVeloxRoute), _p, _p, _i, _p, _sz, _p, _p]),
     "bsa_route_noalloc": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f, _i,
@@ -400,6 +403,53 @@ def bsa_route_velox(q_blk: torch.Tensor, cache: KVCache, n_hist: int, own_first:
         _ptr(cnt), int(max_sel), _ptr(workspace), workspace.numel(), _ptr(error_word(dev)),
         _stream(dev)))
     return idx, cnt
+
+
+def bsa_geometry_prior(cams: torch.Tensor, intr, h_cam: torch.Tensor, h_rect: torch.Tensor,
+                       q_cam: Optional[torch.Tensor] = None, q_rect: Optional[torch.Tensor] = None,
+                       tok_cam: Optional[torch.Tensor] = None,
+                       tok_uvd: Optional[torch.Tensor] = None,
+                       q_valid: Optional[torch.Tensor] = None, grid_n: int = 8,
+                       g: Optional[torch.Tensor] = None, coverage: Optional[torch.Tensor] = None,
+                       want_g: bool = True, want_coverage: bool = True):
+    """Overlap prior g [B, n_q, n_hist] and coverage [B, n_q] from slabs.
+
+    cams float32 [B, n_cams, 12]; intr = (fx, fy, cx, cy); h_cam int32
+    [B, n_hist, S], h_rect float32 [B, n_hist, S, 6]; q_cam/q_rect likewise
+    for the query blocks (needed for g); tok_cam int32 [B, n_q, 128] and
+    tok_uvd float32 [B, n_q, 128, 3] (needed for coverage).  Returns (g,
+    coverage), either None when not requested."""
+    dev = _dev(cams.device)
+    B, n_cams = cams.shape[0], cams.shape[1]
+    _need(cams, "cams", torch.float32, dev, (B, n_cams, 12))
+    n_hist, S = h_cam.shape[1], h_cam.shape[2]
+    _need(h_cam, "h_cam", torch.int32, dev, (B, n_hist, S))
+    _need(h_rect, "h_rect", torch.float32, dev, (B, n_hist, S, 6))
+    n_q = (q_cam if q_cam is not None else tok_cam).shape[1]
+    if want_g:
+        _need(q_cam, "q_cam", torch.int32, dev, (B, n_q, S))
+        _need(q_rect, "q_rect", torch.float32, dev, (B, n_q, S, 6))
+        if g is None:
+            g = torch.empty((B, n_q, n_hist), dtype=torch.float32, device=dev)
+        _need(g, "g", torch.float32, dev, (B, n_q, n_hist))
+    else:
+        g = None
+    if want_coverage:
+        _need(tok_cam, "tok_cam", torch.int32, dev, (B, n_q, BLK))
+        _need(tok_uvd, "tok_uvd", torch.float32, dev, (B, n_q, BLK, 3))
+        if coverage is None:
+            coverage = torch.empty((B, n_q), dtype=torch.float32, device=dev)
+        _need(coverage, "coverage", torch.float32, dev, (B, n_q))
+    else:
+        coverage = None
+    if q_valid is not None:
+        _need(q_valid, "q_valid", torch.int32, dev, (n_q,))
+    fx, fy, cx, cy = (float(v) for v in intr)
+    _check("bsa_geometry_prior", _lib.bsa_geometry_prior(
+        _ptr(cams), int(n_cams), fx, fy, cx, cy, _ptr(q_cam), _ptr(q_rect), int(n_q),
+        _ptr(h_cam), _ptr(h_rect), int(n_hist), int(S), int(grid_n), _ptr(tok_cam), _ptr(tok_uvd),
+        _ptr(q_valid), int(B), _ptr(g), _ptr(coverage), _ptr(error_word(dev)), _stream(dev)))
+    return g, coverage
 
 
 def bsa_attn(q_blk: torch.Tensor, cache: KVCache, idx: torch.Tensor, cnt: torch.Tensor,

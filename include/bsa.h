@@ -276,6 +276,48 @@ bsa_status bsa_route_velox(const void *q_blk, const bsa_kv_cache *cache, const i
                            void *workspace, size_t ws_bytes, int32_t *d_err, void *stream);
 
 /*
+ * Geometric overlap prior g and coverage from slabs (Velox, Methodology
+ * Step 3; slabs as in Step 1).  Each slab (a source-camera token rectangle
+ * [u0, u1] x [v0, v1] in pixel-edge coordinates plus a depth interval
+ * [d0, d1]) becomes the smallest box with its camera's axes that holds its
+ * frustum segment.  g[b, j, m] is the largest IoU between a valid slab box
+ * of query block j and one of history block m, each IoU estimated on an
+ * n x n x n grid of cell centres of the query box after a separating-axis
+ * test (0 when separated); the intersection is capped at the smaller box
+ * volume, so g is in [0, 1].  coverage[b, j] is the fraction of query block
+ * j's valid tokens (q_valid[j] of 128) whose back-projected point lies in a
+ * valid slab of any history block: depth in that slab's camera within
+ * [d0, d1], projection within its rectangle.  Tokens without depth count as
+ * uncovered.  All decisions are float32 with one rounding per operation in
+ * a fixed order, so the counts are reproducible.  g and coverage are the
+ * inputs bsa_route and bsa_route_velox take.
+ *   cams       device float32 [B, n_cams, 12]: R (3x3 row-major, world from
+ *              camera; camera axes x right, y down, z forward) then the
+ *              camera centre; pinhole intrinsics fx, fy, cx, cy (latent
+ *              pixels) shared by all cameras
+ *   q_cam      device int32 [B, n_q, S]: camera of each query slab, -1 = none
+ *   q_rect     device float32 [B, n_q, S, 6]: u0, u1, v0, v1, d0, d1
+ *   h_cam      device int32 [B, n_hist, S], h_rect [B, n_hist, S, 6]: history
+ *   S          slabs per block, 1..4;  grid_n  grid points per axis, 1..16
+ *   tok_cam    device int32 [B, n_q, 128]: camera of each query token, -1 =
+ *              no depth;  tok_uvd  device float32 [B, n_q, 128, 3]: u, v, d
+ *   q_valid    device int32 [n_q] valid tokens per query block, or NULL (128)
+ *   g          device float32 [B, n_q, n_hist] written, or NULL (skipped)
+ *   coverage   device float32 [B, n_q] written, or NULL (skipped)
+ * Errors: BSA_ERR_INVALID_ARG (null input for a requested output, both
+ *         outputs NULL, S or grid_n out of range, fx or fy not positive),
+ *         BSA_ERR_SHAPE, BSA_ERR_CUDA; on the device a camera index outside
+ *         [-1, n_cams) raises BSA_DEV_BAD_INDEX (the slab or token is then
+ *         absent) and a q_valid entry outside [0, 128] BSA_DEV_BAD_VALID.
+ */
+bsa_status bsa_geometry_prior(const float *cams, int n_cams, float fx, float fy, float cx,
+                              float cy, const int32_t *q_cam, const float *q_rect, int n_q,
+                              const int32_t *h_cam, const float *h_rect, int n_hist,
+                              int slabs_per_block, int grid_n, const int32_t *tok_cam,
+                              const float *tok_uvd, const int32_t *q_valid, int B, float *g,
+                              float *coverage, int32_t *d_err, void *stream);
+
+/*
  * bsa_route without a workspace argument, for callers that cannot allocate
  * device memory themselves: for example code running inside another
  * runtime's plugin or enqueue hook, where the host framework owns every

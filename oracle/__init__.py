@@ -7,6 +7,10 @@ shares no code with the CUDA library under ``block_sparse_kv_bsa_b200/``.
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 against closed forms, invariants, brute force on tiny inputs or textbook
 routines (see the test files); none is "parity unpinned".
+
+``oracle.geometry`` holds the overlap prior g and the coverage score
+(slab boxes, separating-axis test, grid IoU), in float32 with a fixed
+operation order because they decide counts.
 """
 from .gilbert import gilbert_cells, gilbert_perm  # noqa: F401
 from .bsa import (  # noqa: F401

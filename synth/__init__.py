@@ -13,3 +13,4 @@ from .workloads import (  # noqa: F401
     prior,
     random_bf16,
 )
+from .geometry import SlabScene, slab_scene  # noqa: F401
