@@ -26,7 +26,8 @@
 // prior_g_kernel: one thread per (history block, query block, batch); the
 //   query block's boxes are built once per CTA in shared memory.
 // coverage_kernel: one CTA per (query block, batch); 128 tokens x 4 slab
-//   groups, the history slabs staged through shared memory in tiles.
+//   groups, the history slabs staged through shared memory in tiles; the
+//   CTA stops once every token with depth has found a slab.
 #include "common.cuh"
 
 namespace bsa {
@@ -251,8 +252,9 @@ coverage_kernel(GeoArgs a) {
   if (grp == 0) s_hit[r] = 0;
   bool hit = false;
   const int n_slabs = a.n_hist * a.S;
+  // Tiles continue only while some token with depth is still uncovered.
   for (int base = 0; base < n_slabs; base += kCovTile) {
-    __syncthreads();   // the previous tile is no longer read
+    if (!__syncthreads_or(live && !hit)) break;   // also: the previous tile is no longer read
     for (int k = threadIdx.x; k < kCovTile; k += kCovThreads) {
       const int si = base + k;
       int ok = 0;
