@@ -25,10 +25,17 @@
 //
 // prior_g_kernel: one thread per (history block, query block, batch); the
 //   query block's boxes are built once per CTA in shared memory.
-// coverage_kernel: one CTA per (query block, batch); 128 tokens x 4 slab
-//   groups, the history slabs staged through shared memory in tiles; the
-//   CTA stops once every token with depth has found a slab.
+// coverage_kernel: a cluster of 4 CTAs per (query block, batch), each
+//   taking a quarter of the history slabs; per CTA 128 tokens x 4 slab
+//   groups test 512-slab tiles staged through shared memory (the next tile
+//   prefetched into registers); a CTA stops once every token with depth has
+//   found a slab; the first CTA ORs the token flags of the cluster through
+//   distributed shared memory.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace bsa {
 
@@ -37,7 +44,8 @@ constexpr int kGeoMaxGrid = 16;      // grid points per axis
 constexpr int kPriorThreads = 128;
 constexpr int kCovGroups = 4;
 constexpr int kCovThreads = kBlk * kCovGroups;
-constexpr int kCovTile = 128;        // history slabs per shared-memory tile
+constexpr int kCovTile = kCovThreads;  // history slabs per shared-memory tile (one per thread)
+constexpr int kCovSplit = 4;           // CTAs (one cluster) per query block
 constexpr float kSatEps = 1e-6f;
 
 struct Box {
@@ -219,17 +227,33 @@ struct CovSlab {
   float rect[6];
 };
 
-__global__ void __launch_bounds__(kCovThreads)
+// One history slab, fetched through its camera (invalid -> ok = 0).
+__device__ __forceinline__ int load_slab(const GeoArgs& a, const float* cams, long long hi, int cam,
+                                         CovSlab& out) {
+  if (cam < 0) return 0;
+  const float* C = cams + cam * 12;
+#pragma unroll
+  for (int e = 0; e < 9; ++e) out.R[e] = C[e];
+#pragma unroll
+  for (int e = 0; e < 3; ++e) out.c[e] = C[9 + e];
+#pragma unroll
+  for (int e = 0; e < 6; ++e) out.rect[e] = a.h_rect[hi * 6 + e];
+  return 1;
+}
+
+__global__ void __cluster_dims__(kCovSplit, 1, 1) __launch_bounds__(kCovThreads)
 coverage_kernel(GeoArgs a) {
   __shared__ CovSlab s_slab[kCovTile];
   __shared__ int s_ok[kCovTile];
   __shared__ int s_hit[kBlk];
-  const int j = blockIdx.x, b = blockIdx.y;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int part = static_cast<int>(cluster.block_rank());
+  const int j = blockIdx.x / kCovSplit, b = blockIdx.y;
   const int r = threadIdx.x % kBlk, grp = threadIdx.x / kBlk;
   const float* cams = a.cams + static_cast<long long>(b) * a.n_cams * 12;
   int nv = a.q_valid != nullptr ? a.q_valid[j] : kBlk;
   if (nv < 0 || nv > kBlk) {
-    report(a.d_err, BSA_DEV_BAD_VALID);
+    if (part == 0 && threadIdx.x == 0) report(a.d_err, BSA_DEV_BAD_VALID);
     nv = nv < 0 ? 0 : kBlk;
   }
   // This thread's token as a world point (if it has depth).
@@ -250,42 +274,40 @@ coverage_kernel(GeoArgs a) {
     }
   }
   if (grp == 0) s_hit[r] = 0;
-  bool hit = false;
+
+  // This CTA's share of the history slabs; one slab per thread per tile,
+  // the next tile fetched into registers while this one is tested (camera
+  // indices one tile further ahead).
   const int n_slabs = a.n_hist * a.S;
-  // Tiles continue only while some token with depth is still uncovered.
-  for (int base = 0; base < n_slabs; base += kCovTile) {
-    if (!__syncthreads_or(live && !hit)) break;   // also: the previous tile is no longer read
-    for (int k = threadIdx.x; k < kCovTile; k += kCovThreads) {
-      const int si = base + k;
-      int ok = 0;
-      if (si < n_slabs) {
-        const long long hi = static_cast<long long>(b) * n_slabs + si;
-        const int cam = check_cam(a, a.h_cam[hi]);
-        if (cam >= 0) {
-          ok = 1;
-          const float* C = cams + cam * 12;
-#pragma unroll
-          for (int e = 0; e < 9; ++e) s_slab[k].R[e] = C[e];
-#pragma unroll
-          for (int e = 0; e < 3; ++e) s_slab[k].c[e] = C[9 + e];
-#pragma unroll
-          for (int e = 0; e < 6; ++e) s_slab[k].rect[e] = a.h_rect[hi * 6 + e];
-        }
-      }
-      s_ok[k] = ok;
-    }
+  const int per = (n_slabs + kCovSplit - 1) / kCovSplit;
+  const int lo = min(n_slabs, part * per), hi = min(n_slabs, lo + per);
+  const long long hbase = static_cast<long long>(b) * n_slabs;
+  auto cam_at = [&](int si) { return si < hi ? check_cam(a, a.h_cam[hbase + si]) : -1; };
+  CovSlab next;
+  int next_ok = load_slab(a, cams, hbase + lo + threadIdx.x, cam_at(lo + threadIdx.x), next);
+  int cam_ahead = cam_at(lo + kCovTile + threadIdx.x);
+  bool hit = false;
+  for (int base = lo; base < hi; base += kCovTile) {
+    // Stop once no token with depth is left uncovered; also fences the
+    // previous tile's readers.
+    if (!__syncthreads_or(live && !hit)) break;
+    s_slab[threadIdx.x] = next;
+    s_ok[threadIdx.x] = next_ok;
     __syncthreads();
+    const int nb = base + kCovTile;
+    next_ok = load_slab(a, cams, hbase + nb + threadIdx.x, cam_ahead, next);
+    cam_ahead = cam_at(nb + kCovTile + threadIdx.x);
     if (live && !hit) {
-      const int nt = min(kCovTile, n_slabs - base);
+      const int nt = min(kCovTile, hi - base);
       for (int k = grp; k < nt; k += kCovGroups) {
         if (!s_ok[k]) continue;
         const CovSlab& sl = s_slab[k];
         const float D[3] = {fs(X[0], sl.c[0]), fs(X[1], sl.c[1]), fs(X[2], sl.c[2])};
-        const float col0[3] = {sl.R[0], sl.R[3], sl.R[6]};
-        const float col1[3] = {sl.R[1], sl.R[4], sl.R[7]};
         const float col2[3] = {sl.R[2], sl.R[5], sl.R[8]};
         const float zs = dot3(col2, D);
         if (!(zs > 0.f && zs >= sl.rect[4] && zs <= sl.rect[5])) continue;
+        const float col0[3] = {sl.R[0], sl.R[3], sl.R[6]};
+        const float col1[3] = {sl.R[1], sl.R[4], sl.R[7]};
         const float us = fa(fd(fm(a.fx, dot3(col0, D)), zs), a.cx);
         const float vs = fa(fd(fm(a.fy, dot3(col1, D)), zs), a.cy);
         if (us >= sl.rect[0] && us <= sl.rect[1] && vs >= sl.rect[2] && vs <= sl.rect[3]) {
@@ -297,16 +319,25 @@ coverage_kernel(GeoArgs a) {
   }
   __syncthreads();
   if (hit) s_hit[r] = 1;   // any group; benign same-value writes
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    int cnt = 0;
-    for (int k = threadIdx.x; k < kBlk; k += 32) cnt += s_hit[k];
+  // The cluster's CTAs covered disjoint slab ranges: CTA 0 ORs their token
+  // flags through distributed shared memory and writes the fraction.
+  cluster.sync();
+  if (part == 0 && threadIdx.x < kBlk) {
+    int any = s_hit[threadIdx.x];
+#pragma unroll
+    for (int q = 1; q < kCovSplit; ++q) any |= cluster.map_shared_rank(s_hit, q)[threadIdx.x];
+    int cnt = any;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-    if (threadIdx.x == 0)
-      a.cov[static_cast<long long>(b) * a.n_q + j] =
-          nv > 0 ? fd(static_cast<float>(cnt), static_cast<float>(nv)) : 0.f;
+    if ((threadIdx.x & 31) == 0) s_ok[threadIdx.x / 32] = cnt;   // reuse: per-warp counts
   }
+  __syncthreads();
+  if (part == 0 && threadIdx.x == 0) {
+    const int total = s_ok[0] + s_ok[1] + s_ok[2] + s_ok[3];
+    a.cov[static_cast<long long>(b) * a.n_q + j] =
+        nv > 0 ? fd(static_cast<float>(total), static_cast<float>(nv)) : 0.f;
+  }
+  cluster.sync();   // the other CTAs stay resident until their flags were read
 }
 
 }  // namespace bsa
@@ -330,7 +361,7 @@ extern "C" bsa_status bsa_geometry_prior(const float* cams, int n_cams, float fx
   }
   if (g != nullptr && (q_cam == nullptr || q_rect == nullptr)) return BSA_ERR_INVALID_ARG;
   if (coverage != nullptr && (tok_cam == nullptr || tok_uvd == nullptr)) return BSA_ERR_INVALID_ARG;
-  if (B > 65535 || n_q > 65535 ||
+  if (B > 65535 || n_q > 65535 || static_cast<long long>(n_q) * kCovSplit >= (1LL << 31) ||
       static_cast<long long>(n_hist) * slabs_per_block >= (1LL << 31))
     return BSA_ERR_SHAPE;
   GeoArgs a{};
@@ -360,7 +391,7 @@ extern "C" bsa_status bsa_geometry_prior(const float* cams, int n_cams, float fx
     prior_g_kernel<<<grid, kPriorThreads, 0, s>>>(a);
   }
   if (coverage != nullptr) {
-    dim3 grid(n_q, B);
+    dim3 grid(n_q * kCovSplit, B);
     coverage_kernel<<<grid, kCovThreads, 0, s>>>(a);
   }
   return launch_status();
