@@ -82,8 +82,8 @@ enum {
   B_V_FULL = B_K_EMPTY + kKSlots,     // + V slot: V tile landed
   B_V_EMPTY = B_V_FULL + kVSlots,     // + V slot: its P V is done
   B_PV_READY = B_V_EMPTY + kVSlots,   // + slot t % 3: P_t stored, V_t and K_{t+3} landed
-  B_S_FULL = B_PV_READY + kVSlots,    // + warpgroup: S of its next tile ready
-  B_O_READY = B_S_FULL + 2,           // + tile parity: the P V of that tile is done
+  B_S_FULL = B_PV_READY + kVSlots,    // + S buffer: the S of its tile is ready
+  B_O_READY = B_S_FULL + kSBufs,      // + tile parity: the P V of that tile is done
   B_MMA_DONE = B_O_READY + 2,         // + issuer (0: P V thread, 1: Q K^T thread)
   B_MMA_DONE_END = B_MMA_DONE + 2,
   B_COUNT = B_MMA_DONE_END
@@ -303,7 +303,7 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                       kIdQK, kk > 0 ? 1u : 0u);
           }
           tc_commit(&bars[B_K_EMPTY + sl]);
-          tc_commit(&bars[B_S_FULL + (t & 1)]);
+          tc_commit(&bars[B_S_FULL + t % kSBufs]);
         }
       } else {
         constexpr uint32_t kIdPV = idesc_bf16(128, D, 1);
@@ -373,12 +373,17 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       blk_ahead = blk_ahead2;
       const uint32_t s_col = static_cast<uint32_t>(t % kSBufs) * 128;
 
-      // Warpgroup g is the only waiter on S_FULL + g and waits for each of
-      // its completions in turn, so the parity is exact.
+      // One barrier per S buffer: its next completion (S_{t+3}) needs the
+      // P V of this tile, which needs this warpgroup's P_t, so it cannot run
+      // two phases ahead of this wait; and S_{t-3} completed before the
+      // token reached this warpgroup, so it is not behind either: the parity
+      // is exact.  (A barrier per warpgroup could take S_t and S_{t+2} before
+      // its warpgroup looked, since S_{t+2} depends only on the other
+      // warpgroup.)
       float s[kBlk];
       if (ok)
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_S_FULL + g], (t >> 1) & 1, s_abort,
-                                                       kWaitLimit));
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_S_FULL + t % kSBufs],
+                                                       (t / kSBufs) & 1, s_abort, kWaitLimit));
       if (ok) {
         tc_fence_after();
         tmem_ld_cols<kBlk>(tmem + lane_base + s_col, s);
