@@ -156,10 +156,26 @@ class ClockSampler:
 
     def __init__(self, device):
         self.samples = []
+        self.nvml_samples = []
         self.proc = None
+        self.nvml_stop = threading.Event()
         try:
             uuid = str(torch.cuda.get_device_properties(device).uuid)
             sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            return
+        # NVML read every 10 ms, so a timed region of a fraction of a second
+        # still gets many samples (read-only queries).
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByUUID(sel)
+            self.nvml_thread = threading.Thread(target=self._poll_nvml, args=(pynvml, handle),
+                                                daemon=True)
+            self.nvml_thread.start()
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-i", sel, "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
@@ -173,7 +189,24 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.samples.append((time.time(), line.strip()))
 
+    def _poll_nvml(self, nv, handle):
+        try:
+            mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            while not self.nvml_stop.is_set():
+                mhz = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.nvml_samples.append((time.time(), float(mhz), float(mx),
+                                          {k for k, b in bits.items() if r & b}))
+                time.sleep(0.01)
+        except Exception:
+            pass
+
     def stop(self):
+        self.nvml_stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -199,26 +232,61 @@ class ClockSampler:
             for name, val in zip(names, parts[5:9]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
+        n_smi = len(mhz)
+        nv = [x for x in self.nvml_samples if t0 <= x[0] <= t1]
+        for _, m, m_max, rs in nv:
+            mhz.append(m)
+            mx = mx if mx is not None else m_max
+            reasons |= rs
         return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(mhz)}
+                "reasons": sorted(reasons), "samples": len(mhz),
+                "sources": f"nvidia-smi -lms 100: {n_smi}, NVML every 10 ms: {len(nv)}"}
 
 
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
+_flush_bufs = {}
+
+
+def l2_flush(device=None):
+    """Write a buffer larger than L2 (kept per device)."""
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    buf = _flush_bufs.get(device)
+    if buf is None:
+        buf = _flush_bufs[device] = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    buf.zero_()
+
+
+def capture(fn):
+    """fn's launches as a CUDA graph.  The library's calls take the current
+    stream and neither allocate nor synchronise when given their outputs and
+    workspace, so they capture as they are; replaying the graph runs the same
+    kernels on the same buffers without the per-call host marshalling."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
 def _time_call(fn, reps=3):
-    """Median CUDA-event time (ms) of fn() over `reps` calls after one warm-up."""
+    """Median CUDA-event time (ms) of fn() over `reps` calls: fn is run once,
+    captured as a CUDA graph, and each timed replay follows an L2 flush, so
+    the GPU is busy while the host records the events."""
     fn()
+    g = capture(fn)
     ts = []
     for _ in range(reps):
+        l2_flush()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
-        fn()
+        g.replay()
         e1.record()
         torch.cuda.synchronize()
         ts.append(e0.elapsed_time(e1))
+    del g
     return sorted(ts)[len(ts) // 2]
 
 
@@ -290,42 +358,47 @@ class State:
         self.o_blk = torch.empty_like(self.q_blk)
         self.lse = torch.empty((w.B, w.Hh, nbc * BLK), dtype=torch.float32, device=device)
         self.o_tok = torch.empty_like(self.q_tok)
-        self.events = []
+        self.step_graph, self.call_graphs = None, []
         bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W)
         torch.cuda.synchronize(device)
         self.q_valid = self.cache.block_valid[self.own_first:self.own_first + nbc].clone()
 
-    def step(self, time_attn=False):
-        """One pass of the whole path; with ``time_attn`` every call is
-        bracketed by CUDA events on the current stream (kept in self.events)."""
+    def calls(self):
+        """The five library calls of one step, in order, as (name, fn)."""
         bsa, w = self.bsa, self.w
         T, H, W = self.grid
-        ev = []
 
-        def mark(name, fn):
-            if not time_attn:
-                fn()
-                return
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            fn()
-            e1.record()
-            ev.append((name, e0, e1))
-
-        self.cache.n_blocks = self.own_first
-        mark("append", lambda: bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W))
-        mark("q_to_blocks", lambda: bsa.bsa_tokens_to_blocks(self.q_tok, T, H, W, out=self.q_blk))
-        mark("route", lambda: bsa.bsa_route(
-            self.q_blk, self.cache, self.n_hist, self.own_first, self.n_own, w.top_k[0], g=self.g,
-            lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale, q_valid=self.q_valid,
-            max_sel=self.max_sel, idx=self.idx, cnt=self.cnt, workspace=self.ws))
-        mark("attn", lambda: bsa.bsa_attn(self.q_blk, self.cache, self.idx, self.cnt,
+        def append():
+            self.cache.n_blocks = self.own_first   # the chunk's blocks are rewritten in place
+            bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W)
+        return [
+            ("append", append),
+            ("q_to_blocks", lambda: bsa.bsa_tokens_to_blocks(self.q_tok, T, H, W,
+                                                             out=self.q_blk)),
+            ("route", lambda: bsa.bsa_route(
+                self.q_blk, self.cache, self.n_hist, self.own_first, self.n_own, w.top_k[0],
+                g=self.g, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale, q_valid=self.q_valid,
+                max_sel=self.max_sel, idx=self.idx, cnt=self.cnt, workspace=self.ws)),
+            ("attn", lambda: bsa.bsa_attn(self.q_blk, self.cache, self.idx, self.cnt,
                                           q_valid=self.q_valid, sm_scale=w.sm_scale,
-                                          o=self.o_blk, lse=self.lse))
-        mark("o_to_tokens", lambda: bsa.bsa_blocks_to_tokens(self.o_blk, T, H, W, out=self.o_tok))
-        if time_attn:
-            self.events.append(ev)
+                                          o=self.o_blk, lse=self.lse)),
+            ("o_to_tokens", lambda: bsa.bsa_blocks_to_tokens(self.o_blk, T, H, W,
+                                                             out=self.o_tok)),
+        ]
+
+    def step(self):
+        """One pass of the whole path through the library's calls."""
+        for _, fn in self.calls():
+            fn()
+
+    def capture(self):
+        """CUDA graphs of the whole step and of each of its calls."""
+        self.step_graph = capture(self.step)
+        self.call_graphs = [(name, capture(fn)) for name, fn in self.calls()]
+
+    def release_graphs(self):
+        self.step_graph = None
+        self.call_graphs = []
 
     def route_bytes(self, from_means: bool = True) -> float:
         """Algorithmic bytes of bsa_route: Q read, the history key means (or the
@@ -438,24 +511,13 @@ class State:
         w, bsa = self.w, self.bsa
         saved = self.cache.kmean
         self.cache.kmean = None
-        ts = []
         try:
-            for i in range(reps + 2):
-                flush.zero_()
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record()
-                bsa.bsa_route(self.q_blk, self.cache, self.n_hist, self.own_first, self.n_own,
-                              w.top_k[0], g=self.g, lam=w.lam, g_ref=w.g_ref,
-                              sm_scale=w.sm_scale, q_valid=self.q_valid, max_sel=self.max_sel,
-                              idx=self.idx, cnt=self.cnt, workspace=self.ws)
-                e1.record()
-                torch.cuda.synchronize()
-                if i >= 2:
-                    ts.append(e0.elapsed_time(e1))
+            return _time_call(lambda: bsa.bsa_route(
+                self.q_blk, self.cache, self.n_hist, self.own_first, self.n_own, w.top_k[0],
+                g=self.g, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale, q_valid=self.q_valid,
+                max_sel=self.max_sel, idx=self.idx, cnt=self.cnt, workspace=self.ws), reps)
         finally:
             self.cache.kmean = saved
-        return sorted(ts)[len(ts) // 2]
 
     def selected_flops(self) -> float:
         c = self.cnt.to(torch.float64).sum().item()
@@ -470,10 +532,20 @@ def run_ours(args, rank, world, local, pg):
     st = State(w, args.chunk, device, seed_rank=rank, sweep_chunks=sweep)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
-    for _ in range(max(args.warmup, 3)):
+    # Warm-up through the library's calls, then the step is captured as a
+    # CUDA graph (one graph per call as well, for the per-call times) and
+    # warmed up again as a graph.
+    warm = max(args.warmup, 3)
+    for _ in range(warm):
         st.step()
     st.bsa.raise_on_device_error(device)
     flops = st.selected_flops()
+    st.capture()
+    for _ in range(warm):
+        flush.zero_()
+        st.step_graph.replay()
+    torch.cuda.synchronize(device)
+    st.bsa.raise_on_device_error(device)
 
     clocks = ClockSampler(device) if rank == 0 else None
     time.sleep(0.25)
@@ -482,13 +554,12 @@ def run_ours(args, rank, world, local, pg):
     t_wall0 = time.time()
     torch.cuda.nvtx.range_push("timed")
     step_ms = []
-    st.events = []
     for _ in range(args.steps):
         flush.zero_()  # L2 flush between steps, outside the timed events
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
-        st.step(time_attn=True)
+        st.step_graph.replay()
         e1.record()
         step_ms.append((e0, e1))
     torch.cuda.nvtx.range_pop()
@@ -496,19 +567,31 @@ def run_ours(args, rank, world, local, pg):
     barrier(pg, device)
     t_wall1 = time.time()
     st.bsa.raise_on_device_error(device)
-    total_ms = sum(a.elapsed_time(b) for a, b in step_ms)
-    phase_ms = {}
-    for ev in st.events:
-        for name, a, b in ev:
-            phase_ms[name] = phase_ms.get(name, 0.0) + a.elapsed_time(b)
-    phase_ms = {k: max_over_ranks(v / len(st.events), pg, device) for k, v in phase_ms.items()}
-    total_ms = max_over_ranks(total_ms, pg, device)
-    attn_avg = phase_ms["attn"]
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in step_ms), pg, device)
     clock_info = None
     if clocks is not None:
         time.sleep(0.3)
         clocks.stop()
         clock_info = clocks.summary(t_wall0, t_wall1)
+
+    # Per-call times: the same step as one graph per call, an event between
+    # consecutive calls (after the timed region, same L2 flush).
+    n_ph = max(3, min(args.steps, 50))
+    phase_ms = {name: 0.0 for name, _ in st.call_graphs}
+    for _ in range(n_ph):
+        flush.zero_()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(st.call_graphs) + 1)]
+        evs[0].record()
+        for i, (_, g) in enumerate(st.call_graphs):
+            g.replay()
+            evs[i + 1].record()
+        torch.cuda.synchronize(device)
+        for i, (name, _) in enumerate(st.call_graphs):
+            phase_ms[name] += evs[i].elapsed_time(evs[i + 1])
+    st.bsa.raise_on_device_error(device)
+    phase_ms = {k: max_over_ranks(v / n_ph, pg, device) for k, v in phase_ms.items()}
+    attn_avg = phase_ms["attn"]
+    st.release_graphs()
 
     route_stream = st.route_stream_ms(flush)
     velox = st.velox_point(flush) if rank == 0 else None

@@ -207,13 +207,67 @@ pool_score_kernel(RouteArgs a) {
 // for all query blocks j of a head and a tile of 64 history blocks, as a
 // register-blocked CUDA-core product (the whole step is ~0.7 GFLOP at chunk
 // 48, far too small for the tensor cores to matter).  Both operands go to
-// shared memory with a 4-float row pad; each thread owns 4 query blocks x 4
-// history blocks and accumulates over D in order, 4 dimensions per step.
+// shared memory with a 4-float row pad; each thread owns up to 8 query
+// blocks x 4 history blocks and accumulates over D, 4 dimensions per step
+// in two-wide FMAs.
 constexpr int kMeanTileN = 64;
-constexpr int kMeanThreads = 256;
+constexpr int kMeanThreads = 128;
+
+// Query blocks jb + tq + 8x (x < X) against history blocks n0 + tk + 16y
+// (y < 4) of the staged tile; X is the number of 8-row groups the tile's
+// query blocks need, so padded rows cost nothing.  Each dot product keeps
+// two running sums, over the even and over the odd dimensions (in order),
+// as one f32x2 accumulator: the two halves of a 16-byte load are already
+// the operand pairs, so one fma.f32x2 does two dimensions.
+template <int D, int X>
+__device__ __forceinline__ void score_means_tile(const RouteArgs& a, const float* qs,
+                                                 const float* ks, long long bh, int n0, int jb) {
+  constexpr int P = D + 4;
+  // With rows P = D+4 floats apart (an odd number of 16-byte units), the 16
+  // history rows a warp reads per step sit in distinct bank groups; the two
+  // query rows of a warp are broadcasts.
+  const int tk = threadIdx.x % 16, tq = threadIdx.x / 16;
+  uint64_t acc[X][4];
+#pragma unroll
+  for (int x = 0; x < X; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) acc[x][y] = 0ull;   // {+0.f, +0.f}
+#pragma unroll 2
+  for (int d = 0; d < D; d += 4) {
+    ulonglong2 q[X], k[4];
+#pragma unroll
+    for (int x = 0; x < X; ++x)
+      q[x] = *reinterpret_cast<const ulonglong2*>(qs + (jb + tq + 8 * x) * P + d);
+#pragma unroll
+    for (int y = 0; y < 4; ++y)
+      k[y] = *reinterpret_cast<const ulonglong2*>(ks + (tk + 16 * y) * P + d);
+    // All first halves, then all second halves: 4X independent FMAs
+    // between the two that update one accumulator.
+#pragma unroll
+    for (int x = 0; x < X; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = f2_fma(q[x].x, k[y].x, acc[x][y]);
+#pragma unroll
+    for (int x = 0; x < X; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = f2_fma(q[x].y, k[y].y, acc[x][y]);
+  }
+#pragma unroll
+  for (int x = 0; x < X; ++x) {
+    const int j = jb + tq + 8 * x;
+    if (j >= a.n_own) continue;
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int n = n0 + tk + 16 * y;
+      float even, odd;
+      f2_unpack(acc[x][y], even, odd);
+      if (n < a.n_hist) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * (even + odd);
+    }
+  }
+}
 
 template <int D>
-__global__ void __launch_bounds__(kMeanThreads)
+__global__ void __launch_bounds__(kMeanThreads, 1)
 score_means_kernel(RouteArgs a) {
   constexpr int P = D + 4;                       // padded row (floats)
   extern __shared__ float sm[];
@@ -225,7 +279,7 @@ score_means_kernel(RouteArgs a) {
   const int n0 = blockIdx.x * kMeanTileN;
   // Stage the query means and this tile's key means, kLoads independent
   // 16-byte loads per thread in flight before any is stored.
-  constexpr int kLoads = 8;
+  constexpr int kLoads = 16;
   const int n_q4 = nq * (D / 4), n_k4 = kMeanTileN * (D / 4);
   for (int base = 0; base < n_q4 + n_k4; base += kLoads * kMeanThreads) {
     float4 v[kLoads];
@@ -254,49 +308,159 @@ score_means_kernel(RouteArgs a) {
     }
   }
   __syncthreads();
-  // History blocks tn, tn+16, tn+32, tn+48 of the tile: with rows P = D+4
-  // floats apart (an odd number of 16-byte units), the 8 lanes of a
-  // 16-byte-load phase hit 8 different bank groups, and the scores of
-  // consecutive lanes are consecutive in memory.
-  const int tn = threadIdx.x % 16;
-  const int tj = threadIdx.x / 16;               // query blocks tj, tj+16, tj+32, ...
-  for (int jb = 0; jb < nq; jb += 64) {
-    float acc[4][4];
-#pragma unroll
-    for (int x = 0; x < 4; ++x)
-#pragma unroll
-      for (int y = 0; y < 4; ++y) acc[x][y] = 0.f;
-#pragma unroll 4
-    for (int d = 0; d < D; d += 4) {
-      float4 q[4], k[4];
-#pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const int j = jb + tj + 16 * x;
-        q[x] = j < nq ? *reinterpret_cast<const float4*>(qs + j * P + d) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int y = 0; y < 4; ++y) k[y] = *reinterpret_cast<const float4*>(ks + (tn + 16 * y) * P + d);
-#pragma unroll
-      for (int x = 0; x < 4; ++x)
-#pragma unroll
-        for (int y = 0; y < 4; ++y) {
-          acc[x][y] = fmaf(q[x].x, k[y].x, acc[x][y]);
-          acc[x][y] = fmaf(q[x].y, k[y].y, acc[x][y]);
-          acc[x][y] = fmaf(q[x].z, k[y].z, acc[x][y]);
-          acc[x][y] = fmaf(q[x].w, k[y].w, acc[x][y]);
-        }
-    }
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-      const int j = jb + tj + 16 * x;
-      if (j >= a.n_own) continue;
-#pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        const int n = n0 + tn + 16 * y;
-        if (n < a.n_hist) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * acc[x][y];
-      }
+  // Query rows in tiles of 64; a tile's last row read is round8(n_own) - 1,
+  // inside the nq staged (zero-filled) rows.
+  for (int jb = 0; jb < a.n_own; jb += 64) {
+    const int groups = min(8, (a.n_own - jb + 7) / 8);
+    switch (groups) {
+      case 1: score_means_tile<D, 1>(a, qs, ks, bh, n0, jb); break;
+      case 2: score_means_tile<D, 2>(a, qs, ks, bh, n0, jb); break;
+      case 3: score_means_tile<D, 3>(a, qs, ks, bh, n0, jb); break;
+      case 4: score_means_tile<D, 4>(a, qs, ks, bh, n0, jb); break;
+      case 5: score_means_tile<D, 5>(a, qs, ks, bh, n0, jb); break;
+      case 6: score_means_tile<D, 6>(a, qs, ks, bh, n0, jb); break;
+      case 7: score_means_tile<D, 7>(a, qs, ks, bh, n0, jb); break;
+      default: score_means_tile<D, 8>(a, qs, ks, bh, n0, jb); break;
     }
   }
+}
+
+// Pipelined form of the same product, for up to 64 query blocks: a
+// persistent grid (one CTA of 256 threads per SM) walks the (head, 128
+// history blocks) tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Each tile's
+// query means and key means are copied to shared memory by cp.async into
+// one of two stages, so the next tile's copy is in flight while the current
+// tile is scored (the one-shot kernel above waits for its copies with the
+// SM idle, once per wave).  Thread (warp w, lane l) scores query blocks
+// w + 8x against history blocks l + 32y (y < 4): the query rows are warp
+// broadcasts and the 32 key rows of a load sit in distinct bank groups.
+constexpr int kPipeTileN = 128;
+constexpr int kPipeThreads = 256;
+constexpr int kPipeMaxOwn = 64;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_prev() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+
+template <int D, int X>
+__device__ __forceinline__ void score_pipe_tile(const RouteArgs& a, const float* qs,
+                                                const float* ks, long long bh, int n0) {
+  constexpr int P = D + 4;
+  const int tk = threadIdx.x % 32, tq = threadIdx.x / 32;
+  uint64_t acc[X][4];
+#pragma unroll
+  for (int x = 0; x < X; ++x)
+#pragma unroll
+    for (int y = 0; y < 4; ++y) acc[x][y] = 0ull;   // {+0.f, +0.f}
+#pragma unroll 2
+  for (int d = 0; d < D; d += 4) {
+    ulonglong2 q[X], k[4];
+#pragma unroll
+    for (int x = 0; x < X; ++x)
+      q[x] = *reinterpret_cast<const ulonglong2*>(qs + (tq + 8 * x) * P + d);
+#pragma unroll
+    for (int y = 0; y < 4; ++y)
+      k[y] = *reinterpret_cast<const ulonglong2*>(ks + (tk + 32 * y) * P + d);
+    // All first halves, then all second halves: 4X independent FMAs
+    // between the two that update one accumulator.
+#pragma unroll
+    for (int x = 0; x < X; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = f2_fma(q[x].x, k[y].x, acc[x][y]);
+#pragma unroll
+    for (int x = 0; x < X; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = f2_fma(q[x].y, k[y].y, acc[x][y]);
+  }
+#pragma unroll
+  for (int x = 0; x < X; ++x) {
+    const int j = tq + 8 * x;
+    if (j >= a.n_own) continue;
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int n = n0 + tk + 32 * y;
+      float even, odd;
+      f2_unpack(acc[x][y], even, odd);
+      if (n < a.n_hist) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * (even + odd);
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPipeThreads, 1) score_means_pipe_kernel(RouteArgs a) {
+  constexpr int P = D + 4;
+  constexpr int R4 = D / 4;                      // 16-byte pieces per row
+  extern __shared__ __align__(16) float sm[];
+  const int nq8 = (a.n_own + 7) & ~7;            // query rows read by the product
+  const int stage = (nq8 + kPipeTileN) * P;      // floats per stage
+  const int per_head = (a.n_hist + kPipeTileN - 1) / kPipeTileN;
+  const int n_tiles = a.B * a.Hh * per_head;
+  auto copy_tile = [&](int tile, int st) {
+    const long long bh = tile / per_head;        // b * Hh + h
+    const int n0 = (tile % per_head) * kPipeTileN;
+    float* qs = sm + st * stage;
+    float* ks = qs + nq8 * P;
+    for (int i = threadIdx.x; i < (nq8 + kPipeTileN) * R4; i += kPipeThreads) {
+      const int r = i / R4, c4 = i % R4;
+      if (r < nq8) {
+        const bool v = r < a.n_own;              // rows past n_own are zero-filled
+        cp_async16(qs + r * P + c4 * 4, v ? a.qm + (bh * a.n_own + r) * D + c4 * 4 : a.qm, v);
+      } else {
+        const int rk = r - nq8;
+        const bool v = n0 + rk < a.n_hist;
+        cp_async16(ks + rk * P + c4 * 4,
+                   v ? a.kmean + (bh * a.max_blocks + n0 + rk) * D + c4 * 4 : a.kmean, v);
+      }
+    }
+  };
+  int tile = blockIdx.x;
+  if (tile >= n_tiles) return;
+  copy_tile(tile, 0);
+  cp_async_commit();
+  const int groups = nq8 / 8;
+  for (int k = 0; tile < n_tiles; ++k, tile += gridDim.x) {
+    // The copy into the other stage: that stage was last read in step k-1,
+    // which every thread finished before the barrier ending step k-1.
+    if (tile + static_cast<int>(gridDim.x) < n_tiles) copy_tile(tile + gridDim.x, (k + 1) & 1);
+    cp_async_commit();                           // (an empty group at the end)
+    cp_async_wait_prev();                        // this thread's copies of tile
+    __syncthreads();                             // ... and everyone's
+    const float* qs = sm + (k & 1) * stage;
+    const float* ks = qs + nq8 * P;
+    const long long bh = tile / per_head;
+    const int n0 = (tile % per_head) * kPipeTileN;
+    switch (groups) {
+      case 1: score_pipe_tile<D, 1>(a, qs, ks, bh, n0); break;
+      case 2: score_pipe_tile<D, 2>(a, qs, ks, bh, n0); break;
+      case 3: score_pipe_tile<D, 3>(a, qs, ks, bh, n0); break;
+      case 4: score_pipe_tile<D, 4>(a, qs, ks, bh, n0); break;
+      case 5: score_pipe_tile<D, 5>(a, qs, ks, bh, n0); break;
+      case 6: score_pipe_tile<D, 6>(a, qs, ks, bh, n0); break;
+      case 7: score_pipe_tile<D, 7>(a, qs, ks, bh, n0); break;
+      default: score_pipe_tile<D, 8>(a, qs, ks, bh, n0); break;
+    }
+    __syncthreads();                             // stage k & 1 is copied into at step k + 1
+  }
+}
+
+// Streaming multiprocessors of the current device (cached per device).
+static int device_sms() {
+  static int cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
 }
 
 // Order-preserving map of a float onto uint32 (larger float -> larger key).
@@ -330,10 +494,13 @@ constexpr int kTopkSmemKeys = 40960;
 
 // Fused score of history block n of row (b, j): the model score plus the
 // prior boost lam * min(g / g_ref, 1) (g shared by all heads).
+__device__ __forceinline__ float fuse_prior(const RouteArgs& a, float sc, float gv) {
+  return sc + a.lam * fminf(gv / a.g_ref, 1.0f);
+}
 __device__ __forceinline__ float fused_score(const RouteArgs& a, const float* sr, const float* gr,
                                              int n) {
   float sc = sr[n];
-  if (gr != nullptr) sc += a.lam * fminf(gr[n] / a.g_ref, 1.0f);
+  if (gr != nullptr) sc = fuse_prior(a, sc, gr[n]);
   return sc;
 }
 
@@ -493,6 +660,130 @@ __device__ void radix_threshold(const uint32_t* keys, int n, int K, int* hist, u
   }
   *thr = prefix;
   *need_eq = remaining;
+}
+
+// Top-K of a row of at most 128 * KPL history blocks: one CTA of 128
+// threads per row, thread t holding the keys of blocks c * 128 + t (c < KPL)
+// in registers.
+//   1. Search, bit by bit from the top, for the largest t with
+//      #{key >= t} >= K (the K-th largest key), one block-wide count per
+//      bit.  It stops early once a count is exactly K: those keys are then
+//      the top K and no key equal to the K-th is left out.
+//   2. Otherwise take the keys > t and the lowest-indexed K - #{key > t}
+//      keys equal to t.
+//   3. Write the selected blocks in ascending order: one ballot per
+//      32-block group, the group totals in shared memory, one barrier.
+// The selected set and its order are those of topk_kernel.
+constexpr int kTopkRowThreads = 128;
+
+template <int KPL>
+__global__ void __launch_bounds__(kTopkRowThreads, KPL <= 18 ? 8 : 6) topk_row_kernel(RouteArgs a) {
+  constexpr int kWarps = kTopkRowThreads / 32;
+  __shared__ unsigned part[2][kWarps];
+  __shared__ unsigned grp[2][KPL][kWarps];     // per-(group, warp) ballot counts: eq, sel
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const long long row = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
+  int32_t* out = a.idx + row * a.max_sel;
+  const float* sr = a.s + row * a.n_hist;
+  const float* gr = a.g != nullptr ? a.g + (static_cast<long long>(b) * a.n_own + j) * a.n_hist
+                                   : nullptr;
+  const int nh = a.n_hist;
+  const int K = a.top_k < nh ? a.top_k : nh;
+  if (K == nh) {
+    for (int n = t; n < nh; n += kTopkRowThreads) out[n] = n;
+  } else if (K > 0) {
+    float f[KPL], gv[KPL];
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      const int n = c * kTopkRowThreads + t;
+      f[c] = n < nh ? sr[n] : 0.f;
+      gv[c] = (gr != nullptr && n < nh) ? gr[n] : 0.f;
+    }
+    uint32_t key[KPL];
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      const int n = c * kTopkRowThreads + t;
+      key[c] = n < nh ? score_key(gr != nullptr ? fuse_prior(a, f[c], gv[c]) : f[c]) : 0u;
+    }
+    // Padding keys are 0: they count only toward t = 0, which every row
+    // satisfies anyway, and the selection below skips them by index.
+    auto block_count = [&](uint32_t cand, bool strict, int parity) -> int {
+      unsigned c0 = 0, c1 = 0;
+#pragma unroll
+      for (int c = 0; c < KPL; c += 2) {
+        c0 += strict ? key[c] > cand : key[c] >= cand;
+        if (c + 1 < KPL) c1 += strict ? key[c + 1] > cand : key[c + 1] >= cand;
+      }
+      const unsigned w = __reduce_add_sync(0xffffffffu, c0 + c1);
+      if (lane == 0) part[parity][warp] = w;
+      __syncthreads();
+      unsigned tot = 0;
+#pragma unroll
+      for (int i = 0; i < kWarps; ++i) tot += part[parity][i];
+      return static_cast<int>(tot);
+    };
+    // part[] alternates between two buffers: a warp can only overwrite a
+    // buffer after the next barrier, which every warp reaches only after
+    // reading it.
+    uint32_t thr = 0;
+    bool exact = false;
+    int parity = 0;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = thr | (1u << bit);
+      const int cnt = block_count(cand, false, parity);
+      parity ^= 1;
+      if (cnt >= K) {
+        thr = cand;
+        if (cnt == K) { exact = true; break; }
+      }
+    }
+    // exact: take key >= thr (K of them); else key > thr plus the first
+    // need_eq keys == thr.
+    const int need_eq = exact ? 0 : K - block_count(thr, true, parity);
+    const unsigned below = (1u << lane) - 1u;
+    bool eq[KPL];
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      eq[c] = !exact && c * kTopkRowThreads + t < nh && key[c] == thr;
+      const unsigned m = __ballot_sync(0xffffffffu, eq[c]);
+      if (lane == 0) grp[0][c][warp] = __popc(m);
+    }
+    __syncthreads();
+    bool sel[KPL];
+    int before = 0;   // equal keys in earlier groups
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      const int n = c * kTopkRowThreads + t;
+      int rank = before + __popc(__ballot_sync(0xffffffffu, eq[c]) & below);
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const int e = static_cast<int>(grp[0][c][w]);
+        rank += w < warp ? e : 0;
+        before += e;
+      }
+      sel[c] = n < nh && (exact ? key[c] >= thr : (key[c] > thr || (eq[c] && rank < need_eq)));
+      const unsigned m = __ballot_sync(0xffffffffu, sel[c]);
+      if (lane == 0) grp[1][c][warp] = __popc(m);
+    }
+    __syncthreads();
+    int pos = 0;      // selected blocks in earlier groups
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      int at = pos + __popc(__ballot_sync(0xffffffffu, sel[c]) & below);
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const int e = static_cast<int>(grp[1][c][w]);
+        at += w < warp ? e : 0;
+        pos += e;
+      }
+      if (sel[c]) out[at] = c * kTopkRowThreads + t;
+    }
+  }
+  for (int i = t; i < a.n_own; i += kTopkRowThreads) out[K + i] = a.own_first + i;
+  for (int i = K + a.n_own + t; i < a.max_sel; i += kTopkRowThreads) out[i] = -1;
+  if (t == 0) a.cnt[row] = K + a.n_own;
 }
 
 __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a, VeloxArgs v) {
@@ -748,9 +1039,25 @@ static bsa_status route_scores(const void* q_blk, const bsa_kv_cache* c, const i
   const int per_cta = kScoreWarps * kScoreBlocksPerWarp;
   dim3 sgrid((n_hist + per_cta - 1) / per_cta, c->Hh, c->B);
   dim3 mgrid((n_hist + kMeanTileN - 1) / kMeanTileN, c->Hh, c->B);
+  // Pipelined product: up to 64 query blocks, one CTA per SM (at most one
+  // per tile); 0 selects the one-shot kernel.
+  const int nq8 = (n_own + 7) & ~7;
+  const size_t pipe_smem = 2 * sizeof(float) * static_cast<size_t>(nq8 + kPipeTileN) * (c->D + 4);
+  int pipe_grid = 0;
+  if (n_own <= kPipeMaxOwn && n_hist > 0) {
+    const long long tiles = static_cast<long long>(c->B) * c->Hh *
+                            ((n_hist + kPipeTileN - 1) / kPipeTileN);
+    pipe_grid = static_cast<int>(std::min<long long>(tiles, device_sms()));
+  }
   if (c->D == 128) {
     pool_q_kernel<16><<<qgrid, kPoolThreads, 0, s>>>(a);
-    if (n_hist > 0 && c->kmean != nullptr) {
+    if (n_hist > 0 && c->kmean != nullptr && pipe_grid > 0) {
+      if (cudaFuncSetAttribute(score_means_pipe_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(pipe_smem)) != cudaSuccess)
+        return BSA_ERR_CUDA;
+      score_means_pipe_kernel<128><<<pipe_grid, kPipeThreads, pipe_smem, s>>>(a);
+    } else if (n_hist > 0 && c->kmean != nullptr) {
       if (cudaFuncSetAttribute(score_means_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(mean_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
@@ -763,7 +1070,13 @@ static bsa_status route_scores(const void* q_blk, const bsa_kv_cache* c, const i
     }
   } else {
     pool_q_kernel<8><<<qgrid, kPoolThreads, 0, s>>>(a);
-    if (n_hist > 0 && c->kmean != nullptr) {
+    if (n_hist > 0 && c->kmean != nullptr && pipe_grid > 0) {
+      if (cudaFuncSetAttribute(score_means_pipe_kernel<64>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(pipe_smem)) != cudaSuccess)
+        return BSA_ERR_CUDA;
+      score_means_pipe_kernel<64><<<pipe_grid, kPipeThreads, pipe_smem, s>>>(a);
+    } else if (n_hist > 0 && c->kmean != nullptr) {
       if (cudaFuncSetAttribute(score_means_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(mean_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
@@ -796,12 +1109,26 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
                                sm_scale, idx, cnt, max_sel, workspace, ws_bytes, d_err, s, &a);
   if (st != BSA_OK) return st;
   a.top_k = top_k;
+  // Rows of up to 3072 history blocks: keys in registers (their count per
+  // thread follows the row length); longer rows: a radix select over keys
+  // staged in shared memory.  One CTA per row either way.
+  dim3 qgrid(n_own, c->Hh, c->B);
+  if (n_hist <= kTopkRowThreads * 24) {
+    if (n_hist <= kTopkRowThreads * 4)
+      topk_row_kernel<4><<<qgrid, kTopkRowThreads, 0, s>>>(a);
+    else if (n_hist <= kTopkRowThreads * 10)
+      topk_row_kernel<10><<<qgrid, kTopkRowThreads, 0, s>>>(a);
+    else if (n_hist <= kTopkRowThreads * 18)
+      topk_row_kernel<18><<<qgrid, kTopkRowThreads, 0, s>>>(a);
+    else
+      topk_row_kernel<24><<<qgrid, kTopkRowThreads, 0, s>>>(a);
+    return launch_status();
+  }
   const size_t topk_smem =
       n_hist <= kTopkSmemKeys ? sizeof(uint32_t) * static_cast<size_t>(n_hist > 0 ? n_hist : 1) : 0;
   if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(topk_smem)) != cudaSuccess)
     return BSA_ERR_CUDA;
-  dim3 qgrid(n_own, c->Hh, c->B);
   topk_kernel<<<qgrid, kTopkThreads, topk_smem, s>>>(a);
   return launch_status();
 }

@@ -5,6 +5,8 @@ Block indices must match the oracle exactly, apart from near-ties within
 1e-5 relative of the K-th score (fp32 on the GPU, fp64 in the oracle), where
 either choice is accepted.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -48,12 +50,22 @@ def test_route_config5_head_sample(top_k):
     _check(hx.build_step(synth.CONFIGS[5], DEV, top_k=top_k), heads=[0, 17, 39])
 
 
-@pytest.mark.parametrize("chunk", [1, 2, 3, 48])
+@pytest.mark.parametrize("chunk", [1, 2, 3, 12, 48, 49])
 def test_route_config4_sweep_chunks(chunk):
     # chunk 1: no history (own chunk only); chunk 2: K >= history (all);
     # chunk 3: K < history; chunk 48: the headline size, one head checked.
+    # The row lengths 98, 539, 2303 and 2352 take each register width of the
+    # warp-per-row top-K (up to 512, 1280, 2304 and 3072 blocks).
     step = hx.build_step(synth.CONFIGS[4], DEV, chunk=chunk)
-    _check(step, heads=[5] if chunk == 48 else [0, 23])
+    _check(step, heads=[5] if chunk >= 12 else [0, 23])
+
+
+def test_route_rows_longer_than_the_warp_select():
+    # 193 history chunks of 16 blocks: rows of 3088 history blocks go to the
+    # block-per-row radix select.
+    step = hx.build_step(synth.CONFIGS[2], DEV, chunk=194)
+    assert step.n_hist > 32 * 96
+    _check(step, heads=[7])
 
 
 def test_route_without_prior_equals_prior_of_zeros():
@@ -90,7 +102,7 @@ def test_route_rejects_bad_arguments():
     assert e.value.status == 2
 
 
-@pytest.mark.parametrize("key,chunk", [(1, None), (2, None), (3, None), (4, 48)])
+@pytest.mark.parametrize("key,chunk", [(1, None), (2, None), (3, None), (4, 48), (5, None)])
 def test_route_from_pooled_keys(key, chunk):
     # Routing from the pooled-key cache (block key means written at append
     # time, scored by a small product kernel) against the oracle, with the
@@ -99,7 +111,7 @@ def test_route_from_pooled_keys(key, chunk):
     # near-ties.
     w = synth.CONFIGS[key]
     b = hx.build_step(w, DEV, chunk=chunk, pooled_keys=True)
-    ib, cb = _check(b, heads=[5] if key == 4 else None)
+    ib, cb = _check(b, heads=[5] if key == 4 else [0, 39] if key == 5 else None)
     # The no-allocation entry point takes the same path, bit for bit.
     import ctypes
     idx = torch.full_like(ib, -7)
@@ -114,3 +126,12 @@ def test_route_from_pooled_keys(key, chunk):
     assert st == 0
     torch.cuda.synchronize()
     assert torch.equal(idx, ib) and torch.equal(cnt, cb)
+
+
+def test_route_from_pooled_keys_many_query_blocks():
+    # 98 query blocks (an 8 x 30 x 52 chunk): more than the pipelined pooled
+    # product takes (64), so the one-shot kernel scores them.
+    w = dataclasses.replace(synth.CONFIGS[3], grid=(8, 30, 52), Hh=4, hist_direct=300)
+    b = hx.build_step(w, DEV, pooled_keys=True)
+    assert b.n_own > 64
+    _check(b)
