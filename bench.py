@@ -239,6 +239,7 @@ class ClockSampler:
             mx = mx if mx is not None else m_max
             reasons |= rs
         return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": mx,
+                "sm_mhz_range": [min(mhz), max(mhz)] if mhz else None,
                 "reasons": sorted(reasons), "samples": len(mhz),
                 "sources": f"nvidia-smi -lms 100: {n_smi}, NVML every 10 ms: {len(nv)}"}
 
@@ -358,7 +359,7 @@ class State:
         self.o_blk = torch.empty_like(self.q_blk)
         self.lse = torch.empty((w.B, w.Hh, nbc * BLK), dtype=torch.float32, device=device)
         self.o_tok = torch.empty_like(self.q_tok)
-        self.step_graph, self.call_graphs = None, []
+        self.call_graphs = []
         bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W)
         torch.cuda.synchronize(device)
         self.q_valid = self.cache.block_valid[self.own_first:self.own_first + nbc].clone()
@@ -392,12 +393,21 @@ class State:
             fn()
 
     def capture(self):
-        """CUDA graphs of the whole step and of each of its calls."""
-        self.step_graph = capture(self.step)
+        """One CUDA graph per call of the step, replayed in order."""
         self.call_graphs = [(name, capture(fn)) for name, fn in self.calls()]
 
+    def replay(self, events=None):
+        """One step from the captured graphs; with ``events`` (one more than
+        the calls), event i is recorded before call i and the last after the
+        step, on the current stream."""
+        if events is not None:
+            events[0].record()
+        for i, (_, g) in enumerate(self.call_graphs):
+            g.replay()
+            if events is not None:
+                events[i + 1].record()
+
     def release_graphs(self):
-        self.step_graph = None
         self.call_graphs = []
 
     def route_bytes(self, from_means: bool = True) -> float:
@@ -532,9 +542,8 @@ def run_ours(args, rank, world, local, pg):
     st = State(w, args.chunk, device, seed_rank=rank, sweep_chunks=sweep)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
-    # Warm-up through the library's calls, then the step is captured as a
-    # CUDA graph (one graph per call as well, for the per-call times) and
-    # warmed up again as a graph.
+    # Warm-up through the library's calls; then each call is captured as a
+    # CUDA graph, and the graphs are warmed up too.
     warm = max(args.warmup, 3)
     for _ in range(warm):
         st.step()
@@ -543,7 +552,7 @@ def run_ours(args, rank, world, local, pg):
     st.capture()
     for _ in range(warm):
         flush.zero_()
-        st.step_graph.replay()
+        st.replay()
     torch.cuda.synchronize(device)
     st.bsa.raise_on_device_error(device)
 
@@ -553,45 +562,34 @@ def run_ours(args, rank, world, local, pg):
     torch.cuda.synchronize(device)
     t_wall0 = time.time()
     torch.cuda.nvtx.range_push("timed")
-    step_ms = []
+    step_events = []
+    n_calls = len(st.call_graphs)
     for _ in range(args.steps):
         flush.zero_()  # L2 flush between steps, outside the timed events
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        st.step_graph.replay()
-        e1.record()
-        step_ms.append((e0, e1))
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_calls + 1)]
+        st.replay(evs)
+        step_events.append(evs)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(device)
     barrier(pg, device)
     t_wall1 = time.time()
     st.bsa.raise_on_device_error(device)
-    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in step_ms), pg, device)
+    per_step = [evs[0].elapsed_time(evs[-1]) for evs in step_events]
+    total_ms = max_over_ranks(sum(per_step), pg, device)
+    # Per-call times from the same timed region: the events between calls.
+    phase_ms = {name: sum(evs[i].elapsed_time(evs[i + 1]) for evs in step_events) / args.steps
+                for i, (name, _) in enumerate(st.call_graphs)}
+    phase_ms = {k: max_over_ranks(v, pg, device) for k, v in phase_ms.items()}
+    attn_avg = phase_ms["attn"]
+    spread = sorted(per_step)
+    step_spread = {"min": round(spread[0], 4), "median": round(spread[len(spread) // 2], 4),
+                   "max": round(spread[-1], 4)}
+    st.release_graphs()
     clock_info = None
     if clocks is not None:
         time.sleep(0.3)
         clocks.stop()
         clock_info = clocks.summary(t_wall0, t_wall1)
-
-    # Per-call times: the same step as one graph per call, an event between
-    # consecutive calls (after the timed region, same L2 flush).
-    n_ph = max(3, min(args.steps, 50))
-    phase_ms = {name: 0.0 for name, _ in st.call_graphs}
-    for _ in range(n_ph):
-        flush.zero_()
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(st.call_graphs) + 1)]
-        evs[0].record()
-        for i, (_, g) in enumerate(st.call_graphs):
-            g.replay()
-            evs[i + 1].record()
-        torch.cuda.synchronize(device)
-        for i, (name, _) in enumerate(st.call_graphs):
-            phase_ms[name] += evs[i].elapsed_time(evs[i + 1])
-    st.bsa.raise_on_device_error(device)
-    phase_ms = {k: max_over_ranks(v / n_ph, pg, device) for k, v in phase_ms.items()}
-    attn_avg = phase_ms["attn"]
-    st.release_graphs()
 
     route_stream = st.route_stream_ms(flush)
     velox = st.velox_point(flush) if rank == 0 else None
@@ -631,6 +629,7 @@ def run_ours(args, rank, world, local, pg):
         "attn": {"ms_per_call": round(attn_avg, 4), "tflops": round(attn_tflops, 2),
                  "selected_tflop_per_call": round(flops / 1e12, 4)},
         "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()},
+        "step_ms_spread": step_spread,
         "route": {"ms_per_call": round(phase_ms["route"], 4),
                   "keys": "pooled-key cache (means written by bsa_kv_append)",
                   "gbs": round(st.route_bytes() / (phase_ms["route"] * 1e-3) / 1e9, 1),
