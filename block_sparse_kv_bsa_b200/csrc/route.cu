@@ -786,6 +786,57 @@ __global__ void __launch_bounds__(kTopkRowThreads, KPL <= 18 ? 8 : 6) topk_row_k
   if (t == 0) a.cnt[row] = K + a.n_own;
 }
 
+// Block-wide exclusive prefix, over threads in index order, of a per-thread
+// count; *total gets the block total.  Two barriers.
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int* total) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kTopkThreads / 32; ++w) {
+    const int c = warp_tot[w];
+    before += (w < warp) ? c : 0;
+    all += c;
+  }
+  __syncthreads();
+  *total = all;
+  return before + incl - v;
+}
+
+// Tree reduction of red[0..255] (already written and synchronised): level w
+// combines red[t] and red[t + w] for t < w, w = 128, 64, ..., 1.  The levels
+// below 32 run in warp 0 with shuffles, which pair the same operands in the
+// same order.  Returns the result to every thread.
+template <typename Op>
+__device__ __forceinline__ float block_tree(float* red, Op op) {
+#pragma unroll
+  for (int w = kTopkThreads / 2; w >= 32; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] = op(red[threadIdx.x], red[threadIdx.x + w]);
+    __syncthreads();
+  }
+  if (threadIdx.x < 32) {
+    float x = red[threadIdx.x];
+#pragma unroll
+    for (int w = 16; w > 0; w >>= 1) x = op(x, __shfl_down_sync(0xffffffffu, x, w));
+    if (threadIdx.x == 0) red[0] = x;
+  }
+  __syncthreads();
+  const float r = red[0];
+  __syncthreads();
+  return r;
+}
+
+// Each thread owns the contiguous blocks [t * run, min((t+1) * run, nh)), so
+// a block scan of per-thread counts orders everything by block index.
+constexpr int kVeloxRankMax = 256;   // budgets up to this are ranked by counting
+
 __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a, VeloxArgs v) {
   extern __shared__ __align__(16) uint8_t vsm[];
   const int nh = a.n_hist;
@@ -797,6 +848,9 @@ __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a,
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining, s_m;
   __shared__ float red[kTopkThreads];
+  __shared__ int nidx[kVeloxRankMax];     // sorted position -> block
+  __shared__ float pr[kVeloxRankMax];     // sorted position -> softmax probability
+  const int t = threadIdx.x;
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const long long row = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
   int32_t* out = a.idx + row * a.max_sel;
@@ -805,12 +859,34 @@ __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a,
   const bool covered = v.coverage != nullptr && v.coverage[b * a.n_own + j] >= v.eta_cov;
   const int p0 = min(max(v.prev_first, 0), nh);
   const int p1 = min(max(v.prev_first + v.n_prev, p0), nh);
+  const int run = (nh + kTopkThreads - 1) / kTopkThreads;
+  const int r0 = min(t * run, nh), r1 = min(r0 + run, nh);
+
+  // Keys > thr, and the need_eq lowest-indexed keys == thr (key 0 never
+  // taken): calls take(n) for each, in ascending n within this thread's run.
+  // Returns this thread's count before the run and the block total.
+  auto select_run = [&](uint32_t thr, int need_eq, auto take) {
+    int eq_local = 0;
+    for (int n = r0; n < r1; ++n) eq_local += (keys[n] == thr && keys[n] != 0u);
+    int eq_tot;
+    int eq_rank = block_excl_scan(eq_local, warp_tot, &eq_tot);
+    for (int n = r0; n < r1; ++n) {
+      const uint32_t k = keys[n];
+      if (k == 0u) continue;
+      if (k > thr) {
+        take(n);
+      } else if (k == thr) {
+        if (eq_rank < need_eq) take(n);
+        ++eq_rank;
+      }
+    }
+  };
 
   if (covered) {
     // s + log(1 + lam * g_hat) ranks like the renormalised product of the
     // importance distribution and 1 + lam * g_hat; the previous chunk is
     // reserved (key 0 keeps it out of the selection).
-    for (int n = threadIdx.x; n < nh; n += kTopkThreads) {
+    for (int n = t; n < nh; n += kTopkThreads) {
       const bool res = n >= p0 && n < p1;
       float f = sr[n];
       if (gr != nullptr) {
@@ -828,130 +904,133 @@ __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a,
       uint32_t thr;
       int need_eq;
       radix_threshold(keys, nh, K, hist, &s_prefix, &s_remaining, &thr, &need_eq);
-      int eq_seen = 0;
-      for (int base = 0; base < nh; base += kTopkThreads) {
-        const int n = base + threadIdx.x;
-        const uint32_t k = n < nh ? keys[n] : 0u;
-        const bool eq = n < nh && k == thr && k != 0u;
-        int eq_tot;
-        const int eq_rank = eq_seen + block_excl_count(eq, warp_tot, &eq_tot);
-        if (n < nh && k != 0u && (k > thr || (eq && eq_rank < need_eq))) flag[n] = 1;
-        eq_seen += eq_tot;
-      }
+      select_run(thr, need_eq, [&](int n) { flag[n] = 1; });
     }
   } else {
-    for (int n = threadIdx.x; n < nh; n += kTopkThreads) {
+    for (int n = t; n < nh; n += kTopkThreads) {
       keys[n] = score_key(sr[n]);
       flag[n] = 0;
     }
-    __syncthreads();
     const int K = min(v.k_unc, nh);
     if (K > 0) {
       // Row maximum and normaliser of softmax(s), in a fixed order.
       float mx = -INFINITY;
-      for (int n = threadIdx.x; n < nh; n += kTopkThreads) mx = fmaxf(mx, sr[n]);
-      red[threadIdx.x] = mx;
+      for (int n = t; n < nh; n += kTopkThreads) mx = fmaxf(mx, sr[n]);
+      red[t] = mx;
       __syncthreads();
-      for (int w = kTopkThreads / 2; w > 0; w >>= 1) {
-        if (threadIdx.x < w) red[threadIdx.x] = fmaxf(red[threadIdx.x], red[threadIdx.x + w]);
-        __syncthreads();
-      }
-      const float smax = red[0];
-      __syncthreads();
+      const float smax = block_tree(red, [](float x, float y) { return fmaxf(x, y); });
       float z = 0.f;
-      for (int n = threadIdx.x; n < nh; n += kTopkThreads) z += expf(sr[n] - smax);
-      red[threadIdx.x] = z;
+      for (int n = t; n < nh; n += kTopkThreads) z += expf(sr[n] - smax);
+      red[t] = z;
       __syncthreads();
-      for (int w = kTopkThreads / 2; w > 0; w >>= 1) {
-        if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-        __syncthreads();
-      }
-      const float zsum = red[0];
-      // The K best blocks, listed in index order, then sorted by (score
-      // descending, index ascending) so the mass prefix can be walked.
+      const float zsum = block_tree(red, [](float x, float y) { return x + y; });
+      // The K best blocks, then their order by (score descending, index
+      // ascending) so the mass prefix can be walked.
       uint32_t thr;
       int need_eq;
       radix_threshold(keys, nh, K, hist, &s_prefix, &s_remaining, &thr, &need_eq);
-      int pos = 0, eq_seen = 0;
-      for (int base = 0; base < nh; base += kTopkThreads) {
-        const int n = base + threadIdx.x;
-        const uint32_t k = n < nh ? keys[n] : 0u;
-        const bool gt = n < nh && k > thr;
-        const bool eq = n < nh && k == thr;
-        int eq_tot, sel_tot;
-        const int eq_rank = eq_seen + block_excl_count(eq, warp_tot, &eq_tot);
-        const bool sel = gt || (eq && eq_rank < need_eq);
-        const int at = pos + block_excl_count(sel, warp_tot, &sel_tot);
-        // ascending order of ~((key << 32) | ~n) = descending key, ascending n
-        if (sel) sortbuf[at] = ~((static_cast<uint64_t>(k) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(n)));
-        pos += sel_tot;
-        eq_seen += eq_tot;
-      }
-      int P = 2;
-      while (P < K) P <<= 1;
-      for (int i = K + threadIdx.x; i < P; i += kTopkThreads) sortbuf[i] = ~0ull;
+      int sel_local = 0;
+      select_run(thr, need_eq, [&](int) { ++sel_local; });
+      int sel_tot;
+      int at = block_excl_scan(sel_local, warp_tot, &sel_tot);
+      // ascending order of ~((key << 32) | ~n) = descending key, ascending n
+      select_run(thr, need_eq, [&](int n) {
+        sortbuf[at++] = ~((static_cast<uint64_t>(keys[n]) << 32) |
+                          (0xFFFFFFFFu - static_cast<uint32_t>(n)));
+      });
       __syncthreads();
-      for (int kk = 2; kk <= P; kk <<= 1) {
-        for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-          for (int i = threadIdx.x; i < P; i += kTopkThreads) {
-            const int ixj = i ^ jj;
-            if (ixj > i) {
-              const uint64_t x = sortbuf[i], y = sortbuf[ixj];
-              const bool up = (i & kk) == 0;
-              if (up ? (x > y) : (x < y)) {
-                sortbuf[i] = y;
-                sortbuf[ixj] = x;
-              }
+      if (K <= kVeloxRankMax) {
+        // Rank by counting (the values are distinct): one barrier instead of
+        // a sorting network.
+        if (t < K) {
+          const uint64_t x = sortbuf[t];
+          int rank = 0;
+          for (int i = 0; i < K; ++i) rank += sortbuf[i] < x;
+          const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~x));
+          nidx[rank] = n;
+          pr[rank] = expf(sr[n] - smax) / zsum;
+        }
+        __syncthreads();
+        if (t == 0) {
+          float acc = 0.f;
+          int m = K;
+          for (int r = 0; r < K; ++r) {
+            acc += pr[r];
+            if (acc >= v.mass) {
+              m = r + 1;
+              break;
             }
           }
-          __syncthreads();
+          s_m = m;
         }
-      }
-      if (threadIdx.x == 0) {
-        float acc = 0.f;
-        int m = K;
-        for (int r = 0; r < K; ++r) {
-          const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]));
-          acc += expf(sr[n] - smax) / zsum;
-          if (acc >= v.mass) {
-            m = r + 1;
-            break;
+        __syncthreads();
+        for (int r = t; r < s_m; r += kTopkThreads) flag[nidx[r]] = 1;
+      } else {
+        int P = 2;
+        while (P < K) P <<= 1;
+        for (int i = K + t; i < P; i += kTopkThreads) sortbuf[i] = ~0ull;
+        __syncthreads();
+        for (int kk = 2; kk <= P; kk <<= 1) {
+          for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+            for (int i = t; i < P; i += kTopkThreads) {
+              const int ixj = i ^ jj;
+              if (ixj > i) {
+                const uint64_t x = sortbuf[i], y = sortbuf[ixj];
+                const bool up = (i & kk) == 0;
+                if (up ? (x > y) : (x < y)) {
+                  sortbuf[i] = y;
+                  sortbuf[ixj] = x;
+                }
+              }
+            }
+            __syncthreads();
           }
         }
-        s_m = m;
+        if (t == 0) {
+          float acc = 0.f;
+          int m = K;
+          for (int r = 0; r < K; ++r) {
+            const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]));
+            acc += expf(sr[n] - smax) / zsum;
+            if (acc >= v.mass) {
+              m = r + 1;
+              break;
+            }
+          }
+          s_m = m;
+        }
+        __syncthreads();
+        for (int r = t; r < s_m; r += kTopkThreads)
+          flag[static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]))] = 1;
       }
-      __syncthreads();
-      for (int r = threadIdx.x; r < s_m; r += kTopkThreads)
-        flag[static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]))] = 1;
     }
   }
   __syncthreads();
   // Window of previous-chunk blocks around this query block's position, and
   // the reference blocks, outside the budget.
-  for (int pos = j - v.window_half + static_cast<int>(threadIdx.x); pos <= j + v.window_half;
-       pos += kTopkThreads) {
+  for (int pos = j - v.window_half + t; pos <= j + v.window_half; pos += kTopkThreads) {
     const int n = v.prev_first + pos;
     if (pos >= 0 && pos < v.n_prev && n >= 0 && n < nh) flag[n] = 1;
   }
-  for (int r = threadIdx.x; r < v.n_ref; r += kTopkThreads) {
+  for (int r = t; r < v.n_ref; r += kTopkThreads) {
     const int n = v.ref_first + r;
     if (n >= 0 && n < nh) flag[n] = 1;
   }
   __syncthreads();
-  int pos = 0;
-  for (int base = 0; base < nh; base += kTopkThreads) {
-    const int n = base + threadIdx.x;
-    const bool sel = n < nh && flag[n];
-    int tot;
-    const int at = pos + block_excl_count(sel, warp_tot, &tot);
-    if (sel && at < a.max_sel) out[at] = n;
-    pos += tot;
-  }
+  int mine = 0;
+  for (int n = r0; n < r1; ++n) mine += flag[n];
+  int pos;
+  int at = block_excl_scan(mine, warp_tot, &pos);
+  for (int n = r0; n < r1; ++n)
+    if (flag[n]) {
+      if (at < a.max_sel) out[at] = n;
+      ++at;
+    }
   const int c = min(pos, a.max_sel - a.n_own);
-  if (pos + a.n_own > a.max_sel && threadIdx.x == 0) report(a.d_err, BSA_DEV_BAD_COUNT);
-  for (int i = threadIdx.x; i < a.n_own; i += kTopkThreads) out[c + i] = a.own_first + i;
-  for (int i = c + a.n_own + threadIdx.x; i < a.max_sel; i += kTopkThreads) out[i] = -1;
-  if (threadIdx.x == 0) a.cnt[row] = c + a.n_own;
+  if (pos + a.n_own > a.max_sel && t == 0) report(a.d_err, BSA_DEV_BAD_COUNT);
+  for (int i = t; i < a.n_own; i += kTopkThreads) out[c + i] = a.own_first + i;
+  for (int i = c + a.n_own + t; i < a.max_sel; i += kTopkThreads) out[i] = -1;
+  if (t == 0) a.cnt[row] = c + a.n_own;
 }
 
 static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
