@@ -27,7 +27,7 @@ def _coverage(w, n_own, seed):
     return cov
 
 
-def _check_rows(step, idx, cnt, scores, cov, heads, n_ref, ref_first):
+def _check_rows(step, idx, cnt, scores, cov, heads, n_ref, ref_first, P=P):
     w = step.w
     nbc = step.n_own
     prev_first, n_prev = step.own_first - nbc, nbc
@@ -82,8 +82,11 @@ def _check_rows(step, idx, cnt, scores, cov, heads, n_ref, ref_first):
     return ties
 
 
-@pytest.mark.parametrize("chunk,heads", [(6, None), (48, [7])])
-def test_velox_route_matches_oracle(chunk, heads):
+@pytest.mark.parametrize("chunk,heads,k_unc", [(6, None, 150), (48, [7], 150), (12, [3, 20], 300)])
+def test_velox_route_matches_oracle(chunk, heads, k_unc):
+    # K_unc = 150 orders the uncovered budget by counting ranks; K_unc = 300
+    # (more than 256) takes the sorting network.
+    prm = dict(P, k_unc=k_unc)
     w = synth.CONFIGS[4]
     step = hx.build_step(w, DEV, chunk=chunk, pooled_keys=True)
     nbc = step.n_own
@@ -93,12 +96,12 @@ def test_velox_route_matches_oracle(chunk, heads):
         step.q_blk, step.cache, step.n_hist, step.own_first, nbc, g=step.g,
         coverage=torch.from_numpy(cov).to(DEV), lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale,
         prev_first=step.own_first - nbc, n_prev=nbc, ref_first=ref_first, n_ref=n_ref,
-        q_valid=step.q_valid, **P)
+        q_valid=step.q_valid, **prm)
     bsa.raise_on_device_error(DEV)
     heads = list(range(w.Hh)) if heads is None else heads
     scores = hx.oracle_scores_model(step, heads)
     ties = _check_rows(step, idx.cpu().numpy(), cnt.cpu().numpy(), scores, cov, heads, n_ref,
-                       ref_first)
+                       ref_first, prm)
     rows = w.B * len(heads) * nbc
     assert ties <= max(2, rows // 20), f"{ties} near-tie rows of {rows}"
     # Both kinds of rows occur, and the routes really differ in size.
