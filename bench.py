@@ -715,7 +715,7 @@ def run_ours(args, rank, world, local, pg):
         "clocks": clock_info,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(st, args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(args.chunk, args.cpu_seconds)
     if pg is not None:
         pg.destroy_process_group()
     if rank == 0:
@@ -831,49 +831,80 @@ def oracle_sample_step(inputs, n_items):
     return flops
 
 
-def oracle_inputs(st, head=0):
-    h = head
-    valid = st.cache.block_valid.cpu().numpy().astype(np.int64)
+def oracle_sample_base(chunk: int, heads) -> dict:
+    """Inputs of the oracle's timed sample for ``heads`` of chunk ``chunk``,
+    made on the host from the seeded generators alone: every chunk's tokens
+    from ``synth`` (drawn by the CPU generator, so the values differ from
+    the device-drawn ones while shapes and distributions are the same), the
+    prior from ``synth.prior`` and the valid-row counts from the oracle.
+    Nothing here comes from the CUDA path."""
+    import oracle
+    w = synth.CONFIGS[CONFIG_KEY]
+    T, H, W = w.grid
+    nbc = w.blocks_per_chunk
+    hs = list(heads)
+    hist = []
+    for c in range(1, chunk):
+        t = synth.chunk_tokens(w, c, device="cpu", want=("k", "v"))
+        hist.append((t["k"][:, :, hs].clone(), t["v"][:, :, hs].clone()))
+    cur = synth.chunk_tokens(w, chunk, device="cpu")
+    n_hist = nbc * (chunk - 1)
+    valid = np.tile(np.asarray(oracle.block_valid_for(T, H, W), dtype=np.int64), chunk)
+    return {"w": w, "hist": hist, "n_hist": n_hist, "valid": valid,
+            "cur": {n: cur[n][:, :, hs].clone() for n in ("q", "k", "v")},
+            "g": synth.prior(w, chunk, nbc, n_hist) if n_hist > 0 else None}
+
+
+def oracle_inputs(base: dict, i: int) -> dict:
+    """fp64 inputs of the i-th sampled head: its history blocks, scattered by
+    the oracle's own Gilbert order (before the timing), and its current-chunk
+    tokens (scattered inside the timed step)."""
+    import oracle
+    w = base["w"]
+    T, H, W = w.grid
+
+    def hist_blocks(which):
+        parts = [oracle.tokens_to_blocks(kv[which][:, :, i:i + 1].double().numpy(), T, H, W)
+                 for kv in base["hist"]]
+        if not parts:
+            return np.zeros((w.B, 1, 0, BLK, w.D))
+        return np.concatenate(parts, axis=2)
     return {
-        "grid": st.grid, "D": st.w.D, "n_hist": st.n_hist, "top_k": st.w.top_k[0],
-        "k_tok": st.k_tok[:, :, h:h + 1].cpu().double().numpy(),
-        "v_tok": st.v_tok[:, :, h:h + 1].cpu().double().numpy(),
-        "q_tok": st.q_tok[:, :, h:h + 1].cpu().double().numpy(),
-        "k_hist": st.cache.k[:, h:h + 1, :st.n_hist].cpu().double().numpy(),
-        "v_hist": st.cache.v[:, h:h + 1, :st.n_hist].cpu().double().numpy(),
-        "valid": valid, "g": None if st.g is None else st.g.cpu().numpy(),
+        "grid": w.grid, "D": w.D, "n_hist": base["n_hist"], "top_k": w.top_k[0],
+        "k_tok": base["cur"]["k"][:, :, i:i + 1].double().numpy(),
+        "v_tok": base["cur"]["v"][:, :, i:i + 1].double().numpy(),
+        "q_tok": base["cur"]["q"][:, :, i:i + 1].double().numpy(),
+        "k_hist": hist_blocks(0), "v_hist": hist_blocks(1),
+        "valid": base["valid"], "g": base["g"],
     }
 
 
-def cpu_baseline(st, seconds):
-    """Oracle throughput on whole heads of chunk 48 (scatter, route of all 49
-    query blocks, attention of all 49), adding heads until about `seconds`."""
-    flops, dt, heads = 0.0, 0.0, 0
-    while dt < seconds and heads < st.w.Hh:
-        inputs = oracle_inputs(st, head=heads)
+def cpu_baseline(chunk: int, seconds: float, n_heads: int = 2):
+    """Oracle throughput on whole heads of the chunk (scatter, route of all
+    query blocks, attention of all of them), cycling over ``n_heads`` heads
+    until about ``seconds`` of timed work."""
+    w = synth.CONFIGS[CONFIG_KEY]
+    base = oracle_sample_base(chunk, range(n_heads))
+    inputs = [oracle_inputs(base, i) for i in range(n_heads)]
+    flops, dt, steps = 0.0, 0.0, 0
+    while dt < seconds:
         t0 = time.perf_counter()
-        flops += oracle_sample_step(inputs, st.n_own)
+        flops += oracle_sample_step(inputs[steps % n_heads], w.blocks_per_chunk)
         dt += time.perf_counter() - t0
-        heads += 1
+        steps += 1
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": host_cores(),
             "kind": "oracle", "seconds": round(dt, 2),
-            "sample": f"fp64 numpy oracle on heads 0-{heads - 1} of chunk 48 (of 24): Gilbert "
-                      f"scatter of K/V/Q, route of all 49 query blocks, attention of all 49"}
+            "sample": f"fp64 numpy oracle, {steps} whole heads of chunk {chunk} (heads "
+                      f"0-{n_heads - 1} in turn, of {w.Hh}): Gilbert scatter of K/V/Q, route of "
+                      f"all {w.blocks_per_chunk} query blocks, attention of all of them; "
+                      f"inputs drawn on the host from the seeded generators"}
 
 
 def run_reference(args, rank, world):
     """Reference arm: the oracle, as it stands, on the host cores."""
     if rank != 0:
         return
-    import block_sparse_kv_bsa_b200 as bsa  # noqa: F401  (only to build the state on the GPU)
-    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
-    torch.cuda.set_device(device)
-    w = synth.CONFIGS[CONFIG_KEY]
-    st = State(w, args.chunk, device)
-    for _ in range(2):
-        st.step()
-    torch.cuda.synchronize(device)
-    inputs = oracle_inputs(st)
+    inputs = oracle_inputs(oracle_sample_base(args.chunk, [0]), 0)
     n_items = 2
     for _ in range(max(args.warmup, 3)):
         oracle_sample_step(inputs, 1)
@@ -884,8 +915,9 @@ def run_reference(args, rank, world):
         times.append(time.perf_counter() - t0)
     ms = 1e3 * sum(times) / len(times)
     value = flops / (ms * 1e-3) / 1e12
-    sample = (f"fp64 numpy oracle per step: head 0 of chunk 48, Gilbert scatter, route of 49 "
-              f"query blocks, attention of {n_items} query blocks")
+    sample = (f"fp64 numpy oracle per step: head 0 of chunk {args.chunk}, Gilbert scatter, "
+              f"route of 49 query blocks, attention of {n_items} query blocks; inputs drawn "
+              f"on the host from the seeded generators")
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
            "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
