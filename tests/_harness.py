@@ -1,5 +1,9 @@
 """Shared helpers of the GPU parity tests: build a workload's state on the
-device through the library, and hand the same bf16 tensors to the oracle."""
+device through the library, and build the oracle's own inputs from the same
+seeded generators.  The oracle never reads an output of the library: its
+cache is its own Gilbert scatter of the generated tokens, its valid-row
+counts its own, and where a test needs a route for attention, the route is
+the oracle's and the library attends over the same list."""
 from __future__ import annotations
 
 import math
@@ -34,6 +38,9 @@ class Step:
     q_valid: torch.Tensor
     chunk: int
     top_k: int
+    hist_chunks: int = 0      # chunks 1..hist_chunks appended as history (after any direct blocks)
+    qc: int = 1               # the chunk whose tokens form the own chunk
+    device: str = "cuda"
 
 
 def build_step(w: synth.Workload, device="cuda", chunk: Optional[int] = None,
@@ -69,7 +76,7 @@ def build_step(w: synth.Workload, device="cuda", chunk: Optional[int] = None,
     g = torch.from_numpy(g_np).to(device) if g_np is not None else None
     q_valid = cache.block_valid[own_first:own_first + nbc].clone()
     return Step(w, cache, t["q"], q_blk, g, g_np, n_hist, own_first, nbc, q_valid, chunk,
-                w.top_k[0] if top_k is None else top_k)
+                w.top_k[0] if top_k is None else top_k, hist_chunks, qc, str(device))
 
 
 def route(step: Step, **kw):
@@ -78,31 +85,98 @@ def route(step: Step, **kw):
                          sm_scale=step.w.sm_scale, q_valid=step.q_valid, **kw)
 
 
-def oracle_scores(step: Step, heads) -> np.ndarray:
-    """Oracle fused scores s' [B, len(heads), n_own, n_hist] on the same bf16 inputs."""
+def oracle_valid(step: Step) -> np.ndarray:
+    """The oracle's valid-row count of every cache block: direct blocks full,
+    each appended chunk's from its own grid."""
     import oracle
-    q = f64(step.q_blk[:, heads])
-    kc = f64(step.cache.k[:, heads, :step.n_hist])
-    valid = step.cache.block_valid.cpu().numpy()
+    T, H, W = step.w.grid
+    per = np.asarray(oracle.block_valid_for(T, H, W), dtype=np.int64)
+    return np.concatenate([np.full(step.w.hist_direct, BLK, dtype=np.int64),
+                           np.tile(per, step.hist_chunks + 1)])
+
+
+def oracle_blocks(step: Step, pairs, want_v: bool = True) -> dict:
+    """The oracle's Q blocks and K/V cache of each (b, h) in ``pairs``, fp64:
+    {(b, h): (q [1, 1, n_own*128, D], k [1, 1, n_hist+n_own, 128, D], v or
+    None)}.  Built from the seeded generators (the same draws the library
+    appended) by the oracle's own Gilbert scatter."""
+    import oracle
+    w = step.w
+    T, H, W = w.grid
+    pairs = sorted(set(pairs))
+    ks = {p: [] for p in pairs}
+    vs = {p: [] for p in pairs}
+    if w.hist_direct:
+        kd, vd = synth.direct_blocks(w, w.hist_direct, device=step.device)
+        for b, h in pairs:
+            ks[(b, h)].append(f64(kd[b:b + 1, h:h + 1]))
+            if want_v:
+                vs[(b, h)].append(f64(vd[b:b + 1, h:h + 1]))
+    for c in list(range(1, step.hist_chunks + 1)) + [step.qc]:
+        t = synth.chunk_tokens(w, c, device=step.device, want=("k", "v"))
+        for b, h in pairs:
+            ks[(b, h)].append(oracle.tokens_to_blocks(f64(t["k"][b:b + 1, :, h:h + 1]), T, H, W))
+            if want_v:
+                vs[(b, h)].append(oracle.tokens_to_blocks(f64(t["v"][b:b + 1, :, h:h + 1]),
+                                                          T, H, W))
+    out = {}
+    for b, h in pairs:
+        q = oracle.tokens_to_blocks(f64(step.q_tok[b:b + 1, :, h:h + 1]), T, H, W)
+        out[(b, h)] = (q.reshape(1, 1, -1, w.D), np.concatenate(ks[(b, h)], axis=2),
+                       np.concatenate(vs[(b, h)], axis=2) if want_v else None)
+    return out
+
+
+def _oracle_model_scores(step: Step, heads) -> np.ndarray:
+    import oracle
+    w = step.w
+    heads = list(heads)
+    blocks = oracle_blocks(step, [(b, h) for b in range(w.B) for h in heads], want_v=False)
+    q = np.stack([np.stack([blocks[(b, h)][0][0, 0] for h in heads]) for b in range(w.B)])
+    kc = np.stack([np.stack([blocks[(b, h)][1][0, 0, :step.n_hist] for h in heads])
+                   for b in range(w.B)])
+    valid = oracle_valid(step)
     B, Hs, R, D = q.shape
     qm = oracle.pool_blocks(q.reshape(B, Hs, step.n_own, BLK, D),
                             [int(v) for v in valid[step.own_first:step.own_first + step.n_own]])
     km = oracle.pool_blocks(kc, valid[:step.n_hist])
-    s = oracle.block_scores(qm, km, step.w.sm_scale)
+    return oracle.block_scores(qm, km, w.sm_scale)
+
+
+def oracle_scores(step: Step, heads) -> np.ndarray:
+    """Oracle fused scores s' [B, len(heads), n_own, n_hist]."""
+    import oracle
+    s = _oracle_model_scores(step, heads)
     return oracle.fuse_prior(s, step.g_np, step.w.lam, step.w.g_ref)
 
 
 def oracle_scores_model(step: Step, heads) -> np.ndarray:
     """Oracle model scores s = sm_scale * <qmean, kmean> (no prior) [B, len(heads), n_own, n_hist]."""
+    return _oracle_model_scores(step, heads)
+
+
+def oracle_routes(step: Step, heads) -> dict:
+    """The oracle's route of every query block of ``heads``: {(b, h, j): blocks}."""
     import oracle
-    q = f64(step.q_blk[:, heads])
-    kc = f64(step.cache.k[:, heads, :step.n_hist])
-    valid = step.cache.block_valid.cpu().numpy()
-    B, Hs, R, D = q.shape
-    qm = oracle.pool_blocks(q.reshape(B, Hs, step.n_own, BLK, D),
-                            [int(v) for v in valid[step.own_first:step.own_first + step.n_own]])
-    km = oracle.pool_blocks(kc, valid[:step.n_hist])
-    return oracle.block_scores(qm, km, step.w.sm_scale)
+    s = oracle_scores(step, heads)
+    return {(b, h, j): oracle.top_k_with_own(s[b, hi, j], step.top_k, step.own_first, step.n_own)
+            for b in range(step.w.B) for hi, h in enumerate(heads) for j in range(step.n_own)}
+
+
+def attn_routes(step: Step, heads):
+    """Routes for an attention parity test: (idx, cnt, routes).  The query
+    blocks of ``heads`` get the oracle's route, so the library and the oracle
+    attend over the same list, chosen by the oracle; the other heads keep the
+    library's own route (their outputs are not compared)."""
+    idx, cnt = route(step)
+    routes = oracle_routes(step, heads)
+    idx_h, cnt_h = idx.cpu(), cnt.cpu()
+    for (b, h, j), r in routes.items():
+        assert len(r) <= idx_h.shape[-1]
+        idx_h[b, h, j] = -1
+        idx_h[b, h, j, :len(r)] = torch.from_numpy(np.asarray(r, dtype=np.int32))
+        cnt_h[b, h, j] = len(r)
+    return idx_h.to(idx.device), cnt_h.to(cnt.device), routes
 
 
 def check_route_rows(idx: np.ndarray, cnt: np.ndarray, scores: np.ndarray, top_k: int,
@@ -141,23 +215,19 @@ def check_route_rows(idx: np.ndarray, cnt: np.ndarray, scores: np.ndarray, top_k
     return ties
 
 
-def oracle_attn_items(step: Step, idx: torch.Tensor, cnt: torch.Tensor, items, sm_scale=None):
-    """Oracle O and LSE for the listed (b, h, j) items on the GPU's own route."""
+def oracle_attn_items(step: Step, routes: dict, items, sm_scale=None):
+    """Oracle O and LSE of the listed (b, h, j) items over ``routes[(b, h, j)]``,
+    on the oracle's own cache and Q blocks."""
     import oracle
     sm = step.w.sm_scale if sm_scale is None else sm_scale
-    valid = step.cache.block_valid.cpu().numpy()
-    qv = step.q_valid.cpu().numpy()
-    idx_np = idx.cpu().numpy()
-    cnt_np = cnt.cpu().numpy()
+    valid = oracle_valid(step)
+    blocks = oracle_blocks(step, [(b, h) for b, h, _ in items])
     out = []
-    kv = {}
     for (b, h, j) in items:
-        if (b, h) not in kv:
-            kv[(b, h)] = (f64(step.cache.k[b:b + 1, h:h + 1]), f64(step.cache.v[b:b + 1, h:h + 1]))
-        kc, vc = kv[(b, h)]
-        sel = [int(x) for x in idx_np[b, h, j, :cnt_np[b, h, j]]]
-        q = f64(step.q_blk[b:b + 1, h:h + 1, j * BLK:(j + 1) * BLK])
-        o, lse = oracle.attn_block(q, kc, vc, valid, int(qv[j]), 0, 0, 0, sel, sm)
+        q, kc, vc = blocks[(b, h)]
+        sel = [int(x) for x in routes[(b, h, j)]]
+        o, lse = oracle.attn_block(q[:, :, j * BLK:(j + 1) * BLK], kc, vc, valid,
+                                   int(valid[step.own_first + j]), 0, 0, 0, sel, sm)
         out.append((o, lse))
     return out
 

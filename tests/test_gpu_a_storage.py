@@ -130,13 +130,15 @@ def test_pooled_key_means_written_at_append(key):
     T, H, W = w.grid
     nb = w.blocks_per_chunk
     cache = bsa.KVCache(w.B, w.Hh, w.D, 2 * nb, device=DEV, pooled_keys=True)
+    heads = list(range(w.Hh)) if w.Hh <= 12 else [0, 9, w.Hh - 1]
+    blocks = []                                    # the oracle's own scatter of the tokens
     for c in (1, 2):
         t = synth.chunk_tokens(w, c, device=DEV, want=("k", "v"))
         bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+        blocks.append(oracle.tokens_to_blocks(t["k"][:, :, heads].cpu().double().numpy(), T, H, W))
     bsa.raise_on_device_error(DEV)
-    valid = cache.block_valid.cpu().numpy()
-    heads = list(range(w.Hh)) if w.Hh <= 12 else [0, 9, w.Hh - 1]
-    exp = oracle.pool_blocks(cache.k[:, heads].cpu().double().numpy(), valid)
+    valid = np.tile(oracle.block_valid_for(T, H, W), 2)
+    exp = oracle.pool_blocks(np.concatenate(blocks, axis=2), valid)
     got = cache.kmean[:, heads].cpu().double().numpy()
     assert np.allclose(got, exp, rtol=2e-6, atol=2e-7)
 
@@ -152,8 +154,9 @@ def test_pool_means_for_directly_written_blocks():
     cache.n_blocks = 20
     bsa.bsa_kv_pool_means(cache, 0, 20)
     bsa.raise_on_device_error(DEV)
-    valid = cache.block_valid.cpu().numpy()
-    exp = oracle.pool_blocks(cache.k[:, [0, 23]].cpu().double().numpy(), valid)
+    valid = np.full(20, 128)
+    valid[7] = 33
+    exp = oracle.pool_blocks(kd[:, [0, 23]].cpu().double().numpy(), valid)
     assert np.allclose(cache.kmean[:, [0, 23]].cpu().double().numpy(), exp, rtol=2e-6, atol=2e-7)
     with pytest.raises(bsa.BsaError):
         bsa.bsa_kv_pool_means(cache, 15, 10)       # past max_blocks
@@ -185,14 +188,17 @@ def test_append_any_permutation():
     t = synth.chunk_tokens(w, 1, device=DEV, want=("k", "v"))
     _append_raw(cache, t["k"], t["v"], T, H, W, perm)
     bsa.raise_on_device_error(DEV)
+    placed = {}
     for name in ("k", "v"):
         x = t[name].cpu()                                   # [B, N, Hh, D]
         exp = torch.zeros(w.B, w.Hh, nb * 128, w.D, dtype=torch.bfloat16)
         exp[:, :, torch.from_numpy(perm_np).long()] = x.permute(0, 2, 1, 3)
         got = getattr(cache, name).cpu().reshape(w.B, w.Hh, nb * 128, w.D)
         assert torch.equal(got.view(torch.int16), exp.view(torch.int16)), name
-    valid = cache.block_valid.cpu().numpy()
-    exp_m = oracle.pool_blocks(cache.k.cpu().double().numpy(), valid)
+        placed[name] = exp
+    valid = np.bincount(perm_np // 128, minlength=nb)      # tokens landing in each block
+    exp_m = oracle.pool_blocks(placed["k"].double().numpy().reshape(w.B, w.Hh, nb, 128, w.D),
+                               valid)
     assert np.allclose(cache.kmean.cpu().double().numpy(), exp_m, rtol=2e-6, atol=2e-7)
 
 
@@ -229,5 +235,5 @@ def test_append_large_chunk():
     assert np.array_equal(bits(cache.k[:, :, :nb]), bf16_of(exp_k))
     valid = cache.block_valid.cpu().numpy()
     assert np.array_equal(valid[:nb], oracle.block_valid_for(T, H, W))
-    exp_m = oracle.pool_blocks(cache.k[:, :, :nb].cpu().double().numpy(), valid[:nb])
+    exp_m = oracle.pool_blocks(exp_k, oracle.block_valid_for(T, H, W))
     assert np.allclose(cache.kmean[:, :, :nb].cpu().double().numpy(), exp_m, rtol=2e-6, atol=2e-7)
