@@ -55,14 +55,15 @@ def test_route_config4_sweep_chunks(chunk):
     # chunk 1: no history (own chunk only); chunk 2: K >= history (all);
     # chunk 3: K < history; chunk 48: the headline size, one head checked.
     # The row lengths 98, 539, 2303 and 2352 take each register width of the
-    # warp-per-row top-K (up to 512, 1280, 2304 and 3072 blocks).
+    # register top-K (up to 512, 1280, 2304 and 3072 blocks).
     step = hx.build_step(synth.CONFIGS[4], DEV, chunk=chunk)
     _check(step, heads=[5] if chunk >= 12 else [0, 23])
 
 
-def test_route_rows_longer_than_the_warp_select():
-    # 193 history chunks of 16 blocks: rows of 3088 history blocks go to the
-    # block-per-row radix select.
+def test_route_rows_longer_than_the_register_select():
+    # 193 history chunks of 16 blocks: rows of 3088 history blocks are longer
+    # than the register top-K takes (3072), so the shared-memory radix select
+    # routes them.
     step = hx.build_step(synth.CONFIGS[2], DEV, chunk=194)
     assert step.n_hist > 32 * 96
     _check(step, heads=[7])
