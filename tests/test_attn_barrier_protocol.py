@@ -157,7 +157,7 @@ def simulate(n, seed, per_warpgroup_s=False):
              "wg0": softmax(p, n, 0, tokens), "wg1": softmax(p, n, 1, tokens)}
     blocked = {k: None for k in roles}
     seen_gen = {}
-    alive = set(roles)
+    alive = dict.fromkeys(roles)                 # insertion order: the same every run
     idle = 0
     # Each role is slow to look by its own random amount in this run.
     slow = {k: p.rng.uniform(0.0, 0.9) for k in roles}
@@ -173,7 +173,7 @@ def simulate(n, seed, per_warpgroup_s=False):
                 try:
                     blocked[k] = next(roles[k])
                 except StopIteration:
-                    alive.discard(k)
+                    del alive[k]
                     continue
                 if blocked[k][0] == "sync":
                     seen_gen[k] = blocked[k][1].gen
@@ -200,5 +200,5 @@ def test_protocol_drains_in_every_interleaving(n):
 
 
 def test_model_catches_a_barrier_per_warpgroup():
-    faults = [simulate(32, seed, per_warpgroup_s=True) for seed in range(40)]
-    assert any(f is not None for f in faults)
+    faults = [simulate(32, seed, per_warpgroup_s=True) for seed in range(200)]
+    assert sum(f is not None for f in faults) >= 5     # 16 of these 200 interleavings stop
