@@ -19,6 +19,8 @@
 //                  index order by a block-wide ordered compaction, followed by
 //                  the own-chunk blocks.
 // All sums run in fp32 in a fixed order, so results are deterministic.
+#include <cuda.h>
+
 #include <algorithm>
 #include <mutex>
 
@@ -1263,25 +1265,66 @@ constexpr size_t kNoAllocScratchBytes = BSA_ROUTE_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxScratchDevices = 64;
-static void* g_scratch_addr[kMaxScratchDevices];
+struct ScratchEntry {
+  unsigned long long ctx_id;  // unique id of the context the address belongs to
+  void* addr;
+};
+static ScratchEntry g_scratch[kMaxScratchDevices];
 static std::mutex g_scratch_mutex;
 
-// Device address of g_route_scratch on the current device.  Host code cannot
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Driver entry points for the current context and its process-unique id,
+// found through the runtime (the library does not link the driver library).
+static bool context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_route_scratch in the current context.  Host code cannot
 // use the symbol itself (on the host it names a shadow object, not device
-// memory), so the address is looked up once per device, with that device
-// current, and cached.
+// memory), so the address is looked up with the device current.  It belongs
+// to the context that loaded the library's module, so it is cached per device
+// together with that context's process-unique id: a device reset or another
+// context on the device has a new id, and the address is looked up again
+// instead of reusing one that is no longer mapped.
 static bsa_status noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxScratchDevices) return BSA_ERR_UNSUPPORTED;
+  // When no context is current on this thread yet, cudaSetDevice makes the
+  // device's primary context current (it allocates nothing).
+  unsigned long long id = 0;
+  if (!context_id(&id)) {
+    if (cudaSetDevice(dev) != cudaSuccess || !context_id(&id)) return BSA_ERR_CUDA;
+  }
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  ScratchEntry& e = g_scratch[dev];
+  if (e.addr == nullptr || e.ctx_id != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr)
       return BSA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    e.addr = p;
+    e.ctx_id = id;
   }
-  *out = g_scratch_addr[dev];
+  *out = e.addr;
   return BSA_OK;
 }
 

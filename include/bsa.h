@@ -36,8 +36,9 @@
  *              touching memory outside its arguments) and are read back
  *              with bsa_check_device_error.  d_err may be NULL to skip that
  *              reporting.
- *   Threads    Calls are thread-safe: there is no global mutable state
- *              apart from the immutable function table.
+ *   Threads    Calls are thread-safe: the only global mutable state is a
+ *              few small host-side caches (driver entry points, the
+ *              bsa_route_noalloc scratch address), each guarded by a lock.
  */
 #ifndef BSA_H_
 #define BSA_H_
@@ -331,7 +332,12 @@ bsa_status bsa_geometry_prior(const float *cams, int n_cams, float fx, float fy,
  *             (no cudaMalloc, no allocating library routine).
  *   Set-up    the first call on a device looks up that device's address of
  *             the array (cudaGetSymbolAddress, with the device current) and
- *             caches it; make that first call before any stream capture.
+ *             caches it together with the process-unique id of the current
+ *             CUDA context; make that first call before any stream capture.
+ *             The address is only valid in that context: after a device
+ *             reset, or from another context on the device, the id differs
+ *             and the next call looks the address up again (that call is
+ *             then a first call again).
  *   Sharing   every call on a device uses the same array.  Nothing in it has
  *             to start at zero (each call writes every entry it reads), but
  *             calls that overlap on the GPU (different streams, or threads

@@ -73,6 +73,69 @@ def test_attn_config4_chunk48_sample():
     _compare(step, routes, o, lse, items)
 
 
+def test_attn_config4_chunk48_every_query_block_of_two_heads():
+    # The launch the bench times (all 24 heads, 49 query blocks of 113 tiles)
+    # compared on every query block of two heads, the tail block included.
+    step = hx.build_step(synth.CONFIGS[4], DEV, chunk=48)
+    heads = (5, 18)
+    idx, cnt, routes = hx.attn_routes(step, heads)
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    items = [(0, h, j) for h in heads for j in range(step.n_own)]
+    _compare(step, routes, o, lse, items)
+
+
+def _velox_attn_routes(step, heads, cov):
+    """The page's route (Velox constants: tau 0.1, eta_cov 0.9, K_cov 80,
+    K_unc 150, mass 0.9, +/-13 window in the previous chunk) for every query
+    block: the library's own for all heads, replaced on ``heads`` by the
+    oracle's, so both sides attend over the oracle's variable-length lists."""
+    import oracle
+    w = step.w
+    nbc = step.n_own
+    prev_first = step.own_first - nbc
+    idx, cnt = bsa.bsa_route_velox(
+        step.q_blk, step.cache, step.n_hist, step.own_first, nbc, g=step.g,
+        coverage=torch.from_numpy(cov).to(DEV), lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale,
+        tau=0.1, eta_cov=0.9, k_cov=80, k_unc=150, mass=0.9, prev_first=prev_first, n_prev=nbc,
+        window_half=13, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    scores = hx.oracle_scores_model(step, heads)
+    idx_h, cnt_h = idx.cpu(), cnt.cpu()
+    routes = {}
+    for b in range(w.B):
+        for hi, h in enumerate(heads):
+            for j in range(nbc):
+                r = oracle.velox_route_row(scores[b, hi, j], step.g_np[b, j], cov[b, j] >= 0.9, j,
+                                           w.lam, w.g_ref, 0.1, 80, 150, 0.9, prev_first, nbc, 13,
+                                           0, 0, step.own_first, nbc)
+                assert len(r) <= idx_h.shape[-1]
+                idx_h[b, h, j] = -1
+                idx_h[b, h, j, :len(r)] = torch.from_numpy(np.asarray(r, dtype=np.int32))
+                cnt_h[b, h, j] = len(r)
+                routes[(b, h, j)] = r
+    return idx_h.to(DEV), cnt_h.to(DEV), routes
+
+
+def test_attn_on_the_pages_variable_length_routes_chunk48():
+    # Velox, Methodology Steps 5-6: covered query blocks get the previous
+    # chunk plus the best blocks up to K_cov, uncovered ones a mass prefix of
+    # up to K_unc, both joined with the window and the own chunk, so one
+    # launch mixes routes of very different lengths (the bench's velox_route
+    # and geometry_prior lines time exactly this).
+    w = synth.CONFIGS[4]
+    step = hx.build_step(w, DEV, chunk=48, pooled_keys=True)
+    cov = synth.coverage(w, 48, step.n_own)
+    heads = (7, 16)
+    idx, cnt, routes = _velox_attn_routes(step, heads, cov)
+    lens = sorted({len(r) for r in routes.values()})
+    assert len(lens) > 5 and lens[0] < 140 and lens[-1] > 200, lens
+    o, lse = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    items = [(0, h, j) for h in heads for j in range(step.n_own)]
+    _compare(step, routes, o, lse, items)
+
+
 @pytest.mark.parametrize("top_k", [256, 32])
 def test_attn_config5_sample(top_k):
     step = hx.build_step(synth.CONFIGS[5], DEV, top_k=top_k)

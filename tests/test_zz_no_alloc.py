@@ -60,6 +60,16 @@ def test_noalloc_route_matches_workspace_route():
     _same_as_workspace_route(hx.build_step(synth.CONFIGS[2], DEV), calls=1)
 
 
+def test_noalloc_route_from_pooled_keys_and_head_dim_64():
+    # Scores from the pooled-key cache (the product kernels write the scores
+    # into the shared array with their own layout), then the D = 64 kernels.
+    _same_as_workspace_route(hx.build_step(synth.CONFIGS[3], DEV, pooled_keys=True), calls=2)
+    _same_as_workspace_route(hx.build_step(synth.CONFIGS[4], DEV, chunk=12, pooled_keys=True),
+                             calls=1)
+    _same_as_workspace_route(hx.build_step(synth.CONFIGS[1], DEV), calls=2)
+    _same_as_workspace_route(hx.build_step(synth.CONFIGS[1], DEV, pooled_keys=True), calls=1)
+
+
 def test_noalloc_route_rejects_problems_larger_than_its_scratch():
     step = hx.build_step(synth.CONFIGS[1], DEV)
     cs = step.cache.c_struct()
