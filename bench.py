@@ -53,7 +53,7 @@ CHUNK = 48
 BLK = 128
 METRIC = "bsa_attn selected-block TFLOP/s at chunk 48 (48-chunk sweep), 1 B200"
 L2_FLUSH_BYTES = 256 << 20
-KERNELS_PER_STEP = 7  # append (fused), Q to blocks, pool_q, score_means, topk, attn, O to tokens
+KERNELS_PER_STEP = 5  # append (fused), Q to blocks + means, score_means, topk, attn (O to tokens)
 
 
 def parse_args():
@@ -66,10 +66,14 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--chunk", type=int, default=CHUNK)
-    ap.add_argument("--sweep", default="1,2,4,8,12,16,24,32,40,47",
+    ap.add_argument("--sweep", default="all",
                     help="chunks of the 48-chunk sweep at which sparse and dense bsa_attn are "
-                         "timed while the cache is built ('' to skip); chunk 48 itself is the "
-                         "timed workload")
+                         "timed while the cache is built: 'all' (every chunk), a comma list, "
+                         "or '' to skip; chunk 48 itself is the timed workload")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-config measurements (configs 1, 2, 3 and 5)")
+    ap.add_argument("--no-oracle-ops", action="store_true",
+                    help="skip the per-op, per-config oracle timings")
     return ap.parse_args()
 
 
@@ -338,6 +342,119 @@ def sweep_point(bsa, w, cache, q_tok, c, own_first, nbc, device):
             "sparse_ms": round(sp, 4), "dense_ms": round(dn, 4), "speedup": round(dn / sp, 2)}
 
 
+# Every synthetic config measured op by op at 1 GPU: (config, top-K).  The
+# dense-equivalence config runs once with every history block selected
+# (top-K 256 = all 256 history blocks) and once with top-32.
+CONFIG_RUNS = ((1, 3), (2, 16), (3, 50), (5, 256), (5, 32))
+
+
+def _frac(x, peak):
+    return round(x / peak, 4) if peak else None
+
+
+def config_point(key: int, top_k: int, device, peaks: dict, reps: int = 5) -> dict:
+    """One synthetic config, op by op: the cache of its history is built
+    (appended chunks, or blocks written directly and pooled), then the query
+    chunk's append (rewritten in place), Q reordering, route (from the
+    pooled-key cache) and attention are each captured as a CUDA graph and
+    timed after an L2 flush (median of ``reps``).  Each op is reported with
+    its algorithmic bytes or selected FLOPs and its roofline fraction."""
+    import block_sparse_kv_bsa_b200 as bsa
+    w = synth.CONFIGS[key]
+    T, H, W = w.grid
+    nbc = w.blocks_per_chunk
+    n_hist = w.n_hist
+    cache = bsa.KVCache(w.B, w.Hh, w.D, n_hist + nbc, device=device, pooled_keys=True)
+    if w.hist_direct:
+        kd, vd = synth.direct_blocks(w, w.hist_direct, device=device)
+        cache.k[:, :, :w.hist_direct] = kd
+        cache.v[:, :, :w.hist_direct] = vd
+        cache.block_valid[:w.hist_direct] = BLK
+        cache.n_blocks = w.hist_direct
+        bsa.bsa_kv_pool_means(cache, 0, w.hist_direct)
+        del kd, vd
+    for c in range(1, w.hist_chunks + 1):
+        t = synth.chunk_tokens(w, c, device=device, want=("k", "v"))
+        bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+    qc = w.hist_chunks + 1 if w.hist_direct == 0 else 1
+    t = synth.chunk_tokens(w, qc, device=device)
+    own_first = cache.n_blocks
+    bsa.bsa_kv_append(cache, t["k"], t["v"], T, H, W)
+    q_tok, k_tok, v_tok = t["q"], t["k"], t["v"]
+    g = synth.prior(w, qc, nbc, n_hist) if n_hist > 0 else None
+    g = torch.from_numpy(g).to(device) if g is not None else None
+    q_valid = cache.block_valid[own_first:own_first + nbc].clone()
+    q_blk = torch.empty((w.B, w.Hh, nbc * BLK, w.D), dtype=torch.bfloat16, device=device)
+    q_mean = torch.empty((w.B, w.Hh, nbc, w.D), dtype=torch.float32, device=device)
+    bsa.bsa_tokens_to_blocks_mean(q_tok, T, H, W, out=q_blk, mean=q_mean)
+    max_sel = bsa.route_max_sel(top_k, n_hist, nbc)
+    idx = torch.empty((w.B, w.Hh, nbc, max_sel), dtype=torch.int32, device=device)
+    cnt = torch.empty((w.B, w.Hh, nbc), dtype=torch.int32, device=device)
+    ws = torch.empty(max(bsa.bsa_route_workspace_size(w.B, w.Hh, w.D, nbc, n_hist), 256),
+                     dtype=torch.uint8, device=device)
+    o = torch.empty_like(q_blk)
+    lse = torch.empty((w.B, w.Hh, nbc * BLK), dtype=torch.float32, device=device)
+
+    def append():
+        cache.n_blocks = own_first
+        bsa.bsa_kv_append(cache, k_tok, v_tok, T, H, W)
+
+    def route():
+        bsa.bsa_route_qmean(q_mean, cache, n_hist, own_first, nbc, top_k, g=g, lam=w.lam,
+                            g_ref=w.g_ref, sm_scale=w.sm_scale, max_sel=max_sel, idx=idx,
+                            cnt=cnt, workspace=ws)
+
+    def attn():
+        bsa.bsa_attn(q_blk, cache, idx, cnt, q_valid=q_valid, sm_scale=w.sm_scale, o=o, lse=lse)
+
+    route()
+    attn()
+    bsa.raise_on_device_error(device)
+    t_app = _time_call(append, reps)
+    t_q = _time_call(lambda: bsa.bsa_tokens_to_blocks_mean(q_tok, T, H, W, out=q_blk,
+                                                           mean=q_mean), reps)
+    t_route = _time_call(route, reps)
+    t_attn = _time_call(attn, reps)
+    bsa.raise_on_device_error(device)
+    sel = cnt.to(torch.float64)
+    flops = float(sel.sum().item()) * 4.0 * BLK * BLK * w.D
+    tok_b = w.B * w.tokens * w.Hh * w.D * 2
+    blk_b = w.B * w.Hh * nbc * BLK * w.D * 2
+    app_b = 2 * (tok_b + blk_b) + w.B * w.Hh * nbc * w.D * 4
+    qm_b = w.B * w.Hh * nbc * w.D * 4
+    q_b = tok_b + blk_b + qm_b
+    route_b = (qm_b + w.B * w.Hh * n_hist * w.D * 4 + (0 if g is None else g.numel() * 4)
+               + 2 * w.B * w.Hh * nbc * n_hist * 4 + (idx.numel() + cnt.numel()) * 4)
+    hbm, tc = peaks["hbm_gbs"], peaks["bf16_tflops"]
+
+    def gbs(b, ms):
+        return round(b / (ms * 1e-3) / 1e9, 1)
+    out = {
+        "config": key, "name": w.name, "top_k": top_k,
+        "shape": f"B{w.B} Hh{w.Hh} D{w.D}, chunk {T}x{H}x{W} ({nbc} blocks), "
+                 f"{n_hist} history blocks" + (", prior" if g is not None else ""),
+        "selected_blocks_per_query_block": {"min": int(sel.min().item()),
+                                            "max": int(sel.max().item())},
+        "attn": {"ms_per_call": round(t_attn, 4),
+                 "tflops": round(flops / (t_attn * 1e-3) / 1e12, 2),
+                 "frac_of_bf16_peak": _frac(flops / (t_attn * 1e-3) / 1e12, tc),
+                 "selected_tflop_per_call": round(flops / 1e12, 5)},
+        "route": {"ms_per_call": round(t_route, 4), "gbs": gbs(route_b, t_route),
+                  "frac_of_hbm": _frac(route_b / (t_route * 1e-3) / 1e9, hbm),
+                  "bytes_per_call": int(route_b), "keys": "pooled-key cache"},
+        "append": {"ms_per_call": round(t_app, 4), "gbs": gbs(app_b, t_app),
+                   "frac_of_hbm": _frac(app_b / (t_app * 1e-3) / 1e9, hbm),
+                   "bytes_per_call": int(app_b)},
+        "q_to_blocks": {"ms_per_call": round(t_q, 4), "gbs": gbs(q_b, t_q),
+                        "frac_of_hbm": _frac(q_b / (t_q * 1e-3) / 1e9, hbm),
+                        "bytes_per_call": int(q_b)},
+    }
+    if key == 5 and top_k >= n_hist:
+        out["note"] = "every history block selected: dense attention over the cache"
+    del cache
+    return out
+
+
 class State:
     """Device-resident inputs and preallocated outputs of one rank's problem."""
 
@@ -371,21 +488,25 @@ class State:
         g = synth.prior(wr, chunk, nbc, self.n_hist)
         self.g = torch.from_numpy(g).to(device) if g is not None else None
         self.q_blk = torch.empty((w.B, w.Hh, nbc * BLK, w.D), dtype=torch.bfloat16, device=device)
+        self.q_mean = torch.empty((w.B, w.Hh, nbc, w.D), dtype=torch.float32, device=device)
         self.max_sel = bsa.route_max_sel(w.top_k[0], self.n_hist, nbc)
         self.idx = torch.empty((w.B, w.Hh, nbc, self.max_sel), dtype=torch.int32, device=device)
         self.cnt = torch.empty((w.B, w.Hh, nbc), dtype=torch.int32, device=device)
         ws = bsa.bsa_route_workspace_size(w.B, w.Hh, w.D, nbc, self.n_hist)
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
-        self.o_blk = torch.empty_like(self.q_blk)
-        self.lse = torch.empty((w.B, w.Hh, nbc * BLK), dtype=torch.float32, device=device)
+        self.lse = torch.empty((w.B, w.tokens, w.Hh), dtype=torch.float32, device=device)
         self.o_tok = torch.empty_like(self.q_tok)
-        self.call_graphs = []
+        self.side = torch.cuda.Stream(device)
+        self.step_graph = None
         bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W)
         torch.cuda.synchronize(device)
         self.q_valid = self.cache.block_valid[self.own_first:self.own_first + nbc].clone()
 
     def calls(self):
-        """The five library calls of one step, in order, as (name, fn)."""
+        """The four library calls of one step, in order, as (name, fn): the
+        query chunk is reordered and pooled in one pass, the route scores
+        from those means (so the query blocks are read once), and the
+        attention writes O and LSE straight back in raster token order."""
         bsa, w = self.bsa, self.w
         T, H, W = self.grid
 
@@ -394,82 +515,120 @@ class State:
             bsa.bsa_kv_append(self.cache, self.k_tok, self.v_tok, T, H, W)
         return [
             ("append", append),
-            ("q_to_blocks", lambda: bsa.bsa_tokens_to_blocks(self.q_tok, T, H, W,
-                                                             out=self.q_blk)),
-            ("route", lambda: bsa.bsa_route(
-                self.q_blk, self.cache, self.n_hist, self.own_first, self.n_own, w.top_k[0],
-                g=self.g, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale, q_valid=self.q_valid,
-                max_sel=self.max_sel, idx=self.idx, cnt=self.cnt, workspace=self.ws)),
-            ("attn", lambda: bsa.bsa_attn(self.q_blk, self.cache, self.idx, self.cnt,
-                                          q_valid=self.q_valid, sm_scale=w.sm_scale,
-                                          o=self.o_blk, lse=self.lse)),
-            ("o_to_tokens", lambda: bsa.bsa_blocks_to_tokens(self.o_blk, T, H, W,
-                                                             out=self.o_tok)),
+            ("q_to_blocks", lambda: bsa.bsa_tokens_to_blocks_mean(
+                self.q_tok, T, H, W, out=self.q_blk, mean=self.q_mean)),
+            ("route", lambda: bsa.bsa_route_qmean(
+                self.q_mean, self.cache, self.n_hist, self.own_first, self.n_own, w.top_k[0],
+                g=self.g, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale, max_sel=self.max_sel,
+                idx=self.idx, cnt=self.cnt, workspace=self.ws)),
+            ("attn", lambda: bsa.bsa_attn_tokens(self.q_blk, self.cache, self.idx, self.cnt,
+                                                 T, H, W, q_valid=self.q_valid,
+                                                 sm_scale=w.sm_scale, o=self.o_tok,
+                                                 lse=self.lse)),
         ]
 
-    def step(self):
-        """One pass of the whole path through the library's calls."""
-        for _, fn in self.calls():
-            fn()
+    def step(self, record=None):
+        """One pass of the whole path through the library's calls.
+
+        The append of the chunk's K/V and the route do not depend on each
+        other (the route reads only the history's pooled keys and valid
+        counts, the append writes only the chunk's own blocks), so the
+        append runs on a side stream while the route runs: the HBM-bound
+        append fills the time of the latency-bound route kernels (started
+        together with the HBM-bound Q reordering instead, the two streams
+        only slowed each other).  The attention waits for both.
+        ``record(i, stream)`` marks the event points 0..5: start, Q
+        reordered, append done (side stream), routed, joined, attention done
+        (O in token order)."""
+        main = torch.cuda.current_stream(self.device)
+        calls = dict(self.calls())
+        mark = record if record is not None else (lambda i, stream: None)
+        mark(0, main)
+        calls["q_to_blocks"]()
+        mark(1, main)
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            calls["append"]()
+            mark(2, self.side)
+        calls["route"]()
+        mark(3, main)
+        main.wait_stream(self.side)
+        mark(4, main)
+        calls["attn"]()
+        mark(5, main)
+
+    # (name, first event, last event) of each timed span of a step
+    SPANS = (("q_to_blocks", 0, 1), ("append", 1, 2), ("route", 1, 3), ("attn", 4, 5),
+             ("step", 0, 5))
+    N_EVENTS = 6
 
     def capture(self):
-        """The step as CUDA graphs, with CUDA events before, between and after
-        its calls.  Preferred: one graph for the whole step whose event-record
-        nodes (cudaEventRecordExternal) time the calls; replaying one graph
-        instead of five saves ~7 us of launch latency per call boundary.  The
-        node events are rewritten by every replay, so each step is read back
-        before the next.  Fallback (runtime entry point not found): one graph
-        per call with the events recorded between the replays."""
+        """The step as one CUDA graph (the side stream's fork and join become
+        graph edges) with event-record nodes (cudaEventRecordExternal) at the
+        step's event points.  The node events are rewritten by every replay,
+        so each step is read back before the next.  Fallback (runtime entry
+        point not found): the graph without event nodes, with events
+        recorded around the replay only (per-call times then come from
+        isolated per-call graphs)."""
         self.call_names = [name for name, _ in self.calls()]
-        self.step_graph, self.call_graphs = None, []
-        self.node_events = [torch.cuda.Event(enable_timing=True)
-                            for _ in range(len(self.call_names) + 1)]
+        self.step_graph = None
+        self.node_events = [torch.cuda.Event(enable_timing=True) for _ in range(self.N_EVENTS)]
         for e in self.node_events:
             e.record()                   # creates the events before the capture
         torch.cuda.synchronize(self.device)
         record = _external_event_record()
         if record is not None:
-            def step_with_nodes():
-                s = torch.cuda.current_stream(self.device).cuda_stream
-                _cuda_ok(record(self.node_events[0].cuda_event, s, 1))
-                for i, (_, fn) in enumerate(self.calls()):
-                    fn()
-                    _cuda_ok(record(self.node_events[i + 1].cuda_event, s, 1))
-            self.step_graph = capture(step_with_nodes)
+            def mark(i, stream):
+                _cuda_ok(record(self.node_events[i].cuda_event, stream.cuda_stream, 1))
+            self.step_graph = capture(lambda: self.step(mark))
+            self.node_timing = True
         else:
-            self.call_graphs = [(name, capture(fn)) for name, fn in self.calls()]
-        self.timing = ("one CUDA graph per step, event-record nodes between the calls"
-                       if self.step_graph is not None else
-                       "one CUDA graph per call, events recorded between the replays")
+            self.step_graph = capture(self.step)
+            self.node_timing = False
+        self.timing = ("one CUDA graph per step (append on a forked stream, overlapping the "
+                       "route), event-record nodes at the step's event points"
+                       if self.node_timing else
+                       "one CUDA graph per step (append on a forked stream), events around "
+                       "the replay")
 
     def replay(self):
-        """One step from the captured graph(s); then self.read_times() gives
-        the per-call times (ms), after the step has completed."""
-        if self.step_graph is not None:
+        """One step from the captured graph; then self.read_times() gives the
+        span times (ms) of SPANS, after the step has completed."""
+        if self.node_timing:
             self.step_graph.replay()
             return
         ev = self.node_events
         ev[0].record()
-        for i, (_, g) in enumerate(self.call_graphs):
-            g.replay()
-            ev[i + 1].record()
+        self.step_graph.replay()
+        ev[-1].record()
 
     def read_times(self):
         ev = self.node_events
-        return [ev[i].elapsed_time(ev[i + 1]) for i in range(len(ev) - 1)]
+        if not self.node_timing:
+            return {"step": ev[0].elapsed_time(ev[-1])}
+        return {name: ev[a].elapsed_time(ev[b]) for name, a, b in self.SPANS}
+
+    def isolated_ms(self, reps: int = 10) -> dict:
+        """Each call of the step timed on its own (a CUDA graph of the call,
+        replayed after an L2 flush, median of ``reps``): the per-call
+        figures behind the HBM fractions, free of the overlap inside a step."""
+        return {name: _time_call(fn, reps) for name, fn in self.calls()}
 
     def release_graphs(self):
-        self.step_graph, self.call_graphs = None, []
+        self.step_graph = None
 
     def route_bytes(self, from_means: bool = True) -> float:
-        """Algorithmic bytes of bsa_route: Q read, the history key means (or the
-        history keys themselves when streaming), g read, model scores written
-        and read back by top-K, idx/cnt written."""
+        """Algorithmic bytes of the route.  From means (bsa_route_qmean on the
+        pooled-key cache): the query means and the history key means read.
+        Streaming (bsa_route on the query blocks, no pooled-key cache): the
+        query blocks and every history key block read.  Both: g read, model
+        scores written and read back by top-K, idx/cnt written."""
         w = self.w
-        q = w.B * w.Hh * self.n_own * BLK * w.D * 2
         if from_means:
+            q = w.B * w.Hh * self.n_own * w.D * 4
             k = w.B * w.Hh * self.n_hist * w.D * 4
         else:
+            q = w.B * w.Hh * self.n_own * BLK * w.D * 2
             k = w.B * w.Hh * self.n_hist * BLK * w.D * 2
         g = 0 if self.g is None else self.g.numel() * 4
         s = 2 * w.B * w.Hh * self.n_own * self.n_hist * 4
@@ -497,7 +656,7 @@ class State:
         idx, cnt = bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist, self.own_first,
                                        self.n_own, **kw)
         o = torch.empty_like(self.q_blk)
-        lse = torch.empty_like(self.lse)
+        lse = torch.empty(self.q_blk.shape[:3], dtype=torch.float32, device=self.device)
         rt = _time_call(lambda: bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist,
                                                     self.own_first, self.n_own, idx=idx,
                                                     cnt=cnt, **kw), reps)
@@ -543,7 +702,7 @@ class State:
         idx, cnt = bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist, self.own_first,
                                        self.n_own, **kw)
         o = torch.empty_like(self.q_blk)
-        lse = torch.empty_like(self.lse)
+        lse = torch.empty(self.q_blk.shape[:3], dtype=torch.float32, device=self.device)
         rt = _time_call(lambda: bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist,
                                                     self.own_first, self.n_own, idx=idx,
                                                     cnt=cnt, **kw), 10)
@@ -585,11 +744,34 @@ class State:
         return c * 4.0 * BLK * BLK * self.w.D
 
 
+def append_entry(st, ms: float, in_step_ms, peaks: dict, traffic) -> dict:
+    """The append's figures: algorithmic bytes over its isolated time, and,
+    beside them, the DRAM bytes one ncu capture measured over the same time.
+    Part of the append's writes are still in L2 when it ends (they reach
+    DRAM during the next kernels), so the DRAM figure is the lower one."""
+    b = st.append_bytes()
+    out = {"ms_per_call": round(ms, 4),
+           "in_step_ms": round(in_step_ms, 4) if in_step_ms is not None else None,
+           "gbs": round(b / (ms * 1e-3) / 1e9, 1),
+           "frac_of_hbm": round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+           "bytes_per_call": int(b), "traffic": traffic}
+    if traffic:
+        out["dram_gbs"] = round(traffic / (ms * 1e-3) / 1e9, 1)
+        out["dram_frac_of_hbm"] = round(traffic / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
+        out["dram_note"] = ("traffic = DRAM bytes of one ncu capture; writes still in L2 at "
+                            "the kernel's end are not in it")
+    return out
+
+
 def run_ours(args, rank, world, local, pg):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = synth.CONFIGS[CONFIG_KEY]
-    sweep = {int(x) for x in args.sweep.split(",") if x.strip()} if rank == 0 else set()
+    sweep = set()
+    if rank == 0 and args.sweep.strip() == "all":
+        sweep = set(range(1, args.chunk))
+    elif rank == 0:
+        sweep = {int(x) for x in args.sweep.split(",") if x.strip()}
     st = State(w, args.chunk, device, seed_rank=rank, sweep_chunks=sweep)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     _flush_bufs[device] = flush            # the same buffer for the per-call timings
@@ -626,17 +808,22 @@ def run_ours(args, rank, world, local, pg):
     barrier(pg, device)
     t_wall1 = time.time()
     st.bsa.raise_on_device_error(device)
-    per_step = [sum(t) for t in step_times]
+    per_step = [t["step"] for t in step_times]
     total_ms = max_over_ranks(sum(per_step), pg, device)
-    # Per-call times from the same timed region: the events between calls.
-    phase_ms = {name: sum(t[i] for t in step_times) / args.steps
-                for i, name in enumerate(st.call_names)}
+    st.release_graphs()
+    # Each call alone (its own graph, L2 flushed): the figures behind the
+    # per-call HBM fractions, since inside a step the append overlaps the
+    # Q reorder and the route.
+    isolated = {k: max_over_ranks(v, pg, device) for k, v in st.isolated_ms().items()}
+    # Span times from the timed region itself (event nodes of the step graph);
+    # the attention span has the GPU to itself.
+    phase_ms = {name: sum(t[name] for t in step_times) / args.steps
+                for name, _, _ in st.SPANS if name in step_times[0]}
     phase_ms = {k: max_over_ranks(v, pg, device) for k, v in phase_ms.items()}
-    attn_avg = phase_ms["attn"]
+    attn_avg = phase_ms.get("attn", isolated["attn"])
     spread = sorted(per_step)
     step_spread = {"min": round(spread[0], 4), "median": round(spread[len(spread) // 2], 4),
                    "max": round(spread[-1], 4)}
-    st.release_graphs()
     clock_info = None
     if clocks is not None:
         time.sleep(0.3)
@@ -652,6 +839,9 @@ def run_ours(args, rank, world, local, pg):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(st, args, device, pg, flops)
+    per_config = None
+    if rank == 0 and not args.no_configs:
+        per_config = [config_point(k, kk, device, load_peaks()) for k, kk in CONFIG_RUNS]
 
     ms_per_step = total_ms / args.steps
     value = flops * world / (ms_per_step * 1e-3) / 1e12
@@ -681,11 +871,16 @@ def run_ours(args, rank, world, local, pg):
         "attn": {"ms_per_call": round(attn_avg, 4), "tflops": round(attn_tflops, 2),
                  "selected_tflop_per_call": round(flops / 1e12, 4)},
         "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()},
+        "phases_note": "spans inside the timed steps: append runs on a forked stream while "
+                       "the route runs, so those two overlap; q_to_blocks and attn (which "
+                       "writes O and LSE in token order) have the GPU to themselves",
+        "isolated_ms": {k: round(v, 4) for k, v in isolated.items()},
         "step_ms_spread": step_spread,
         "timing": st.timing + "; each step read back before the next",
-        "route": {"ms_per_call": round(phase_ms["route"], 4),
+        "route": {"ms_per_call": round(isolated["route"], 4),
+                  "in_step_ms": round(phase_ms["route"], 4) if "route" in phase_ms else None,
                   "keys": "pooled-key cache (means written by bsa_kv_append)",
-                  "gbs": round(st.route_bytes() / (phase_ms["route"] * 1e-3) / 1e9, 1),
+                  "gbs": round(st.route_bytes() / (isolated["route"] * 1e-3) / 1e9, 1),
                   "bytes_per_call": int(st.route_bytes())},
         "route_stream": {"ms_per_call": round(route_stream, 4),
                          "keys": "history keys streamed from the cache (no pooled-key cache)",
@@ -695,28 +890,28 @@ def run_ours(args, rank, world, local, pg):
                          "bytes_per_call": int(st.route_bytes(False)),
                          "pool_score_traffic": (measured_traffic("pool_score_kernel<16>")
                                                 if args.chunk == CHUNK else None)},
-        "append": {"ms_per_call": round(phase_ms["append"], 4),
-                   "gbs": round(st.append_bytes() / (phase_ms["append"] * 1e-3) / 1e9, 1),
-                   "frac_of_hbm": round(st.append_bytes() / (phase_ms["append"] * 1e-3) / 1e9
-                                        / peaks["hbm_gbs"], 4),
-                   "bytes_per_call": int(st.append_bytes()),
-                   "traffic": (append_traffic() if args.chunk == CHUNK else None)},
+        "append": append_entry(st, isolated["append"], phase_ms.get("append"), peaks,
+                               append_traffic() if args.chunk == CHUNK else None),
         "roofline": {"bound": "tensor", "achieved": round(attn_tflops, 2),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} burst dense bf16 (cuBLAS)",
-                     "kernel": "bsa_attn_kernel<128>",
+                     "kernel": "bsa_attn_kernel<128, true>",
                      "traffic": (measured_traffic("bsa_attn_kernel<128>")
                                  if args.chunk == CHUNK else None)},
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "sweep": st.sweep,
+        "per_config": per_config,
         "velox_route": velox,
         "geometry_prior": geometry,
         "clocks": clock_info,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args.chunk, args.cpu_seconds)
+        base = oracle_sample_base(args.chunk, range(2))
+        out["cpu_baseline"] = cpu_baseline(args.chunk, args.cpu_seconds, base=base)
+        if not args.no_oracle_ops and args.chunk == CHUNK:
+            out["cpu_baseline"]["per_op"] = oracle_per_config(base)
     if pg is not None:
         pg.destroy_process_group()
     if rank == 0:
@@ -880,12 +1075,13 @@ def oracle_inputs(base: dict, i: int) -> dict:
     }
 
 
-def cpu_baseline(chunk: int, seconds: float, n_heads: int = 2):
+def cpu_baseline(chunk: int, seconds: float, n_heads: int = 2, base=None):
     """Oracle throughput on whole heads of the chunk (scatter, route of all
     query blocks, attention of all of them), cycling over ``n_heads`` heads
     until about ``seconds`` of timed work."""
     w = synth.CONFIGS[CONFIG_KEY]
-    base = oracle_sample_base(chunk, range(n_heads))
+    if base is None:
+        base = oracle_sample_base(chunk, range(n_heads))
     inputs = [oracle_inputs(base, i) for i in range(n_heads)]
     flops, dt, steps = 0.0, 0.0, 0
     while dt < seconds:
@@ -899,6 +1095,122 @@ def cpu_baseline(chunk: int, seconds: float, n_heads: int = 2):
                       f"0-{n_heads - 1} in turn, of {w.Hh}): Gilbert scatter of K/V/Q, route of "
                       f"all {w.blocks_per_chunk} query blocks, attention of all of them; "
                       f"inputs drawn on the host from the seeded generators"}
+
+
+def _oracle_case(w, chunk: int, hist_kv, cur: dict) -> dict:
+    """fp64 inputs of head (0, 0) of a config for the oracle's per-op timing:
+    the history blocks (the oracle's own Gilbert scatter of the seeded
+    history tokens, or the blocks written directly), the query chunk's raster
+    tokens, the valid-row counts and the prior.  Made on the host from the
+    seeded generators; nothing comes from the CUDA path."""
+    import oracle
+    T, H, W = w.grid
+    nbc = w.blocks_per_chunk
+
+    def head(x):
+        return x[:1, :, :1].double().numpy()
+    parts_k, parts_v = [], []
+    valid = []
+    if w.hist_direct:
+        kd, vd = synth.direct_blocks(w, w.hist_direct, device="cpu")
+        parts_k.append(kd[:1, :1].double().numpy())
+        parts_v.append(vd[:1, :1].double().numpy())
+        valid.append(np.full(w.hist_direct, BLK, dtype=np.int64))
+    per = np.asarray(oracle.block_valid_for(T, H, W), dtype=np.int64)
+    for k, v in hist_kv:
+        parts_k.append(oracle.tokens_to_blocks(head(k), T, H, W))
+        parts_v.append(oracle.tokens_to_blocks(head(v), T, H, W))
+        valid.append(per)
+    valid.append(per)
+    n_hist = sum(x.shape[2] for x in parts_k)
+    g = synth.prior(w, chunk, nbc, n_hist) if n_hist > 0 else None
+    return {"w": w, "grid": (T, H, W), "n_hist": n_hist,
+            "k_hist": np.concatenate(parts_k, axis=2) if parts_k else
+            np.zeros((1, 1, 0, BLK, w.D)),
+            "v_hist": np.concatenate(parts_v, axis=2) if parts_v else
+            np.zeros((1, 1, 0, BLK, w.D)),
+            "valid": np.concatenate(valid), "g": None if g is None else g[:1],
+            "q_tok": head(cur["q"]), "k_tok": head(cur["k"]), "v_tok": head(cur["v"])}
+
+
+def _timed(fn, min_s: float = 0.2, max_reps: int = 3):
+    """Median wall time (s) of fn() over 1..max_reps runs (stops after min_s)."""
+    ts = []
+    while len(ts) < max_reps and (not ts or sum(ts) < min_s):
+        t0 = time.perf_counter()
+        fn()
+        ts.append(time.perf_counter() - t0)
+    return sorted(ts)[len(ts) // 2]
+
+
+def oracle_op_times(case: dict, top_k: int, attn_items: int = 2) -> dict:
+    """The oracle, as it stands, timed op by op on head (0, 0) of a config,
+    each op scaled to a full call of the config by its unit count: the
+    append by the (batch, head) pairs, the route likewise, the attention by
+    the (batch, head, query block) items."""
+    import oracle
+    w = case["w"]
+    T, H, W = case["grid"]
+    nbc = w.blocks_per_chunk
+    n_hist = case["n_hist"]
+    sm = w.sm_scale
+    t_app = _timed(lambda: (oracle.tokens_to_blocks(case["k_tok"], T, H, W),
+                            oracle.tokens_to_blocks(case["v_tok"], T, H, W)))
+    kb = oracle.tokens_to_blocks(case["k_tok"], T, H, W)
+    vb = oracle.tokens_to_blocks(case["v_tok"], T, H, W)
+    qb = oracle.tokens_to_blocks(case["q_tok"], T, H, W).reshape(1, 1, nbc * BLK, w.D)
+    kc = np.concatenate([case["k_hist"], kb], axis=2)
+    vc = np.concatenate([case["v_hist"], vb], axis=2)
+    valid = case["valid"]
+    res = {}
+
+    def rt():
+        res["idx"], _ = oracle.route(qb, kc, valid, n_hist, n_hist, nbc, case["g"], w.lam,
+                                     w.g_ref, sm, top_k)
+    t_route = _timed(rt)
+    sel = res["idx"][0][0]
+    m = min(attn_items, nbc)
+
+    def at():
+        for j in range(m):
+            oracle.attn_block(qb, kc, vc, valid, int(valid[n_hist + j]), 0, 0, j, sel[j], sm)
+    t_attn = _timed(at) / m
+    pairs = w.B * w.Hh
+    return {"append_ms": round(1e3 * t_app * pairs, 2),
+            "route_ms": round(1e3 * t_route * pairs, 2),
+            "attn_ms": round(1e3 * t_attn * pairs * nbc, 2),
+            "sample": f"head (0, 0): append and route of the whole head, attention of "
+                      f"{m} query block(s); scaled by {pairs} (batch, head) pairs and "
+                      f"{pairs * nbc} attention items"}
+
+
+def oracle_per_config(base48: dict) -> dict:
+    """Per-op oracle timings for every config run and for the 48-chunk
+    sweep at chunks 1, 12, 24 and 48 (the history of the sweep is shared
+    with the whole-path CPU baseline's)."""
+    out = {"cores": host_cores(), "kind": "oracle", "configs": [], "sweep_chunks": []}
+    done = {}
+    for key, top_k in CONFIG_RUNS:
+        w = synth.CONFIGS[key]
+        if key not in done:
+            hist = [tuple(synth.chunk_tokens(w, c, device="cpu", want=("k", "v"))[n]
+                          for n in ("k", "v")) for c in range(1, w.hist_chunks + 1)]
+            qc = w.hist_chunks + 1 if w.hist_direct == 0 else 1
+            done[key] = _oracle_case(w, qc, hist, synth.chunk_tokens(w, qc, device="cpu"))
+        out["configs"].append({"config": key, "top_k": top_k,
+                               **oracle_op_times(done[key], top_k)})
+    w4 = synth.CONFIGS[CONFIG_KEY]
+    for c in (1, 12, 24, 48):
+        if c == 48:
+            cur = {n: base48["cur"][n] for n in ("q", "k", "v")}
+        else:
+            t = synth.chunk_tokens(w4, c, device="cpu", want=("q",))
+            cur = {"q": t["q"][:, :, :1], "k": base48["hist"][c - 1][0],
+                   "v": base48["hist"][c - 1][1]}
+        case = _oracle_case(w4, c, base48["hist"][:c - 1], cur)
+        out["sweep_chunks"].append({"chunk": c, "top_k": w4.top_k[0],
+                                    **oracle_op_times(case, w4.top_k[0])})
+    return out
 
 
 def run_reference(args, rank, world):

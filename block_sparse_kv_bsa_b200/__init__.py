@@ -12,8 +12,11 @@ The functions carry the C names:
 * :func:`bsa_gilbert_perm` - host Gilbert order of a T x H x W chunk
 * :func:`bsa_kv_append` - scatter a chunk's K/V into the block cache
 * :func:`bsa_tokens_to_blocks` / :func:`bsa_blocks_to_tokens` - reorder Q / O
+* :func:`bsa_tokens_to_blocks_mean` - reorder Q and pool its blocks in one pass
 * :func:`bsa_route` - pooled-score top-K route per query block
+* :func:`bsa_route_qmean` - the same route from precomputed query means
 * :func:`bsa_attn` - indexed block-sparse attention (O and LSE)
+* :func:`bsa_attn_tokens` - the same with O and LSE in raster token order
 * :func:`bsa_check_device_error` - read and clear the device error word
 
 Method: "Velox: Spatial Memory Makes World Models Efficient" (Key
@@ -44,8 +47,9 @@ DEV_CODES = {0: "BSA_DEV_OK", 1: "BSA_DEV_BAD_INDEX", 2: "BSA_DEV_BAD_COUNT",
 # Every symbol include/bsa.h declares (checked by the tests).
 EXPORTS = ("bsa_abi_version", "bsa_status_string", "bsa_gilbert_perm", "bsa_kv_append",
            "bsa_kv_pool_means",
-           "bsa_tokens_to_blocks", "bsa_blocks_to_tokens", "bsa_route_workspace_size",
-           "bsa_route", "bsa_route_velox", "bsa_route_noalloc", "bsa_attn",
+           "bsa_tokens_to_blocks", "bsa_tokens_to_blocks_mean", "bsa_blocks_to_tokens",
+           "bsa_route_workspace_size", "bsa_route", "bsa_route_qmean", "bsa_route_velox",
+           "bsa_route_noalloc", "bsa_attn", "bsa_attn_tokens",
            "bsa_geometry_prior",
            "bsa_check_device_error",
            "bsa_selftest_bounded_wait")
@@ -94,10 +98,13 @@ _sig = {
     "bsa_kv_append": (_i, [ctypes.POINTER(CCache), _p, _p, _i, _i, _i, _p, _p, _p]),
     "bsa_kv_pool_means": (_i, [ctypes.POINTER(CCache), _i, _i, _p, _p]),
     "bsa_tokens_to_blocks": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
+    "bsa_tokens_to_blocks_mean": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "bsa_blocks_to_tokens": (_i, [_p, _p, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "bsa_route_workspace_size": (_i, [_i, _i, _i, _i, _i, ctypes.POINTER(_sz)]),
     "bsa_route": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f, _i,
                        _p, _p, _i, _p, _sz, _p, _p]),
+    "bsa_route_qmean": (_i, [_p, ctypes.POINTER(CCache), _i, _i, _i, _p, _f, _f, _f, _i,
+                             _p, _p, _i, _p, _sz, _p, _p]),
     "bsa_geometry_prior": (_i, [_p, _i, _f, _f, _f, _f, _p, _p, _i, _p, _p, _i, _i, _i, _p, _p,
                                 _p, _i, _p, _p, _p, _p]),
     "bsa_route_velox": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f,
@@ -105,6 +112,8 @@ _sig = {
     "bsa_route_noalloc": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f, _i,
                                _p, _p, _i, _p, _p]),
     "bsa_attn": (_i, [_p, ctypes.POINTER(CCache), _p, _p, _p, _i, _i, _f, _p, _p, _p, _p]),
+    "bsa_attn_tokens": (_i, [_p, ctypes.POINTER(CCache), _p, _p, _p, _i, _f, _i, _i, _i, _p, _p,
+                             _p, _p, _p]),
     "bsa_check_device_error": (_i, [_p, _p, ctypes.POINTER(ctypes.c_int32)]),
     "bsa_selftest_bounded_wait": (_i, [_p, ctypes.c_longlong, _p]),
 }
@@ -285,6 +294,30 @@ def bsa_tokens_to_blocks(x_tok: torch.Tensor, T: int, H: int, W: int,
     return out
 
 
+def bsa_tokens_to_blocks_mean(x_tok: torch.Tensor, T: int, H: int, W: int,
+                              out: Optional[torch.Tensor] = None,
+                              mean: Optional[torch.Tensor] = None
+                              ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """bsa_tokens_to_blocks plus the fp32 mean of every block's valid rows:
+    returns (blocks [B, Hh, nb*128, D], means [B, Hh, nb, D])."""
+    if x_tok.dim() != 4:
+        raise ValueError("x_tok must be [B, T*H*W, Hh, D]")
+    B, N, Hh, D = x_tok.shape
+    _need(x_tok, "x_tok", torch.bfloat16)
+    nb = n_blocks_for(T, H, W)
+    if out is None:
+        out = torch.empty((B, Hh, nb * BLK, D), dtype=torch.bfloat16, device=x_tok.device)
+    if mean is None:
+        mean = torch.empty((B, Hh, nb, D), dtype=torch.float32, device=x_tok.device)
+    _need(out, "out", torch.bfloat16, x_tok.device, (B, Hh, nb * BLK, D))
+    _need(mean, "mean", torch.float32, x_tok.device, (B, Hh, nb, D))
+    perm = gilbert_perm_device(T, H, W, x_tok.device)
+    _check("bsa_tokens_to_blocks_mean", _lib.bsa_tokens_to_blocks_mean(
+        _ptr(x_tok), _ptr(out), _ptr(mean), B, Hh, D, int(T), int(H), int(W), _ptr(perm),
+        _ptr(error_word(x_tok.device)), _stream(x_tok.device)))
+    return out, mean
+
+
 def bsa_blocks_to_tokens(x_blk: torch.Tensor, T: int, H: int, W: int,
                          out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """[B, Hh, nb*128, D] Gilbert blocks -> [B, T*H*W, Hh, D] raster tokens."""
@@ -350,6 +383,41 @@ def bsa_route(q_blk: torch.Tensor, cache: KVCache, n_hist: int, own_first: int, 
     _check("bsa_route", _lib.bsa_route(
         _ptr(q_blk), ctypes.byref(cs), _ptr(q_valid), int(n_hist), int(own_first), int(n_own),
         _ptr(g), float(lam), float(g_ref), float(sm_scale), int(top_k), _ptr(idx), _ptr(cnt),
+        int(max_sel), _ptr(workspace), workspace.numel(), _ptr(error_word(dev)), _stream(dev)))
+    return idx, cnt
+
+
+def bsa_route_qmean(q_mean: torch.Tensor, cache: KVCache, n_hist: int, own_first: int,
+                    n_own: int, top_k: int, g: Optional[torch.Tensor] = None, lam: float = 2.0,
+                    g_ref: float = 0.2, sm_scale: Optional[float] = None,
+                    max_sel: Optional[int] = None, idx: Optional[torch.Tensor] = None,
+                    cnt: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None
+                    ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """bsa_route from the query-block means [B, Hh, n_own, D] (fp32), e.g.
+    those of bsa_tokens_to_blocks_mean; returns (idx, cnt)."""
+    dev = cache.device
+    _need(q_mean, "q_mean", torch.float32, dev, (cache.B, cache.Hh, n_own, cache.D))
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(cache.D)
+    if max_sel is None:
+        max_sel = route_max_sel(top_k, n_hist, n_own)
+    if idx is None:
+        idx = torch.empty((cache.B, cache.Hh, n_own, max_sel), dtype=torch.int32, device=dev)
+    if cnt is None:
+        cnt = torch.empty((cache.B, cache.Hh, n_own), dtype=torch.int32, device=dev)
+    _need(idx, "idx", torch.int32, dev, (cache.B, cache.Hh, n_own, max_sel))
+    _need(cnt, "cnt", torch.int32, dev, (cache.B, cache.Hh, n_own))
+    if g is not None:
+        _need(g, "g", torch.float32, dev, (cache.B, n_own, n_hist))
+    ws_bytes = bsa_route_workspace_size(cache.B, cache.Hh, cache.D, n_own, n_hist)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    cs = cache.c_struct()
+    _check("bsa_route_qmean", _lib.bsa_route_qmean(
+        _ptr(q_mean), ctypes.byref(cs), int(n_hist), int(own_first), int(n_own), _ptr(g),
+        float(lam), float(g_ref), float(sm_scale), int(top_k), _ptr(idx), _ptr(cnt),
         int(max_sel), _ptr(workspace), workspace.numel(), _ptr(error_word(dev)), _stream(dev)))
     return idx, cnt
 
@@ -484,6 +552,45 @@ def bsa_attn(q_blk: torch.Tensor, cache: KVCache, idx: torch.Tensor, cnt: torch.
     _check("bsa_attn", _lib.bsa_attn(
         _ptr(q_blk), ctypes.byref(cs), _ptr(q_valid), _ptr(idx), _ptr(cnt), int(nqb),
         int(max_sel), float(sm_scale), _ptr(o), _ptr(lse), _ptr(error_word(dev)), _stream(dev)))
+    return o, lse
+
+
+def bsa_attn_tokens(q_blk: torch.Tensor, cache: KVCache, idx: torch.Tensor, cnt: torch.Tensor,
+                    T: int, H: int, W: int, q_valid: Optional[torch.Tensor] = None,
+                    sm_scale: Optional[float] = None, o: Optional[torch.Tensor] = None,
+                    lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """bsa_attn writing O and LSE in raster token order; returns
+    (O bf16 [B, T*H*W, Hh, D], LSE fp32 [B, T*H*W, Hh])."""
+    dev = cache.device
+    if q_blk.dim() != 4:
+        raise ValueError("q_blk must be [B, Hh, nQB*128, D]")
+    B, Hh, R, D = q_blk.shape
+    nqb = n_blocks_for(T, H, W)
+    if (B, Hh, D) != (cache.B, cache.Hh, cache.D) or R != nqb * BLK:
+        raise ValueError("q_blk does not match the cache and the chunk shape")
+    _need(q_blk, "q_blk", torch.bfloat16, dev)
+    if idx.dim() != 4 or tuple(idx.shape[:3]) != (B, Hh, nqb):
+        raise ValueError("idx must be [B, Hh, nQB, max_sel]")
+    max_sel = idx.shape[3]
+    _need(idx, "idx", torch.int32, dev)
+    _need(cnt, "cnt", torch.int32, dev, (B, Hh, nqb))
+    if q_valid is not None:
+        _need(q_valid, "q_valid", torch.int32, dev, (nqb,))
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    N = T * H * W
+    if o is None:
+        o = torch.empty((B, N, Hh, D), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((B, N, Hh), dtype=torch.float32, device=dev)
+    _need(o, "o", torch.bfloat16, dev, (B, N, Hh, D))
+    _need(lse, "lse", torch.float32, dev, (B, N, Hh))
+    perm = gilbert_perm_device(T, H, W, dev)
+    cs = cache.c_struct()
+    _check("bsa_attn_tokens", _lib.bsa_attn_tokens(
+        _ptr(q_blk), ctypes.byref(cs), _ptr(q_valid), _ptr(idx), _ptr(cnt), int(max_sel),
+        float(sm_scale), int(T), int(H), int(W), _ptr(perm), _ptr(o), _ptr(lse),
+        _ptr(error_word(dev)), _stream(dev)))
     return o, lse
 
 

@@ -73,6 +73,9 @@ constexpr uint32_t kColO = 384;
 constexpr long long kWaitLimit = 1LL << 31;  // SM clocks (about a second)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
+// Token-order output: the row -> token table is built by one warp scanning
+// the permutation while the tiles run, which stays hidden up to this size.
+constexpr int kTokOutMaxTokens = 1 << 14;
 
 // mbarrier slots
 enum {
@@ -98,7 +101,8 @@ struct AttnLayout {
   static constexpr int kBars = kV + kVSlots * kTileBytes;
   static constexpr int kMisc = kBars + B_COUNT * 8;
   static constexpr int kTok = (kMisc + 64 + 15) & ~15;  // float [2 warpgroups][128 rows]
-  static constexpr int kTotal = kTok + 2 * kBlk * 4;
+  static constexpr int kSlotTok = kTok + 2 * kBlk * 4;  // int [128]: raster token of each row
+  static constexpr int kTotal = kSlotTok + kBlk * 4;
   static constexpr int kAlloc = kTotal + 1024;          // room to align to 1024
   // The epilogue's [2][2][128] floats reuse K slot 0: by then every Q K^T
   // has completed and no K copy is in flight.
@@ -115,6 +119,8 @@ struct AttnArgs {
   __nv_bfloat16* o;
   float* lse;
   int32_t* d_err;
+  const int32_t* perm;      // token -> curve slot (token-order output only)
+  int n_tok;                // tokens of the chunk (token-order output only)
   int Hh, n_q_blocks, max_sel, max_blocks, n_blocks;
   float scale_log2;
 };
@@ -147,6 +153,41 @@ __device__ __forceinline__ void named_bar_arrive(int id, int count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Exponentials of the first kPolyPairs column pairs of every 64 are computed
+// on the FMA pipe (ex2_poly2) instead of the MUFU, which is otherwise as busy
+// per tile as the tensor core: 128 x 128 exponentials per tile at 16 per SM
+// clock take as long as the tile's two 128x128x128 products.
+#ifndef BSA_ATTN_POLY_PAIRS
+#define BSA_ATTN_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = BSA_ATTN_POLY_PAIRS;
+
+// 2^x for a pair of arguments without the MUFU.  x = j + f with j = round(x)
+// (adding and subtracting 1.5 * 2^23 rounds to an integer, whose bits end up
+// in the low mantissa of the sum) and f in [-0.5, 0.5]; 2^f is a cubic
+// fitted for this kernel by Remez exchange to minimise the relative error on
+// [-0.5, 0.5] (at most 7.5e-5, far below the bf16 rounding of P); 2^j is
+// added to the exponent field: (bits(x + 1.5*2^23) << 23) == j << 23 modulo
+// 2^32.  x is clamped at -126 first, so masked keys (-inf) give about 1e-38.
+__device__ __forceinline__ void ex2_poly2(uint64_t x2, float& e0, float& e1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
+  const uint64_t jf = f2_add(t, f2_pack(-kMagic, -kMagic));
+  const uint64_t fr = f2_fma(jf, f2_pack(-1.f, -1.f), xc);
+  uint64_t p = f2_fma(fr, f2_pack(kC3, kC3), f2_pack(kC2, kC2));
+  p = f2_fma(p, fr, f2_pack(kC1, kC1));
+  p = f2_fma(p, fr, f2_pack(kC0, kC0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // Maximum of three floats in one instruction (sm_100).
 __device__ __forceinline__ float fmax3(float x, float y, float z) {
   float d;
@@ -154,7 +195,11 @@ __device__ __forceinline__ float fmax3(float x, float y, float z) {
   return d;
 }
 
-template <int D>
+// kTokOut: O and LSE go straight to raster token order ([B, N, Hh, D] and
+// [B, N, Hh]) through the chunk's permutation, instead of block order; the
+// otherwise idle warp 3 inverts the permutation for the CTA's 128 rows while
+// the tiles are computed.
+template <int D, bool kTokOut>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
@@ -189,6 +234,10 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  // Barriers and tensor memory are set up while the predecessor grid (the
+  // router) finishes; the route and Q are read only after it completed.
+  pdl_wait();
+  pdl_trigger();
   const int n = route_count(a, item);
 
   if (warp == 0) {
@@ -311,6 +360,44 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_commit(&bars[B_MMA_DONE + (warp - 1)]);
       mbar_wait_bounded(&bars[B_MMA_DONE + (warp - 1)], 0, nullptr, kWaitLimit);
     }
+  } else if (warp == 3) {
+    // ---------------- row -> raster token table (token-order output) ----------------
+    // s_tok[r] = the token whose curve slot is j*128 + r, or -1 (pad row):
+    // the lanes scan perm with 16 loads in flight each.  Released to the
+    // softmax warps through named barrier 10 (arrive; they sync before
+    // their stores).
+    if (kTokOut) {
+      int* s_tok = reinterpret_cast<int*>(sm + L::kSlotTok);
+      for (int i = lane; i < kBlk; i += 32) s_tok[i] = -1;
+      __syncwarp();
+      const int slot0 = j * kBlk;
+      constexpr int kScan = 16;
+      for (int base = 0; base < a.n_tok; base += kScan * 32) {
+        int pv[kScan];
+#pragma unroll
+        for (int k = 0; k < kScan; ++k) {
+          const int t = base + lane + k * 32;
+          pv[k] = t < a.n_tok ? __ldg(a.perm + t) : -1;
+        }
+#pragma unroll
+        for (int k = 0; k < kScan; ++k) {
+          const int t = base + lane + k * 32;
+          if (t >= a.n_tok) break;
+          if (pv[k] < 0 || pv[k] >= a.n_tok) {
+            report(a.d_err, BSA_DEV_BAD_PERM);
+            continue;
+          }
+          const unsigned d = static_cast<unsigned>(pv[k] - slot0);
+          if (d < static_cast<unsigned>(kBlk)) s_tok[d] = t;
+        }
+      }
+      __syncwarp();
+      // A slot of a token row that no token maps to: perm is no permutation.
+      const int rows = min(kBlk, a.n_tok - slot0);
+      for (int i = lane; i < rows; i += 32)
+        if (s_tok[i] < 0) report(a.d_err, BSA_DEV_BAD_PERM);
+      named_bar_arrive(10, kSoftmaxThreads + 32);
+    }
   } else if (warp >= 4) {
     // ---------------- softmax / epilogue (warps 4..11) ----------------
     // The reference maximum m_t of tile t is decided in tile order: the
@@ -413,10 +500,17 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[64 * q + 2 * c], s[64 * q + 2 * c + 1]), scale2, neg_m2), x0,
-                    x1);
-          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+          const uint64_t x2 =
+              f2_fma(f2_pack(s[64 * q + 2 * c], s[64 * q + 2 * c + 1]), scale2, neg_m2);
+          float e0, e1;
+          if (c < kPolyPairs) {
+            ex2_poly2(x2, e0, e1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            e0 = ex2_approx(x0);
+            e1 = ex2_approx(x1);
+          }
           acc2[c & 1] = f2_add(acc2[c & 1], f2_pack(e0, e1));
           pk[c] = pack_bf16x2(e0, e1);
         }
@@ -480,7 +574,6 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // normalises D/2 output columns; warpgroup 0 writes the LSE.
     const int q_valid = a.q_valid != nullptr ? a.q_valid[j] : kBlk;
     const long long grow_idx = item * kBlk + r;
-    __nv_bfloat16* orow = a.o + grow_idx * D + g * (D / 2);
     // The last P V (tile n - 1) is awaited by the warpgroup that did not
     // process tile n - 1: in its loop it waited for every earlier completion
     // of that barrier, so the parity is exact.  The named barrier then
@@ -510,6 +603,18 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       l_tot = fin[2 * kBlk + r] * ex2_approx(m0 - m_fin) + fin[3 * kBlk + r] * ex2_approx(m1 - m_fin);
     }
     const float inv_l = have ? 1.0f / l_tot : 0.f;
+    // Destination of this row: block order, or the raster token of the row
+    // (a pad row has none and writes nothing).
+    long long out_row = grow_idx;  // in units of D (O) and of 1 (LSE)
+    bool write_row = true;
+    if (kTokOut) {
+      named_bar_sync(10, kSoftmaxThreads + 32);
+      const int tok = reinterpret_cast<const int*>(sm + L::kSlotTok)[r];
+      const long long b = bh / a.Hh, h = bh % a.Hh;
+      out_row = (b * a.n_tok + tok) * a.Hh + h;
+      write_row = tok >= 0;
+    }
+    __nv_bfloat16* orow = a.o + out_row * D + g * (D / 2);
 #pragma unroll
     for (int c = 0; c < D / 64; ++c) {
       float o[32];
@@ -523,11 +628,11 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         v.y = pack_bf16x2(have ? o[e + 2] * inv_l : 0.f, have ? o[e + 3] * inv_l : 0.f);
         v.z = pack_bf16x2(have ? o[e + 4] * inv_l : 0.f, have ? o[e + 5] * inv_l : 0.f);
         v.w = pack_bf16x2(have ? o[e + 6] * inv_l : 0.f, have ? o[e + 7] * inv_l : 0.f);
-        *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
+        if (write_row) *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
       }
     }
-    if (g == 0)
-      a.lse[grow_idx] = have ? (m_fin + __log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
+    if (g == 0 && write_row)
+      a.lse[out_row] = have ? (m_fin + __log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
   }
 
   tc_fence_before();
@@ -577,7 +682,7 @@ static bool device_is_sm100() {
   return major == 10;
 }
 
-template <int D>
+template <int D, bool kTokOut>
 static bsa_status launch_attn(const void* q, const bsa_kv_cache* c, const AttnArgs& a,
                               long long items, cudaStream_t s) {
   CUtensorMap tq, tk, tv;
@@ -586,29 +691,33 @@ static bsa_status launch_attn(const void* q, const bsa_kv_cache* c, const AttnAr
       !make_map(&tv, c->v, crows, D))
     return BSA_ERR_CUDA;
   const int smem = AttnLayout<D>::kAlloc;
-  if (cudaFuncSetAttribute(bsa_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(bsa_attn_kernel<D, kTokOut>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BSA_ERR_CUDA;
-  bsa_attn_kernel<D><<<static_cast<unsigned>(items), kAttnThreads, smem, s>>>(tq, tk, tv, a);
-  return launch_status();
+  return launch_pdl(bsa_attn_kernel<D, kTokOut>, dim3(static_cast<unsigned>(items)),
+                    dim3(kAttnThreads), static_cast<size_t>(smem), s, tq, tk, tv, a);
 }
 
 }  // namespace bsa
 
 using namespace bsa;
 
-extern "C" bsa_status bsa_attn(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
-                               const int32_t* idx, const int32_t* cnt, int n_q_blocks, int max_sel,
-                               float sm_scale, void* o_blk, float* lse, int32_t* d_err,
-                               void* stream) {
-  if (q_blk == nullptr || c == nullptr || idx == nullptr || cnt == nullptr || o_blk == nullptr ||
+namespace bsa {
+
+// bsa_attn and bsa_attn_tokens: argument checks, then one launch.  perm is
+// NULL for block-order output.
+static bsa_status attn_call(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
+                            const int32_t* idx, const int32_t* cnt, int n_q_blocks, int max_sel,
+                            float sm_scale, const int32_t* perm, int n_tok, void* o, float* lse,
+                            int32_t* d_err, void* stream) {
+  if (q_blk == nullptr || c == nullptr || idx == nullptr || cnt == nullptr || o == nullptr ||
       lse == nullptr || c->k == nullptr || c->v == nullptr || c->block_valid == nullptr)
     return BSA_ERR_INVALID_ARG;
   if (c->B <= 0 || c->Hh <= 0 || n_q_blocks <= 0 || max_sel <= 0 || c->max_blocks <= 0 ||
       c->n_blocks < 0 || c->n_blocks > c->max_blocks || !(sm_scale == sm_scale))
     return BSA_ERR_INVALID_ARG;
   if (c->D != 64 && c->D != 128) return BSA_ERR_UNSUPPORTED;
-  if (!aligned16(q_blk) || !aligned16(o_blk) || !aligned16(c->k) || !aligned16(c->v))
+  if (!aligned16(q_blk) || !aligned16(o) || !aligned16(c->k) || !aligned16(c->v))
     return BSA_ERR_INVALID_ARG;
   const long long items = static_cast<long long>(c->B) * c->Hh * n_q_blocks;
   const long long crows = static_cast<long long>(c->B) * c->Hh * c->max_blocks * kBlk;
@@ -619,9 +728,11 @@ extern "C" bsa_status bsa_attn(const void* q_blk, const bsa_kv_cache* c, const i
   a.cnt = cnt;
   a.block_valid = c->block_valid;
   a.q_valid = q_valid;
-  a.o = static_cast<__nv_bfloat16*>(o_blk);
+  a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.d_err = d_err;
+  a.perm = perm;
+  a.n_tok = n_tok;
   a.Hh = c->Hh;
   a.n_q_blocks = n_q_blocks;
   a.max_sel = max_sel;
@@ -629,6 +740,32 @@ extern "C" bsa_status bsa_attn(const void* q_blk, const bsa_kv_cache* c, const i
   a.n_blocks = c->n_blocks;
   a.scale_log2 = sm_scale * kLog2e;
   cudaStream_t s = as_stream(stream);
-  return c->D == 128 ? launch_attn<128>(q_blk, c, a, items, s)
-                     : launch_attn<64>(q_blk, c, a, items, s);
+  if (perm != nullptr)
+    return c->D == 128 ? launch_attn<128, true>(q_blk, c, a, items, s)
+                       : launch_attn<64, true>(q_blk, c, a, items, s);
+  return c->D == 128 ? launch_attn<128, false>(q_blk, c, a, items, s)
+                     : launch_attn<64, false>(q_blk, c, a, items, s);
+}
+
+}  // namespace bsa
+
+extern "C" bsa_status bsa_attn(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
+                               const int32_t* idx, const int32_t* cnt, int n_q_blocks, int max_sel,
+                               float sm_scale, void* o_blk, float* lse, int32_t* d_err,
+                               void* stream) {
+  return attn_call(q_blk, c, q_valid, idx, cnt, n_q_blocks, max_sel, sm_scale, nullptr, 0, o_blk,
+                   lse, d_err, stream);
+}
+
+extern "C" bsa_status bsa_attn_tokens(const void* q_blk, const bsa_kv_cache* c,
+                                      const int32_t* q_valid, const int32_t* idx,
+                                      const int32_t* cnt, int max_sel, float sm_scale, int T,
+                                      int H, int W, const int32_t* d_perm, void* o_tok,
+                                      float* lse_tok, int32_t* d_err, void* stream) {
+  if (d_perm == nullptr || T <= 0 || H <= 0 || W <= 0) return BSA_ERR_INVALID_ARG;
+  const long long n = static_cast<long long>(T) * H * W;
+  if (n > kTokOutMaxTokens) return BSA_ERR_UNSUPPORTED;
+  const int nb = static_cast<int>((n + kBlk - 1) / kBlk);
+  return attn_call(q_blk, c, q_valid, idx, cnt, nb, max_sel, sm_scale, d_perm,
+                   static_cast<int>(n), o_tok, lse_tok, d_err, stream);
 }

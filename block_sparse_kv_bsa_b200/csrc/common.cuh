@@ -32,6 +32,44 @@ inline bsa_status launch_status() {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Programmatic dependent launch.  A kernel launched by launch_pdl may begin
+// (be scheduled, set up shared memory and barriers) while the kernel before
+// it on the stream is still finishing; it reaches global memory only after
+// pdl_wait(), which returns once that predecessor grid has completed and its
+// writes are visible.  Every kernel launched this way therefore calls
+// pdl_wait() before its first global-memory access, which also keeps the
+// ordering transitive along the stream.  pdl_trigger() lets the successor
+// start launching (it is scheduled once every CTA of this grid has started
+// and triggered, so it never takes an SM from a CTA of this grid that has
+// not yet started).  Both are no-ops for a kernel launched the ordinary way.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Returns from the calling function with the status of `expr` unless BSA_OK.
+#define BSA_TRY(expr)                  \
+  do {                                 \
+    const bsa_status st_ = (expr);     \
+    if (st_ != BSA_OK) return st_;     \
+  } while (0)
+
+template <typename... KArgs, typename... Args>
+inline bsa_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // 16-byte global memory accesses
 // ---------------------------------------------------------------------------

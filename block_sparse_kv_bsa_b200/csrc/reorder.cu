@@ -44,6 +44,8 @@ struct ReorderArgs {
 template <int VPR, bool kToBlocks>
 __global__ void __launch_bounds__(kReorderThreads)
 reorder_kernel(ReorderArgs a) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
   __shared__ int s_slot[kRowsPerCta];
   const int r0 = blockIdx.x * kRowsPerCta;
   const int h0 = blockIdx.y * kHeadsPerCta;
@@ -128,11 +130,9 @@ static bsa_status launch_reorder(const ReorderArgs& a, int D, cudaStream_t s) {
   dim3 grid((rows + kRowsPerCta - 1) / kRowsPerCta, (a.Hh + kHeadsPerCta - 1) / kHeadsPerCta,
             a.B);
   if (D == 128) {
-    reorder_kernel<16, kToBlocks><<<grid, kReorderThreads, 0, s>>>(a);
-  } else {
-    reorder_kernel<8, kToBlocks><<<grid, kReorderThreads, 0, s>>>(a);
+    return launch_pdl(reorder_kernel<16, kToBlocks>, grid, dim3(kReorderThreads), 0, s, a);
   }
-  return launch_status();
+  return launch_pdl(reorder_kernel<8, kToBlocks>, grid, dim3(kReorderThreads), 0, s, a);
 }
 
 // Pooled-key cache: one warp per (b, h, block) writes the fp32 mean of the
@@ -178,6 +178,41 @@ static bsa_status launch_block_means(const bsa_kv_cache* c, int first, int count
   return launch_status();
 }
 
+// Slot -> token for the 128 curve slots [slot0, slot0 + 128) of one block:
+// s_tok[d] is the raster token whose perm entry is slot0 + d, or -1.  The
+// CTA's NT threads (NT >= 128) scan perm in rounds of kScan independent loads
+// per thread (one L2 round trip per round); entries outside [0, N) are
+// skipped, and reported when `report_bad`.  Ends with a CTA barrier.
+template <int NT>
+__device__ __forceinline__ void invert_block_slots(const int32_t* perm, int N, int slot0,
+                                                   int* s_tok, bool report_bad, int32_t* d_err) {
+  static_assert(NT >= kBlk, "one thread per slot clears the table");
+  if (threadIdx.x < kBlk) s_tok[threadIdx.x] = -1;
+  __syncthreads();
+  constexpr int kScan = 16;
+  for (int base = 0; base < N; base += kScan * NT) {
+    int pv[kScan];
+#pragma unroll
+    for (int k = 0; k < kScan; ++k) {
+      const int r = base + threadIdx.x + k * NT;
+      pv[k] = r < N ? __ldg(perm + r) : 0;
+    }
+#pragma unroll
+    for (int k = 0; k < kScan; ++k) {
+      const int r = base + threadIdx.x + k * NT;
+      if (r >= N) break;
+      const int p = pv[k];
+      if (p < 0 || p >= N) {
+        if (report_bad) report(d_err, BSA_DEV_BAD_PERM);
+        continue;
+      }
+      const unsigned d = static_cast<unsigned>(p - slot0);
+      if (d < static_cast<unsigned>(kBlk)) s_tok[d] = r;
+    }
+  }
+  __syncthreads();
+}
+
 // Fused append for chunks of up to kGatherMaxTokens tokens: one CTA per
 // (chunk block, group of kAppendHeads heads, batch) gathers the block's 128
 // curve slots from the token-major K and V and writes whole cache rows; each
@@ -204,6 +239,8 @@ struct AppendArgs {
 template <int VPR>
 __global__ void __launch_bounds__(kAppendThreads)
 append_gather_kernel(AppendArgs a) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
   constexpr int D = VPR * 8;
   __shared__ int s_tok[kBlk];
   const int j = blockIdx.x;
@@ -211,32 +248,7 @@ append_gather_kernel(AppendArgs a) {
   const int slot0 = j * kBlk;
   const int valid = min(kBlk, a.N - slot0);
   const bool first_cta = blockIdx.y == 0 && b == 0;
-  if (threadIdx.x < kBlk) s_tok[threadIdx.x] = -1;
-  __syncthreads();
-  // Slot -> token for this block's slots, scanning perm in rounds of
-  // kScan independent loads per thread (one L2 round trip per round).
-  constexpr int kScan = 16;
-  for (int base = 0; base < a.N; base += kScan * kAppendThreads) {
-    int pv[kScan];
-#pragma unroll
-    for (int k = 0; k < kScan; ++k) {
-      const int r = base + threadIdx.x + k * kAppendThreads;
-      pv[k] = r < a.N ? __ldg(a.perm + r) : 0;
-    }
-#pragma unroll
-    for (int k = 0; k < kScan; ++k) {
-      const int r = base + threadIdx.x + k * kAppendThreads;
-      if (r >= a.N) break;
-      const int p = pv[k];
-      if (p < 0 || p >= a.N) {
-        if (j == 0 && first_cta) report(a.d_err, BSA_DEV_BAD_PERM);
-        continue;
-      }
-      const unsigned d = static_cast<unsigned>(p - slot0);
-      if (d < static_cast<unsigned>(kBlk)) s_tok[d] = r;
-    }
-  }
-  __syncthreads();
+  invert_block_slots<kAppendThreads>(a.perm, a.N, slot0, s_tok, j == 0 && first_cta, a.d_err);
   if (first_cta && threadIdx.x == 0) a.block_valid[a.base_block + j] = valid;
   // A slot of the chunk that no token maps to: perm is not a permutation.
   if (first_cta && threadIdx.x < valid && s_tok[threadIdx.x] < 0) report(a.d_err, BSA_DEV_BAD_PERM);
@@ -272,11 +284,66 @@ append_gather_kernel(AppendArgs a) {
 
 static bsa_status launch_append_gather(const AppendArgs& a, int B, int D, int nb, cudaStream_t s) {
   dim3 grid(nb, (a.Hh + kAppendHeads - 1) / kAppendHeads, B);
-  if (D == 128)
-    append_gather_kernel<16><<<grid, kAppendThreads, 0, s>>>(a);
-  else
-    append_gather_kernel<8><<<grid, kAppendThreads, 0, s>>>(a);
-  return launch_status();
+  if (D == 128) return launch_pdl(append_gather_kernel<16>, grid, dim3(kAppendThreads), 0, s, a);
+  return launch_pdl(append_gather_kernel<8>, grid, dim3(kAppendThreads), 0, s, a);
+}
+
+// One tensor (the query chunk) into blocks together with the fp32 mean of
+// each block's valid rows: one CTA per (chunk block, kMeanHeads heads,
+// batch); warp w moves head w of the group, writing whole block rows (pads as
+// zeros), and pools the rows while it moves them with pool.cuh's summation,
+// the one every block mean of the library uses, so the router can score from
+// these means without reading the blocks again.
+constexpr int kMeanHeads = 4;
+constexpr int kMeanGatherThreads = kMeanHeads * 32;
+
+struct GatherMeanArgs {
+  const uint4* x_tok;
+  uint4* x_blk;
+  float* x_mean;
+  const int32_t* perm;
+  int32_t* d_err;
+  int N, Hh, nb;
+};
+
+template <int VPR>
+__global__ void __launch_bounds__(kMeanGatherThreads)
+gather_mean_kernel(GatherMeanArgs a) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
+  constexpr int D = VPR * 8;
+  __shared__ int s_tok[kBlk];
+  const int j = blockIdx.x;
+  const int b = blockIdx.z;
+  const int slot0 = j * kBlk;
+  const int valid = min(kBlk, a.N - slot0);
+  const bool first_cta = blockIdx.y == 0 && b == 0;
+  invert_block_slots<kMeanGatherThreads>(a.perm, a.N, slot0, s_tok, j == 0 && first_cta,
+                                         a.d_err);
+  if (first_cta && threadIdx.x < valid && s_tok[threadIdx.x] < 0) report(a.d_err, BSA_DEV_BAD_PERM);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int h = blockIdx.y * kMeanHeads + warp;
+  if (h >= a.Hh) return;
+  const int c = lane % VPR, g = lane / VPR;
+  const long long tok_stride = static_cast<long long>(a.Hh) * VPR;  // vectors per token
+  const long long tok_base = static_cast<long long>(b) * a.N * tok_stride +
+                             static_cast<long long>(h) * VPR + c;
+  const long long blk = (static_cast<long long>(b) * a.Hh + h) * a.nb + j;
+  uint4* dst = a.x_blk + blk * kBlk * VPR + c;
+  auto load = [&](int row) {
+    const int tok = s_tok[row];
+    return tok >= 0 ? ld_nc_v4(a.x_tok + tok_base + static_cast<long long>(tok) * tok_stride)
+                    : make_uint4(0, 0, 0, 0);
+  };
+  auto store = [&](int row, uint4 x) { st_v4(dst + row * VPR, x); };
+  float acc[8];
+  warp_colsum_rows<VPR>(load, store, valid, g, acc);
+  if (g == 0) {
+    float4* out = reinterpret_cast<float4*>(a.x_mean + blk * D + c * 8);
+    const float inv = static_cast<float>(valid);
+    out[0] = make_float4(acc[0] / inv, acc[1] / inv, acc[2] / inv, acc[3] / inv);
+    out[1] = make_float4(acc[4] / inv, acc[5] / inv, acc[6] / inv, acc[7] / inv);
+  }
 }
 
 static bsa_status check_chunk(int B, int Hh, int D, int T, int H, int W) {
@@ -407,6 +474,32 @@ extern "C" bsa_status bsa_tokens_to_blocks(const void* x_tok, void* x_blk, int B
   a.blk_stride = a.nb;
   a.base_block = 0;
   return launch_reorder<true>(a, D, as_stream(stream));
+}
+
+extern "C" bsa_status bsa_tokens_to_blocks_mean(const void* x_tok, void* x_blk, float* x_mean,
+                                                int B, int Hh, int D, int T, int H, int W,
+                                                const int32_t* d_perm, int32_t* d_err,
+                                                void* stream) {
+  if (x_tok == nullptr || x_blk == nullptr || x_mean == nullptr || d_perm == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  bsa_status st = check_chunk(B, Hh, D, T, H, W);
+  if (st != BSA_OK) return st;
+  if (!aligned16(x_tok) || !aligned16(x_blk) || !aligned16(x_mean)) return BSA_ERR_INVALID_ARG;
+  const int n = T * H * W;
+  if (n > kGatherMaxTokens) return BSA_ERR_UNSUPPORTED;
+  GatherMeanArgs a{};
+  a.x_tok = static_cast<const uint4*>(x_tok);
+  a.x_blk = static_cast<uint4*>(x_blk);
+  a.x_mean = x_mean;
+  a.perm = d_perm;
+  a.d_err = d_err;
+  a.N = n;
+  a.Hh = Hh;
+  a.nb = (n + kBlk - 1) / kBlk;
+  dim3 grid(a.nb, (Hh + kMeanHeads - 1) / kMeanHeads, B);
+  cudaStream_t s = as_stream(stream);
+  if (D == 128) return launch_pdl(gather_mean_kernel<16>, grid, dim3(kMeanGatherThreads), 0, s, a);
+  return launch_pdl(gather_mean_kernel<8>, grid, dim3(kMeanGatherThreads), 0, s, a);
 }
 
 extern "C" bsa_status bsa_blocks_to_tokens(const void* x_blk, void* x_tok, int B, int Hh, int D,

@@ -29,7 +29,6 @@
 
 namespace bsa {
 
-constexpr int kPoolThreads = 256;
 constexpr int kTopkThreads = 256;
 
 struct RouteArgs {
@@ -56,78 +55,31 @@ __device__ __forceinline__ int clamp_valid(int v, int32_t* d_err) {
   return v;
 }
 
-// One 128 x D bf16 block is read as VPR 16-byte vectors per row: thread t
-// owns vector column t % VPR and rows t / VPR + RG*i (RG = 256 / VPR).
-template <int VPR>
-struct BlockRegs {
-  static constexpr int RG = kPoolThreads / VPR;
-  static constexpr int RPT = kBlk / RG;
-  uint4 x[RPT];
-};
-
-// Issue the loads of the first `valid` rows of a block (rows past it read 0).
-template <int VPR>
-__device__ __forceinline__ void block_load(const uint4* blk, int valid, BlockRegs<VPR>& r) {
-  const int vc = threadIdx.x % VPR;
-  const int rg = threadIdx.x / VPR;
-#pragma unroll
-  for (int i = 0; i < BlockRegs<VPR>::RPT; ++i) {
-    int row = rg + BlockRegs<VPR>::RG * i;
-    r.x[i] = row < valid ? ld_nc_v4(blk + row * VPR + vc) : make_uint4(0, 0, 0, 0);
-  }
-}
-
-// Column sums of this thread's rows -> red [RG][D]; the caller reduces.
-template <int VPR>
-__device__ __forceinline__ void block_colsum_store(const BlockRegs<VPR>& r, float* red) {
-  const int vc = threadIdx.x % VPR;
-  const int rg = threadIdx.x / VPR;
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-  for (int i = 0; i < BlockRegs<VPR>::RPT; ++i) {
-    acc[0] += bf16lo(r.x[i].x); acc[1] += bf16hi(r.x[i].x);
-    acc[2] += bf16lo(r.x[i].y); acc[3] += bf16hi(r.x[i].y);
-    acc[4] += bf16lo(r.x[i].z); acc[5] += bf16hi(r.x[i].z);
-    acc[6] += bf16lo(r.x[i].w); acc[7] += bf16hi(r.x[i].w);
-  }
-#pragma unroll
-  for (int e = 0; e < 8; ++e) red[rg * (VPR * 8) + vc * 8 + e] = acc[e];
-}
+// Query-block means: one warp per (b, h, query block), with pool.cuh's
+// summation, the same as bsa_tokens_to_blocks_mean's and the pooled-key
+// cache's, so every block mean in the library comes from one summation.
+constexpr int kPoolQWarps = 8;
 
 template <int VPR>
-__device__ __forceinline__ void block_colsum_partial(const uint4* blk, int valid, float* red) {
-  BlockRegs<VPR> r;
-  block_load<VPR>(blk, valid, r);
-  block_colsum_store<VPR>(r, red);
-}
-
-// Finish the mean: out[d] = sum_rg red[rg][d] / valid (threads d < D).
-template <int VPR>
-__device__ __forceinline__ void block_mean_finish(const float* red, int valid, float* out) {
+__global__ void __launch_bounds__(kPoolQWarps * 32) pool_q_kernel(RouteArgs a) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
   constexpr int D = VPR * 8;
-  constexpr int RG = kPoolThreads / VPR;
-  if (threadIdx.x < D) {
-    float t = 0.f;
-#pragma unroll 4
-    for (int rg = 0; rg < RG; ++rg) t += red[rg * D + threadIdx.x];
-    out[threadIdx.x] = t / static_cast<float>(valid);
-  }
-}
-
-template <int VPR>
-__global__ void __launch_bounds__(kPoolThreads) pool_q_kernel(RouteArgs a) {
-  constexpr int D = VPR * 8;
-  __shared__ float red[kPoolThreads / VPR * D];
-  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int j = blockIdx.x * kPoolQWarps + warp;
+  if (j >= a.n_own) return;
+  const int h = blockIdx.y, b = blockIdx.z;
   int valid = a.q_valid != nullptr ? a.q_valid[j] : a.block_valid[a.own_first + j];
   valid = clamp_valid(valid, a.d_err);
-  const long long bh = static_cast<long long>(b) * a.Hh + h;
-  const uint4* blk = a.q + (bh * a.n_own + j) * kBlk * VPR;
-  block_colsum_partial<VPR>(blk, valid, red);
-  __syncthreads();
-  block_mean_finish<VPR>(red, valid, a.qm + (bh * a.n_own + j) * D);
+  const long long blk = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
+  const int c = lane % VPR, g = lane / VPR;
+  float m[8];
+  warp_block_mean<VPR>(a.q + blk * kBlk * VPR, valid, c, g, m);
+  if (g == 0) {
+    float4* out = reinterpret_cast<float4*>(a.qm + blk * D + c * 8);
+    out[0] = make_float4(m[0], m[1], m[2], m[3]);
+    out[1] = make_float4(m[4], m[5], m[6], m[7]);
+  }
 }
 
 // K-stream kernel: one warp reduces one history block at a time.  A CTA of
@@ -145,6 +97,8 @@ constexpr int kScoreBlocksPerWarp = 8;
 template <int VPR>
 __global__ void __launch_bounds__(kScoreWarps * 32)
 pool_score_kernel(RouteArgs a) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
   constexpr int D = VPR * 8;
   constexpr int LPR = VPR;              // lanes per row (one 16-byte chunk each)
   constexpr int RPI = 32 / LPR;         // rows per warp-wide load (2 or 4)
@@ -271,6 +225,8 @@ __device__ __forceinline__ void score_means_tile(const RouteArgs& a, const float
 template <int D>
 __global__ void __launch_bounds__(kMeanThreads, 1)
 score_means_kernel(RouteArgs a) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
   constexpr int P = D + 4;                       // padded row (floats)
   extern __shared__ float sm[];
   const int nq = (a.n_own + 15) & ~15;           // query rows, rounded up to 16
@@ -397,6 +353,8 @@ __device__ __forceinline__ void score_pipe_tile(const RouteArgs& a, const float*
 
 template <int D>
 __global__ void __launch_bounds__(kPipeThreads, 1) score_means_pipe_kernel(RouteArgs a) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
   constexpr int P = D + 4;
   constexpr int R4 = D / 4;                      // 16-byte pieces per row
   extern __shared__ __align__(16) float sm[];
@@ -507,6 +465,8 @@ __device__ __forceinline__ float fused_score(const RouteArgs& a, const float* sr
 }
 
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(RouteArgs a) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
   extern __shared__ uint32_t keys[];   // [n_hist] when staged
   __shared__ int hist[256];
   __shared__ int warp_tot[kTopkThreads / 32];
@@ -680,6 +640,8 @@ constexpr int kTopkRowThreads = 128;
 
 template <int KPL>
 __global__ void __launch_bounds__(kTopkRowThreads, KPL <= 18 ? 8 : 6) topk_row_kernel(RouteArgs a) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
   constexpr int kWarps = kTopkRowThreads / 32;
   __shared__ unsigned part[2][kWarps];
   __shared__ unsigned grp[2][KPL][kWarps];     // per-(group, warp) ballot counts: eq, sel
@@ -840,6 +802,8 @@ __device__ __forceinline__ float block_tree(float* red, Op op) {
 constexpr int kVeloxRankMax = 256;   // budgets up to this are ranked by counting
 
 __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a, VeloxArgs v) {
+  pdl_wait();     // global memory only after the predecessor grid completed
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t vsm[];
   const int nh = a.n_hist;
   uint64_t* sortbuf = reinterpret_cast<uint64_t*>(vsm);                 // [kVeloxSortMax]
@@ -1064,14 +1028,18 @@ namespace bsa {
 // Validation shared by both routes, the query means and the model scores
 // (from the pooled-key cache or by streaming the history keys).  Fills `a`
 // for the selection kernel the caller launches next.
-static bsa_status route_scores(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
-                               int n_hist, int own_first, int n_own, const float* g,
-                               float lambda, float g_ref, float sm_scale, int32_t* idx,
-                               int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
-                               int32_t* d_err, cudaStream_t s, RouteArgs* out) {
-  if (q_blk == nullptr || c == nullptr || idx == nullptr || cnt == nullptr ||
-      workspace == nullptr || c->k == nullptr || c->block_valid == nullptr)
+// The query means come from q_blk (pooled here, by pool_q_kernel) or, when
+// q_mean is given, from the caller (q_blk is then not read).
+static bsa_status route_scores(const void* q_blk, const float* q_mean, const bsa_kv_cache* c,
+                               const int32_t* q_valid, int n_hist, int own_first, int n_own,
+                               const float* g, float lambda, float g_ref, float sm_scale,
+                               int32_t* idx, int32_t* cnt, int max_sel, void* workspace,
+                               size_t ws_bytes, int32_t* d_err, cudaStream_t s, RouteArgs* out) {
+  if ((q_blk == nullptr && q_mean == nullptr) || c == nullptr || idx == nullptr ||
+      cnt == nullptr || workspace == nullptr || c->k == nullptr || c->block_valid == nullptr)
     return BSA_ERR_INVALID_ARG;
+  if (q_mean != nullptr && !aligned16(q_mean)) return BSA_ERR_INVALID_ARG;
+  if (q_mean != nullptr) q_blk = c->k;  // not read; keeps the alignment check below uniform
   if (c->B <= 0 || c->Hh <= 0 || n_own <= 0 || n_hist < 0 || max_sel <= 0)
     return BSA_ERR_INVALID_ARG;
   if (c->D != 64 && c->D != 128) return BSA_ERR_UNSUPPORTED;
@@ -1100,7 +1068,7 @@ static bsa_status route_scores(const void* q_blk, const bsa_kv_cache* c, const i
   a.q_valid = q_valid;
   a.g = g;
   a.kmean = c->kmean;
-  a.qm = static_cast<float*>(workspace);
+  a.qm = q_mean != nullptr ? const_cast<float*>(q_mean) : static_cast<float*>(workspace);
   a.s = reinterpret_cast<float*>(static_cast<char*>(workspace) + qm_b);
   a.idx = idx;
   a.cnt = cnt;
@@ -1116,7 +1084,7 @@ static bsa_status route_scores(const void* q_blk, const bsa_kv_cache* c, const i
   a.lam = lambda;
   a.g_ref = g_ref;
 
-  dim3 qgrid(n_own, c->Hh, c->B);
+  dim3 pgrid((n_own + kPoolQWarps - 1) / kPoolQWarps, c->Hh, c->B);
   const int per_cta = kScoreWarps * kScoreBlocksPerWarp;
   dim3 sgrid((n_hist + per_cta - 1) / per_cta, c->Hh, c->B);
   dim3 mgrid((n_hist + kMeanTileN - 1) / kMeanTileN, c->Hh, c->B);
@@ -1131,42 +1099,46 @@ static bsa_status route_scores(const void* q_blk, const bsa_kv_cache* c, const i
     pipe_grid = static_cast<int>(std::min<long long>(tiles, device_sms()));
   }
   if (c->D == 128) {
-    pool_q_kernel<16><<<qgrid, kPoolThreads, 0, s>>>(a);
+    if (q_mean == nullptr)
+      BSA_TRY(launch_pdl(pool_q_kernel<16>, pgrid, dim3(kPoolQWarps * 32), 0, s, a));
     if (n_hist > 0 && c->kmean != nullptr && pipe_grid > 0) {
       if (cudaFuncSetAttribute(score_means_pipe_kernel<128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(pipe_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      score_means_pipe_kernel<128><<<pipe_grid, kPipeThreads, pipe_smem, s>>>(a);
+      BSA_TRY(launch_pdl(score_means_pipe_kernel<128>, dim3(pipe_grid), dim3(kPipeThreads),
+                         pipe_smem, s, a));
     } else if (n_hist > 0 && c->kmean != nullptr) {
       if (cudaFuncSetAttribute(score_means_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(mean_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      score_means_kernel<128><<<mgrid, kMeanThreads, mean_smem, s>>>(a);
+      BSA_TRY(launch_pdl(score_means_kernel<128>, mgrid, dim3(kMeanThreads), mean_smem, s, a));
     } else if (n_hist > 0) {
       if (cudaFuncSetAttribute(pool_score_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(qm_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      pool_score_kernel<16><<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
+      BSA_TRY(launch_pdl(pool_score_kernel<16>, sgrid, dim3(kScoreWarps * 32), qm_smem, s, a));
     }
   } else {
-    pool_q_kernel<8><<<qgrid, kPoolThreads, 0, s>>>(a);
+    if (q_mean == nullptr)
+      BSA_TRY(launch_pdl(pool_q_kernel<8>, pgrid, dim3(kPoolQWarps * 32), 0, s, a));
     if (n_hist > 0 && c->kmean != nullptr && pipe_grid > 0) {
       if (cudaFuncSetAttribute(score_means_pipe_kernel<64>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(pipe_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      score_means_pipe_kernel<64><<<pipe_grid, kPipeThreads, pipe_smem, s>>>(a);
+      BSA_TRY(launch_pdl(score_means_pipe_kernel<64>, dim3(pipe_grid), dim3(kPipeThreads),
+                         pipe_smem, s, a));
     } else if (n_hist > 0 && c->kmean != nullptr) {
       if (cudaFuncSetAttribute(score_means_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(mean_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      score_means_kernel<64><<<mgrid, kMeanThreads, mean_smem, s>>>(a);
+      BSA_TRY(launch_pdl(score_means_kernel<64>, mgrid, dim3(kMeanThreads), mean_smem, s, a));
     } else if (n_hist > 0) {
       if (cudaFuncSetAttribute(pool_score_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(qm_smem)) != cudaSuccess)
         return BSA_ERR_CUDA;
-      pool_score_kernel<8><<<sgrid, kScoreWarps * 32, qm_smem, s>>>(a);
+      BSA_TRY(launch_pdl(pool_score_kernel<8>, sgrid, dim3(kScoreWarps * 32), qm_smem, s, a));
     }
   }
   return launch_status();
@@ -1176,18 +1148,23 @@ static bsa_status route_scores(const void* q_blk, const bsa_kv_cache* c, const i
 
 using namespace bsa;
 
-extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
-                                int n_hist, int own_first, int n_own, const float* g,
-                                float lambda, float g_ref, float sm_scale, int top_k, int32_t* idx,
-                                int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
-                                int32_t* d_err, void* stream) {
+namespace bsa {
+
+// bsa_route and bsa_route_qmean: scores (query means from q_blk or given),
+// then the top-K of every row.
+static bsa_status route_topk(const void* q_blk, const float* q_mean, const bsa_kv_cache* c,
+                             const int32_t* q_valid, int n_hist, int own_first, int n_own,
+                             const float* g, float lambda, float g_ref, float sm_scale, int top_k,
+                             int32_t* idx, int32_t* cnt, int max_sel, void* workspace,
+                             size_t ws_bytes, int32_t* d_err, void* stream) {
   if (top_k < 0) return BSA_ERR_INVALID_ARG;
   const int K = top_k < n_hist ? top_k : n_hist;
   if (n_hist >= 0 && n_own > 0 && max_sel > 0 && max_sel < K + n_own) return BSA_ERR_CAPACITY;
   cudaStream_t s = as_stream(stream);
   RouteArgs a;
-  bsa_status st = route_scores(q_blk, c, q_valid, n_hist, own_first, n_own, g, lambda, g_ref,
-                               sm_scale, idx, cnt, max_sel, workspace, ws_bytes, d_err, s, &a);
+  bsa_status st = route_scores(q_blk, q_mean, c, q_valid, n_hist, own_first, n_own, g, lambda,
+                               g_ref, sm_scale, idx, cnt, max_sel, workspace, ws_bytes, d_err, s,
+                               &a);
   if (st != BSA_OK) return st;
   a.top_k = top_k;
   // Rows of up to 3072 history blocks: keys in registers (their count per
@@ -1196,13 +1173,13 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   dim3 qgrid(n_own, c->Hh, c->B);
   if (n_hist <= kTopkRowThreads * 24) {
     if (n_hist <= kTopkRowThreads * 4)
-      topk_row_kernel<4><<<qgrid, kTopkRowThreads, 0, s>>>(a);
+      BSA_TRY(launch_pdl(topk_row_kernel<4>, qgrid, dim3(kTopkRowThreads), 0, s, a));
     else if (n_hist <= kTopkRowThreads * 10)
-      topk_row_kernel<10><<<qgrid, kTopkRowThreads, 0, s>>>(a);
+      BSA_TRY(launch_pdl(topk_row_kernel<10>, qgrid, dim3(kTopkRowThreads), 0, s, a));
     else if (n_hist <= kTopkRowThreads * 18)
-      topk_row_kernel<18><<<qgrid, kTopkRowThreads, 0, s>>>(a);
+      BSA_TRY(launch_pdl(topk_row_kernel<18>, qgrid, dim3(kTopkRowThreads), 0, s, a));
     else
-      topk_row_kernel<24><<<qgrid, kTopkRowThreads, 0, s>>>(a);
+      BSA_TRY(launch_pdl(topk_row_kernel<24>, qgrid, dim3(kTopkRowThreads), 0, s, a));
     return launch_status();
   }
   const size_t topk_smem =
@@ -1210,8 +1187,30 @@ extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const 
   if (cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(topk_smem)) != cudaSuccess)
     return BSA_ERR_CUDA;
-  topk_kernel<<<qgrid, kTopkThreads, topk_smem, s>>>(a);
+  BSA_TRY(launch_pdl(topk_kernel, qgrid, dim3(kTopkThreads), topk_smem, s, a));
   return launch_status();
+}
+
+}  // namespace bsa
+
+extern "C" bsa_status bsa_route(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
+                                int n_hist, int own_first, int n_own, const float* g,
+                                float lambda, float g_ref, float sm_scale, int top_k, int32_t* idx,
+                                int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
+                                int32_t* d_err, void* stream) {
+  if (q_blk == nullptr) return BSA_ERR_INVALID_ARG;
+  return route_topk(q_blk, nullptr, c, q_valid, n_hist, own_first, n_own, g, lambda, g_ref,
+                    sm_scale, top_k, idx, cnt, max_sel, workspace, ws_bytes, d_err, stream);
+}
+
+extern "C" bsa_status bsa_route_qmean(const float* q_mean, const bsa_kv_cache* c, int n_hist,
+                                      int own_first, int n_own, const float* g, float lambda,
+                                      float g_ref, float sm_scale, int top_k, int32_t* idx,
+                                      int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
+                                      int32_t* d_err, void* stream) {
+  if (q_mean == nullptr) return BSA_ERR_INVALID_ARG;
+  return route_topk(nullptr, q_mean, c, nullptr, n_hist, own_first, n_own, g, lambda, g_ref,
+                    sm_scale, top_k, idx, cnt, max_sel, workspace, ws_bytes, d_err, stream);
 }
 
 extern "C" bsa_status bsa_route_velox(const void* q_blk, const bsa_kv_cache* c,
@@ -1236,8 +1235,9 @@ extern "C" bsa_status bsa_route_velox(const void* q_blk, const bsa_kv_cache* c,
   if (max_sel < bound) return BSA_ERR_CAPACITY;
   cudaStream_t s = as_stream(stream);
   RouteArgs a;
-  bsa_status st = route_scores(q_blk, c, q_valid, n_hist, own_first, n_own, g, lambda, g_ref,
-                               sm_scale, idx, cnt, max_sel, workspace, ws_bytes, d_err, s, &a);
+  bsa_status st = route_scores(q_blk, nullptr, c, q_valid, n_hist, own_first, n_own, g, lambda,
+                               g_ref, sm_scale, idx, cnt, max_sel, workspace, ws_bytes, d_err, s,
+                               &a);
   if (st != BSA_OK) return st;
   VeloxArgs v{o.coverage, o.eta_cov, o.tau, o.mass, o.k_cov, o.k_unc, o.prev_first, o.n_prev,
               o.window_half, o.ref_first, o.n_ref};
@@ -1247,7 +1247,7 @@ extern "C" bsa_status bsa_route_velox(const void* q_blk, const bsa_kv_cache* c,
                            static_cast<int>(smem)) != cudaSuccess)
     return BSA_ERR_CUDA;
   dim3 qgrid(n_own, c->Hh, c->B);
-  velox_select_kernel<<<qgrid, kTopkThreads, smem, s>>>(a, v);
+  BSA_TRY(launch_pdl(velox_select_kernel, qgrid, dim3(kTopkThreads), smem, s, a, v));
   return launch_status();
 }
 

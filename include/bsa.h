@@ -155,6 +155,24 @@ bsa_status bsa_tokens_to_blocks(const void *x_tok, void *x_blk, int B, int Hh, i
                                 int T, int H, int W, const int32_t *d_perm,
                                 int32_t *d_err, void *stream);
 
+/*
+ * bsa_tokens_to_blocks that also pools (Velox, Methodology Step 4: the block
+ * importance uses the mean query of each block): besides x_blk it writes
+ *   x_mean  device fp32 [B, Hh, nb, D], 16-byte aligned: the mean of the
+ *           valid rows of every block (rows 0 .. min(128, T*H*W - 128*j) - 1
+ *           of block j), summed in fp32 in the same fixed order as every
+ *           other block mean of the library (bsa_route's own pooling, the
+ *           pooled-key cache), so bsa_route_qmean on these means selects
+ *           exactly what bsa_route on x_blk selects.
+ * One pass over the tokens: the route then needs no second read of the
+ * query blocks.  Chunks of up to 16384 tokens.
+ * Errors: those of bsa_tokens_to_blocks; BSA_ERR_UNSUPPORTED above 16384
+ *         tokens.
+ */
+bsa_status bsa_tokens_to_blocks_mean(const void *x_tok, void *x_blk, float *x_mean, int B,
+                                     int Hh, int D, int T, int H, int W,
+                                     const int32_t *d_perm, int32_t *d_err, void *stream);
+
 /* Inverse gather, e.g. the attention output back to raster tokens:
  *   x_blk [B, Hh, nb*128, D]  ->  x_tok [B, T*H*W, Hh, D]. */
 bsa_status bsa_blocks_to_tokens(const void *x_blk, void *x_tok, int B, int Hh, int D,
@@ -193,6 +211,19 @@ bsa_status bsa_route(const void *q_blk, const bsa_kv_cache *cache, const int32_t
                      void *workspace, size_t ws_bytes, int32_t *d_err, void *stream);
 
 /*
+ * bsa_route with the query-block means given instead of the query blocks
+ * (Velox, Methodology Steps 4-5), e.g. from bsa_tokens_to_blocks_mean:
+ *   q_mean  device fp32 [B, Hh, n_own, D], 16-byte aligned
+ * Everything else, the result and the errors are those of bsa_route (the
+ * workspace is sized by bsa_route_workspace_size as there).  With the means
+ * of bsa_tokens_to_blocks_mean the routes equal bsa_route's bit for bit.
+ */
+bsa_status bsa_route_qmean(const float *q_mean, const bsa_kv_cache *cache, int n_hist,
+                           int own_first, int n_own, const float *g, float lambda, float g_ref,
+                           float sm_scale, int top_k, int32_t *idx, int32_t *cnt, int max_sel,
+                           void *workspace, size_t ws_bytes, int32_t *d_err, void *stream);
+
+/*
  * Indexed block-sparse attention (Velox, Methodology Step 6).  For query row
  * r of block j of head (b, h), over the valid rows k of the blocks
  * idx[b,h,j,0:cnt[b,h,j]] (order irrelevant, no causal mask):
@@ -212,6 +243,26 @@ bsa_status bsa_route(const void *q_blk, const bsa_kv_cache *cache, const int32_t
 bsa_status bsa_attn(const void *q_blk, const bsa_kv_cache *cache, const int32_t *q_valid,
                     const int32_t *idx, const int32_t *cnt, int n_q_blocks, int max_sel,
                     float sm_scale, void *o_blk, float *lse, int32_t *d_err, void *stream);
+
+/*
+ * bsa_attn with O and LSE written straight to raster token order (Velox,
+ * Methodology Step 6, followed by the inverse of the query reordering):
+ * row r of query block j is the token t with d_perm[t] = 128*j + r, so
+ *   o_tok[b, t, h, :] = O of that row           device bf16 [B, T*H*W, Hh, D]
+ *   lse_tok[b, t, h]  = LSE of that row          device fp32 [B, T*H*W, Hh]
+ * and pad rows (slots no token maps to) are not written.  This saves the
+ * separate bsa_blocks_to_tokens pass over O.  The query chunk has
+ * ceil(T*H*W / 128) blocks; q_blk, q_valid, idx, cnt, max_sel and sm_scale
+ * are those of bsa_attn, and d_perm is the table the query was reordered
+ * with (bsa_tokens_to_blocks).  Chunks of up to 16384 tokens.
+ * Errors: those of bsa_attn; BSA_ERR_UNSUPPORTED above 16384 tokens; on the
+ *         device BSA_DEV_BAD_PERM for a d_perm that is not a permutation
+ *         (rows without a token are then not written).
+ */
+bsa_status bsa_attn_tokens(const void *q_blk, const bsa_kv_cache *cache, const int32_t *q_valid,
+                           const int32_t *idx, const int32_t *cnt, int max_sel, float sm_scale,
+                           int T, int H, int W, const int32_t *d_perm, void *o_tok,
+                           float *lse_tok, int32_t *d_err, void *stream);
 
 /*
  * Self-test of the bounded-wait failure path used by every pipeline wait in

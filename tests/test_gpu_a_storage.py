@@ -237,3 +237,42 @@ def test_append_large_chunk():
     assert np.array_equal(valid[:nb], oracle.block_valid_for(T, H, W))
     exp_m = oracle.pool_blocks(exp_k, oracle.block_valid_for(T, H, W))
     assert np.allclose(cache.kmean[:, :, :nb].cpu().double().numpy(), exp_m, rtol=2e-6, atol=2e-7)
+
+
+@pytest.mark.parametrize("key", [1, 3, 5])
+def test_tokens_to_blocks_mean(key):
+    # One pass that reorders the query chunk and pools its blocks (Velox,
+    # Methodology Step 4: block importance from the mean query).  The blocks
+    # must equal bsa_tokens_to_blocks bit for bit, the means the oracle's
+    # fp64 means of the valid rows (pads excluded).
+    w = synth.CONFIGS[key]
+    T, H, W = w.grid
+    t = synth.chunk_tokens(w, 1, device=DEV, want=("q",))
+    ref = bsa.bsa_tokens_to_blocks(t["q"], T, H, W)
+    blk, mean = bsa.bsa_tokens_to_blocks_mean(t["q"], T, H, W)
+    bsa.raise_on_device_error(DEV)
+    assert torch.equal(blk.view(torch.int16), ref.view(torch.int16))
+    heads = list(range(w.Hh)) if w.Hh <= 12 else [0, 17, w.Hh - 1]
+    exp_blk = oracle.tokens_to_blocks(t["q"][:, :, heads].cpu().double().numpy(), T, H, W)
+    exp = oracle.pool_blocks(exp_blk, oracle.block_valid_for(T, H, W))
+    assert np.allclose(mean[:, heads].cpu().double().numpy(), exp, rtol=2e-6, atol=2e-7)
+
+
+@pytest.mark.parametrize("key,chunk,pooled", [(1, None, False), (3, None, True),
+                                              (4, 12, True), (5, None, False)])
+def test_route_from_query_means_equals_route(key, chunk, pooled):
+    # bsa_route_qmean on the means of bsa_tokens_to_blocks_mean selects what
+    # bsa_route selects from the query blocks, bit for bit: every block mean
+    # of the library comes from one summation.
+    from tests import _harness as hx
+    w = synth.CONFIGS[key]
+    T, H, W = w.grid
+    step = hx.build_step(w, DEV, chunk=chunk, pooled_keys=pooled)
+    idx, cnt = hx.route(step)
+    _, qm = bsa.bsa_tokens_to_blocks_mean(step.q_tok, T, H, W)
+    idx2, cnt2 = bsa.bsa_route_qmean(qm, step.cache, step.n_hist, step.own_first, step.n_own,
+                                     step.top_k, g=step.g, lam=w.lam, g_ref=w.g_ref,
+                                     sm_scale=w.sm_scale)
+    bsa.raise_on_device_error(DEV)
+    assert torch.equal(cnt2, cnt)
+    assert torch.equal(idx2, idx)

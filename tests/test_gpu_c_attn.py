@@ -226,3 +226,51 @@ def test_attn_bad_index_reported_not_faulted():
     bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
     status, code = bsa.bsa_check_device_error(DEV)
     assert status == 6 and code == 2
+
+
+@pytest.mark.parametrize("key", [1, 3, 4])
+def test_attn_tokens_equals_attn_then_reorder(key):
+    # O and LSE written straight to raster token order: the same numbers as
+    # bsa_attn followed by bsa_blocks_to_tokens (same arithmetic, only the
+    # destination differs), and the pad rows of the tail block write nothing.
+    w = synth.CONFIGS[key]
+    T, H, W = w.grid
+    step = hx.build_step(w, DEV, chunk=6 if key == 4 else None)
+    idx, cnt = hx.route(step)
+    o_blk, lse_blk = bsa.bsa_attn(step.q_blk, step.cache, idx, cnt, q_valid=step.q_valid)
+    o_ref = bsa.bsa_blocks_to_tokens(o_blk, T, H, W)
+    N = T * H * W
+    o_tok = torch.full((w.B, N, w.Hh, w.D), 7.0, dtype=torch.bfloat16, device=DEV)
+    lse_tok = torch.full((w.B, N, w.Hh), 7.0, dtype=torch.float32, device=DEV)
+    bsa.bsa_attn_tokens(step.q_blk, step.cache, idx, cnt, T, H, W, q_valid=step.q_valid,
+                        o=o_tok, lse=lse_tok)
+    bsa.raise_on_device_error(DEV)
+    assert torch.equal(o_tok.view(torch.int16), o_ref.view(torch.int16))
+    perm = torch.from_numpy(bsa.bsa_gilbert_perm(T, H, W).astype(np.int64)).to(DEV)
+    lse_ref = lse_blk[:, :, perm].permute(0, 2, 1)            # [B, N, Hh]
+    assert torch.equal(lse_tok, lse_ref)
+
+
+def test_attn_tokens_against_the_oracle_config3():
+    # Parity of the token-order output itself: the oracle's O and LSE of two
+    # heads, gathered back to raster order by the oracle's own curve.
+    import oracle
+    w = synth.CONFIGS[3]
+    T, H, W = w.grid
+    step = hx.build_step(w, DEV)
+    heads = (2, 21)
+    idx, cnt, routes = hx.attn_routes(step, heads)
+    o_tok, lse_tok = bsa.bsa_attn_tokens(step.q_blk, step.cache, idx, cnt, T, H, W,
+                                         q_valid=step.q_valid)
+    bsa.raise_on_device_error(DEV)
+    items = [(0, h, j) for h in heads for j in range(step.n_own)]
+    refs = hx.oracle_attn_items(step, routes, items)
+    for hi, h in enumerate(heads):
+        ro = np.concatenate([refs[hi * step.n_own + j][0] for j in range(step.n_own)])
+        rl = np.concatenate([refs[hi * step.n_own + j][1] for j in range(step.n_own)])
+        ro_tok = oracle.blocks_to_tokens(ro[None, None], T, H, W)[0, :, 0]       # [N, D]
+        rl_tok = oracle.blocks_to_tokens(rl[None, None, :, None], T, H, W)[0, :, 0, 0]
+        got = o_tok[0, :, h].double().cpu().numpy()
+        rel = np.linalg.norm(got - ro_tok) / np.linalg.norm(ro_tok)
+        assert rel <= hx.O_REL_L2 and np.max(np.abs(got - ro_tok)) <= hx.O_MAX_ABS, (h, rel)
+        assert np.max(np.abs(lse_tok[0, :, h].double().cpu().numpy() - rl_tok)) <= hx.LSE_MAX_ABS
