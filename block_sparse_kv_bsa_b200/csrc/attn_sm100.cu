@@ -86,8 +86,7 @@ enum {
   B_V_EMPTY = B_V_FULL + kVSlots,     // + V slot: its P V is done
   B_PV_READY = B_V_EMPTY + kVSlots,   // + slot t % 3: P_t stored, V_t and K_{t+3} landed
   B_S_FULL = B_PV_READY + kVSlots,    // + S buffer: the S of its tile is ready
-  B_O_READY = B_S_FULL + kSBufs,      // + tile parity: the P V of that tile is done
-  B_MMA_DONE = B_O_READY + 2,         // + issuer (0: P V thread, 1: Q K^T thread)
+  B_MMA_DONE = B_S_FULL + kSBufs,     // + issuer (0: P V thread, 1: Q K^T thread)
   B_MMA_DONE_END = B_MMA_DONE + 2,
   B_COUNT = B_MMA_DONE_END
 };
@@ -151,41 +150,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
 }
 __device__ __forceinline__ void named_bar_arrive(int id, int count) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-// Exponentials of the first kPolyPairs column pairs of every 64 are computed
-// on the FMA pipe (ex2_poly2) instead of the MUFU, which is otherwise as busy
-// per tile as the tensor core: 128 x 128 exponentials per tile at 16 per SM
-// clock take as long as the tile's two 128x128x128 products.
-#ifndef BSA_ATTN_POLY_PAIRS
-#define BSA_ATTN_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = BSA_ATTN_POLY_PAIRS;
-
-// 2^x for a pair of arguments without the MUFU.  x = j + f with j = round(x)
-// (adding and subtracting 1.5 * 2^23 rounds to an integer, whose bits end up
-// in the low mantissa of the sum) and f in [-0.5, 0.5]; 2^f is a cubic
-// fitted for this kernel by Remez exchange to minimise the relative error on
-// [-0.5, 0.5] (at most 7.5e-5, far below the bf16 rounding of P); 2^j is
-// added to the exponent field: (bits(x + 1.5*2^23) << 23) == j << 23 modulo
-// 2^32.  x is clamped at -126 first, so masked keys (-inf) give about 1e-38.
-__device__ __forceinline__ void ex2_poly2(uint64_t x2, float& e0, float& e1) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  constexpr float kC0 = 0.99992806f, kC1 = 0.69326097f, kC2 = 0.24261113f, kC3 = 0.05517167f;
-  float x0, x1;
-  f2_unpack(x2, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
-  const uint64_t jf = f2_add(t, f2_pack(-kMagic, -kMagic));
-  const uint64_t fr = f2_fma(jf, f2_pack(-1.f, -1.f), xc);
-  uint64_t p = f2_fma(fr, f2_pack(kC3, kC3), f2_pack(kC2, kC2));
-  p = f2_fma(p, fr, f2_pack(kC1, kC1));
-  p = f2_fma(p, fr, f2_pack(kC0, kC0));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 // Maximum of three floats in one instruction (sm_100).
@@ -349,7 +313,6 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                       (i > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(&bars[B_V_EMPTY + sl]);
-          tc_commit(&bars[B_O_READY + (i & 1)]);
         }
       }
       if (!ok) {
@@ -500,17 +463,10 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
-          const uint64_t x2 =
-              f2_fma(f2_pack(s[64 * q + 2 * c], s[64 * q + 2 * c + 1]), scale2, neg_m2);
-          float e0, e1;
-          if (c < kPolyPairs) {
-            ex2_poly2(x2, e0, e1);
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            e0 = ex2_approx(x0);
-            e1 = ex2_approx(x1);
-          }
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[64 * q + 2 * c], s[64 * q + 2 * c + 1]), scale2, neg_m2), x0,
+                    x1);
+          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
           acc2[c & 1] = f2_add(acc2[c & 1], f2_pack(e0, e1));
           pk[c] = pack_bf16x2(e0, e1);
         }
@@ -526,20 +482,22 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       l += rs;
 
-      // The P V of the previous tile (accumulated against m_prev) completes
-      // before this tile's P is released, so that a larger reference can
-      // rescale O in between; this also keeps the arrivals of consecutive
-      // tiles on the PV_READY barriers apart.  It costs the tensor pipe
-      // nothing: this tile's P V queues behind Q K^T of tile t + 2 anyway.
-      // Warpgroup g is the only waiter on O_READY + (g ^ 1) here and waits
-      // for each of its completions in turn, so the parity is exact.
-      // tcgen05.ld/st are warp-collective: the branch is warp-uniform and a
-      // lane whose reference did not move scales by exactly 1.
-      if (ok && t > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_O_READY + (g ^ 1)],
-                                                       ((t - 1) >> 1) & 1, s_abort, kWaitLimit));
+      // A row whose reference moved (rare under the stale-maximum rule)
+      // rescales O after the P V of tile t - 1 has completed and before this
+      // tile's P is released; a warp with no such row releases at once.
+      // That completion is V_EMPTY of slot (t - 1) % 3, phase (t - 1) / 3.
+      // The wait is exact: the previous phase (P V of tile t - 4) completed
+      // before Q K^T of tile t - 1 was issued, whose S the other warpgroup
+      // saw before handing over the token this warpgroup holds; and the next
+      // phase (P V of tile t + 2) needs this tile's P V first, which needs
+      // this release.  tcgen05.ld/st are warp-collective: the branch is
+      // warp-uniform and a lane whose reference did not move scales by 1.
+      if (ok && t > 0 && __any_sync(0xffffffffu, m_t != m_prev)) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait_bounded(&bars[B_V_EMPTY + (t - 1) % kVSlots],
+                                          ((t - 1) / kVSlots) & 1, s_abort, kWaitLimit));
         const bool grow = m_t != m_prev;
-        if (ok && __any_sync(0xffffffffu, grow)) {
+        if (ok) {
           tc_fence_after();
           const float alpha = grow ? ex2_approx(m_prev - m_t) : 1.0f;
 #pragma unroll
@@ -574,24 +532,26 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // normalises D/2 output columns; warpgroup 0 writes the LSE.
     const int q_valid = a.q_valid != nullptr ? a.q_valid[j] : kBlk;
     const long long grow_idx = item * kBlk + r;
-    // The last P V (tile n - 1) is awaited by the warpgroup that did not
-    // process tile n - 1: in its loop it waited for every earlier completion
-    // of that barrier, so the parity is exact.  The named barrier then
-    // releases both; that commit covers every earlier MMA of the issuer.
-    if (ok && n > 0 && g == (n & 1)) {
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_O_READY + ((n - 1) & 1)],
-                                                     ((n - 1) >> 1) & 1, s_abort, kWaitLimit));
+    // The last P V (tile n - 1) is awaited by the warpgroup that processed
+    // tile n - 1 (it saw S_{n-1}, issued after the P V of tile n - 4 had
+    // completed, so the phase of V_EMPTY is exact); that completion covers
+    // every earlier MMA of the issuer, and every Q K^T completed before
+    // S_{n-1}.  The named barrier then releases both warpgroups: K slot 0 is
+    // free for the merge and O is final.
+    if (ok && n > 0 && g == ((n - 1) & 1)) {
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded(&bars[B_V_EMPTY + (n - 1) % kVSlots],
+                                        ((n - 1) / kVSlots) & 1, s_abort, kWaitLimit));
       if (!ok) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
         *s_abort = 1;
       }
     }
-    // Every Q K^T has completed by now (warpgroup (n - 1) & 1 saw the last
-    // S, the other the last P V), so K slot 0 is free for the merge.
+    tc_fence_before();
+    named_bar_sync(9, kSoftmaxThreads);
     float* fin = reinterpret_cast<float*>(sm + L::kFin);  // [m, l][warpgroup][128 rows]
     fin[(0 * 2 + g) * kBlk + r] = m_last;
     fin[(1 * 2 + g) * kBlk + r] = l;
-    tc_fence_before();
     named_bar_sync(9, kSoftmaxThreads);
     tc_fence_after();
     ok = __all_sync(0xffffffffu, ok && *s_abort == 0);
