@@ -897,7 +897,7 @@ def run_ours(args, rank, world, local, pg):
                      "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} burst dense bf16 (cuBLAS)",
                      "kernel": "bsa_attn_kernel<128, true>",
-                     "traffic": (measured_traffic("bsa_attn_kernel<128>")
+                     "traffic": (measured_traffic("bsa_attn_kernel<128, true>")
                                  if args.chunk == CHUNK else None)},
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
