@@ -9,7 +9,8 @@ with 30% zeros, lambda = 2, g_ref = 0.2).  The cache of the 47 earlier
 chunks is built before timing.
 
 One step = one pass of the whole path over chunk 48:
-  bsa_kv_append (K, V) -> bsa_tokens_to_blocks (Q) -> bsa_route ->
+  bsa_tokens_to_blocks_mean (Q and its block means) -> bsa_route_qmean,
+  with bsa_kv_append (K, V) on a forked stream beside the route ->
   bsa_attn -> bsa_blocks_to_tokens (O)
 and the chunk's blocks are rewritten in place every step.
 
@@ -53,7 +54,7 @@ CHUNK = 48
 BLK = 128
 METRIC = "bsa_attn selected-block TFLOP/s at chunk 48 (48-chunk sweep), 1 B200"
 L2_FLUSH_BYTES = 256 << 20
-KERNELS_PER_STEP = 5  # append (fused), Q to blocks + means, score_means, topk, attn (O to tokens)
+KERNELS_PER_STEP = 6  # append (fused), Q to blocks + means, score_means, topk, attn, O to tokens
 
 
 def parse_args():
@@ -494,7 +495,8 @@ class State:
         self.cnt = torch.empty((w.B, w.Hh, nbc), dtype=torch.int32, device=device)
         ws = bsa.bsa_route_workspace_size(w.B, w.Hh, w.D, nbc, self.n_hist)
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=device)
-        self.lse = torch.empty((w.B, w.tokens, w.Hh), dtype=torch.float32, device=device)
+        self.o_blk = torch.empty_like(self.q_blk)
+        self.lse = torch.empty((w.B, w.Hh, nbc * BLK), dtype=torch.float32, device=device)
         self.o_tok = torch.empty_like(self.q_tok)
         self.side = torch.cuda.Stream(device)
         self.step_graph = None
@@ -503,10 +505,12 @@ class State:
         self.q_valid = self.cache.block_valid[self.own_first:self.own_first + nbc].clone()
 
     def calls(self):
-        """The four library calls of one step, in order, as (name, fn): the
+        """The five library calls of one step, in order, as (name, fn): the
         query chunk is reordered and pooled in one pass, the route scores
-        from those means (so the query blocks are read once), and the
-        attention writes O and LSE straight back in raster token order."""
+        from those means (so the query blocks are read once), and O goes
+        back to raster token order after the attention.  (bsa_attn_tokens,
+        which writes O in token order from the attention epilogue, measured
+        slower at chunk 48: 1.016 ms against 0.967 + 0.020 ms.)"""
         bsa, w = self.bsa, self.w
         T, H, W = self.grid
 
@@ -521,10 +525,11 @@ class State:
                 self.q_mean, self.cache, self.n_hist, self.own_first, self.n_own, w.top_k[0],
                 g=self.g, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale, max_sel=self.max_sel,
                 idx=self.idx, cnt=self.cnt, workspace=self.ws)),
-            ("attn", lambda: bsa.bsa_attn_tokens(self.q_blk, self.cache, self.idx, self.cnt,
-                                                 T, H, W, q_valid=self.q_valid,
-                                                 sm_scale=w.sm_scale, o=self.o_tok,
-                                                 lse=self.lse)),
+            ("attn", lambda: bsa.bsa_attn(self.q_blk, self.cache, self.idx, self.cnt,
+                                          q_valid=self.q_valid, sm_scale=w.sm_scale,
+                                          o=self.o_blk, lse=self.lse)),
+            ("o_to_tokens", lambda: bsa.bsa_blocks_to_tokens(self.o_blk, T, H, W,
+                                                             out=self.o_tok)),
         ]
 
     def step(self, record=None):
@@ -537,9 +542,9 @@ class State:
         append fills the time of the latency-bound route kernels (started
         together with the HBM-bound Q reordering instead, the two streams
         only slowed each other).  The attention waits for both.
-        ``record(i, stream)`` marks the event points 0..5: start, Q
-        reordered, append done (side stream), routed, joined, attention done
-        (O in token order)."""
+        ``record(i, stream)`` marks the event points 0..6: start, Q
+        reordered, append done (side stream), routed, joined, attention
+        done, O reordered."""
         main = torch.cuda.current_stream(self.device)
         calls = dict(self.calls())
         mark = record if record is not None else (lambda i, stream: None)
@@ -556,11 +561,13 @@ class State:
         mark(4, main)
         calls["attn"]()
         mark(5, main)
+        calls["o_to_tokens"]()
+        mark(6, main)
 
     # (name, first event, last event) of each timed span of a step
     SPANS = (("q_to_blocks", 0, 1), ("append", 1, 2), ("route", 1, 3), ("attn", 4, 5),
-             ("step", 0, 5))
-    N_EVENTS = 6
+             ("o_to_tokens", 5, 6), ("step", 0, 6))
+    N_EVENTS = 7
 
     def capture(self):
         """The step as one CUDA graph (the side stream's fork and join become
@@ -872,8 +879,8 @@ def run_ours(args, rank, world, local, pg):
                  "selected_tflop_per_call": round(flops / 1e12, 4)},
         "phases_ms": {k: round(v, 4) for k, v in phase_ms.items()},
         "phases_note": "spans inside the timed steps: append runs on a forked stream while "
-                       "the route runs, so those two overlap; q_to_blocks and attn (which "
-                       "writes O and LSE in token order) have the GPU to themselves",
+                       "the route runs, so those two overlap; q_to_blocks, attn and "
+                       "o_to_tokens have the GPU to themselves",
         "isolated_ms": {k: round(v, 4) for k, v in isolated.items()},
         "step_ms_spread": step_spread,
         "timing": st.timing + "; each step read back before the next",
@@ -896,8 +903,8 @@ def run_ours(args, rank, world, local, pg):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} burst dense bf16 (cuBLAS)",
-                     "kernel": "bsa_attn_kernel<128, true>",
-                     "traffic": (measured_traffic("bsa_attn_kernel<128, true>")
+                     "kernel": "bsa_attn_kernel<128, false>",
+                     "traffic": (measured_traffic("bsa_attn_kernel<128, false>")
                                  if args.chunk == CHUNK else None)},
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * args.steps,
