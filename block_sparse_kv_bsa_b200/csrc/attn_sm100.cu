@@ -27,10 +27,10 @@
 //               rows x D bf16 in 128-byte swizzled boxes of 64 columns; K runs
 //               two tiles ahead of V, the order in which the products consume
 //               them.  Tile row = ((b*Hh + h)*max_blocks + blk)*128.
-//   warp 1      allocates tensor memory; one lane issues O += P_t V_t once
+//   warp 1      allocates tensor memory; one elected lane issues O += P_t V_t once
 //               the softmax warpgroup has stored P_t and seen V_t land (one
 //               barrier per tile).
-//   warp 2      one lane issues S_t = Q K_t^T once K_t has landed and the
+//   warp 2      one elected lane issues S_t = Q K_t^T once K_t has landed and the
 //               P V of tile t - 3 (which read P from the same buffer) is done.
 //               The tensor pipe is fed only as fast as its issuing threads
 //               issue: a wait in an issuing thread, and every instruction it
@@ -133,13 +133,15 @@ __device__ __forceinline__ int route_count(const AttnArgs& a, long long item) {
   return n;
 }
 
-__device__ __forceinline__ int route_block(const AttnArgs& a, long long item, int i) {
-  int blk = a.idx[item * a.max_sel + i];
+__device__ __forceinline__ int checked_block(const AttnArgs& a, int blk) {
   if (blk < 0 || blk >= a.n_blocks) {
     report(a.d_err, BSA_DEV_BAD_INDEX);
     blk = 0;
   }
   return blk;
+}
+__device__ __forceinline__ int route_block(const AttnArgs& a, long long item, int i) {
+  return checked_block(a, a.idx[item * a.max_sel + i]);
 }
 
 // Named barriers 1-8 carry the row-maximum tokens between the two softmax
@@ -166,7 +168,8 @@ __device__ __forceinline__ float fmax3(float x, float y, float z) {
 template <int D, bool kTokOut>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                AttnArgs a) {
   using L = AttnLayout<D>;
   constexpr int kBoxes = D / 64;
   constexpr uint32_t kTileBytes = L::kTileBytes;
@@ -202,11 +205,11 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // router) finishes; the route and Q are read only after it completed.
   pdl_wait();
   pdl_trigger();
-  const int n = route_count(a, item);
-
+  // The producer starts Q's copy and reads the first route entry before the
+  // route count arrives (every row of idx has max_sel >= 1 entries).
+  int first_blk = 0;
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0 && n > 0) {
+    if (elect_one()) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -214,13 +217,23 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int bx = 0; bx < kBoxes; ++bx)
         tma_load_2d(sm + L::kQ + bx * (kBlk * 128), &tm_q, bx * 64, static_cast<int>(item * kBlk),
                     &bars[B_Q_FULL]);
+    }
+    __syncwarp();
+    first_blk = a.idx[item * a.max_sel];
+  }
+  const int n = route_count(a, item);
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
       int k_issued = 0, v_issued = 0;
       bool ok = true;
       // Step s issues K_s (while s < n), then V_{s - kKLead}.
       for (int step = 0; ok && step < n + kKLead; ++step) {
         if (step < n) {
           const int t = step, sl = t % kKSlots;
-          const int row = static_cast<int>((bh * a.max_blocks + route_block(a, item, t)) * kBlk);
+          const int blk = t == 0 ? checked_block(a, first_blk) : route_block(a, item, t);
+          const int row = static_cast<int>((bh * a.max_blocks + blk) * kBlk);
           if (t >= kKSlots)
             ok = mbar_wait_bounded(&bars[B_K_EMPTY + sl], ((t / kKSlots) - 1) & 1, s_abort,
                                    kWaitLimit);
@@ -250,7 +263,8 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
         *s_abort = 1;
       }
-      // Drain: every copy this thread issued must land before the CTA exits.
+      // Drain: every copy this warp issued (Q's too, issued whatever n is)
+      // must land before the CTA exits.
       mbar_wait_bounded(&bars[B_Q_FULL], 0, nullptr, kWaitLimit);
       for (int sl = 0; sl < kKSlots; ++sl) {
         int last = -1;
@@ -270,58 +284,72 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // Warp 1 issues O += P_t V_t, warp 2 issues S_t = Q K_t^T: two threads on
     // two SM sub-partitions, so that one's waits do not leave the tensor pipe
     // without queued work.  Q K^T_t overwrites the S buffer whose P the
-    // P V of tile t - 3 read, so it waits for that P V to complete.
-    if (lane == 0 && n > 0) {
+    // P V of tile t - 3 read, so it waits for that P V to complete.  The
+    // whole warp runs the loop and the waits and one elected lane issues
+    // (measured 1-1.5 % faster than a loop run by lane 0 alone).
+    if (n > 0) {
       constexpr uint32_t kSlot16 = kTileBytes >> 4;
       bool ok = true;
       if (warp == 2) {
         constexpr uint32_t kIdQK = idesc_bf16(128, 128, 0);
         const uint64_t q_desc = smem_desc(smem_u32(sm + L::kQ), 16, 1024);
         const uint64_t k_desc0 = smem_desc(smem_u32(sm + L::kK), 16, 1024);
-        ok = mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit);
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_Q_FULL], 0, s_abort, kWaitLimit));
         for (int t = 0; ok && t < n; ++t) {
           const int sl = t % kKSlots;
-          ok = mbar_wait_bounded(&bars[B_K_FULL + sl], (t / kKSlots) & 1, s_abort, kWaitLimit);
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_K_FULL + sl], (t / kKSlots) & 1,
+                                                         s_abort, kWaitLimit));
           if (ok && t >= kSBufs)
-            ok = mbar_wait_bounded(&bars[B_V_EMPTY + t % kVSlots], ((t / kVSlots) - 1) & 1,
-                                   s_abort, kWaitLimit);
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait_bounded(&bars[B_V_EMPTY + t % kVSlots],
+                                              ((t / kVSlots) - 1) & 1, s_abort, kWaitLimit));
           if (!ok) break;
           tc_fence_after();
           const uint64_t k_desc = desc_add(k_desc0, sl * kSlot16);
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * (kBlk * 128) + (kk % 4) * 32) >> 4;
-            tc_mma_ss(tmem + (t % kSBufs) * 128, desc_add(q_desc, off), desc_add(k_desc, off),
-                      kIdQK, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = ((kk / 4) * (kBlk * 128) + (kk % 4) * 32) >> 4;
+              tc_mma_ss(tmem + (t % kSBufs) * 128, desc_add(q_desc, off), desc_add(k_desc, off),
+                        kIdQK, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bars[B_K_EMPTY + sl]);
+            tc_commit(&bars[B_S_FULL + t % kSBufs]);
           }
-          tc_commit(&bars[B_K_EMPTY + sl]);
-          tc_commit(&bars[B_S_FULL + t % kSBufs]);
+          __syncwarp();
         }
       } else {
         constexpr uint32_t kIdPV = idesc_bf16(128, D, 1);
         const uint64_t v_desc0 = smem_desc(smem_u32(sm + L::kV), kBlk * 128, 1024);
         for (int i = 0; ok && i < n; ++i) {
           const int sl = i % kVSlots;
-          ok = mbar_wait_bounded(&bars[B_PV_READY + sl], (i / kVSlots) & 1, s_abort, kWaitLimit);
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[B_PV_READY + sl], (i / kVSlots) & 1,
+                                                         s_abort, kWaitLimit));
           if (!ok) break;
           tc_fence_after();
           const uint32_t p_col = tmem + (i % kSBufs) * 128;
           const uint64_t v_desc = desc_add(v_desc0, sl * kSlot16);
+          if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk) {
-            tc_mma_ts(tmem + kColO, p_col + kk * 8, desc_add(v_desc, (kk * 2048) >> 4), kIdPV,
-                      (i > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < kBlk / 16; ++kk) {
+              tc_mma_ts(tmem + kColO, p_col + kk * 8, desc_add(v_desc, (kk * 2048) >> 4), kIdPV,
+                        (i > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&bars[B_V_EMPTY + sl]);
           }
-          tc_commit(&bars[B_V_EMPTY + sl]);
+          __syncwarp();
         }
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
         *s_abort = 1;
       }
-      // Drain: all MMAs issued by this thread complete before TMEM is freed.
-      tc_commit(&bars[B_MMA_DONE + (warp - 1)]);
-      mbar_wait_bounded(&bars[B_MMA_DONE + (warp - 1)], 0, nullptr, kWaitLimit);
+      // Drain: all MMAs issued by lane 0 complete before TMEM is freed.
+      if (lane == 0) {
+        tc_commit(&bars[B_MMA_DONE + (warp - 1)]);
+        mbar_wait_bounded(&bars[B_MMA_DONE + (warp - 1)], 0, nullptr, kWaitLimit);
+      }
+      __syncwarp();
     }
   } else if (warp == 3) {
     // ---------------- row -> raster token table (token-order output) ----------------
@@ -588,11 +616,36 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         v.y = pack_bf16x2(have ? o[e + 2] * inv_l : 0.f, have ? o[e + 3] * inv_l : 0.f);
         v.z = pack_bf16x2(have ? o[e + 4] * inv_l : 0.f, have ? o[e + 5] * inv_l : 0.f);
         v.w = pack_bf16x2(have ? o[e + 6] * inv_l : 0.f, have ? o[e + 7] * inv_l : 0.f);
-        if (write_row) *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
+        if (kTokOut) {
+          if (write_row) *reinterpret_cast<uint4*>(orow + c * 32 + e) = v;
+        } else {
+          // Block order: staged in K slot 1 (free: every Q K^T has
+          // completed) in the layout of a loaded tile -- 64-column boxes
+          // of 128 rows x 128 bytes, 16-byte chunk j of row r at chunk
+          // j ^ (r % 8) -- and written by TMA below.
+          const int col = g * (D / 2) + c * 32 + e;
+          uint8_t* stage = sm + L::kK + kTileBytes + (col / 64) * (kBlk * 128);
+          *reinterpret_cast<uint4*>(stage + r * 128 + ((((col % 64) / 8) ^ (r & 7)) * 16)) = v;
+        }
       }
     }
     if (g == 0 && write_row)
       a.lse[out_row] = have ? (m_fin + __log2f(l_tot)) * 0.6931471805599453f : -INFINITY;
+    if (!kTokOut) {
+      // Both warpgroups' halves are staged; one thread writes the tile
+      // (coalesced, where 128 threads writing their own rows would each
+      // touch a different 256-byte row per store) and waits until the
+      // copy has read shared memory, before the CTA can exit.
+      fence_proxy_async_smem();
+      named_bar_sync(9, kSoftmaxThreads);
+      if (warp == 4 && elect_one()) {
+        for (int bx = 0; bx < kBoxes; ++bx)
+          tma_store_2d(&tm_o, bx * 64, static_cast<int>(item * kBlk),
+                       sm + L::kK + kTileBytes + bx * (kBlk * 128));
+        bulk_commit_group();
+        bulk_wait_read_all();
+      }
+    }
   }
 
   tc_fence_before();
@@ -645,17 +698,23 @@ static bool device_is_sm100() {
 template <int D, bool kTokOut>
 static bsa_status launch_attn(const void* q, const bsa_kv_cache* c, const AttnArgs& a,
                               long long items, cudaStream_t s) {
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   const long long crows = static_cast<long long>(c->B) * c->Hh * c->max_blocks * kBlk;
   if (!make_map(&tq, q, items * kBlk, D) || !make_map(&tk, c->k, crows, D) ||
       !make_map(&tv, c->v, crows, D))
     return BSA_ERR_CUDA;
+  // O in block order has Q's layout; the token-order kernel stores O itself.
+  if (kTokOut) {
+    to = tq;
+  } else if (!make_map(&to, a.o, items * kBlk, D)) {
+    return BSA_ERR_CUDA;
+  }
   const int smem = AttnLayout<D>::kAlloc;
   if (cudaFuncSetAttribute(bsa_attn_kernel<D, kTokOut>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BSA_ERR_CUDA;
   return launch_pdl(bsa_attn_kernel<D, kTokOut>, dim3(static_cast<unsigned>(items)),
-                    dim3(kAttnThreads), static_cast<size_t>(smem), s, tq, tk, tv, a);
+                    dim3(kAttnThreads), static_cast<size_t>(smem), s, tq, tk, tv, to, a);
 }
 
 }  // namespace bsa
