@@ -55,6 +55,8 @@ BLK = 128
 METRIC = "bsa_attn selected-block TFLOP/s at chunk 48 (48-chunk sweep), 1 B200"
 L2_FLUSH_BYTES = 256 << 20
 KERNELS_PER_STEP = 6  # append (fused), Q to blocks + means, score_means, topk, attn, O to tokens
+# The step's attention kernel as ncu names it (block-order output, D = 128).
+ATTN_KERNEL = "bsa_attn_kernel<128, false>"
 
 
 def parse_args():
@@ -903,8 +905,8 @@ def run_ours(args, rank, world, local, pg):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peaks["bf16_tflops"], 4),
                      "peak_source": f"{peaks['source']} burst dense bf16 (cuBLAS)",
-                     "kernel": "bsa_attn_kernel<128, false>",
-                     "traffic": (measured_traffic("bsa_attn_kernel<128, false>")
+                     "kernel": ATTN_KERNEL,
+                     "traffic": (measured_traffic(ATTN_KERNEL)
                                  if args.chunk == CHUNK else None)},
         "e2e": e2e,
         "gpu_launches": KERNELS_PER_STEP * args.steps,

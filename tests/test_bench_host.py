@@ -56,7 +56,7 @@ def test_stored_traffic_matches_the_current_sources():
     with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
         table = json.load(f)
     kernels = [k for k in table if not k.startswith("_")]
-    assert "bsa_attn_kernel<128>" in kernels and "append_gather_kernel<16>" in kernels
+    assert bench.ATTN_KERNEL in kernels and "append_gather_kernel<16>" in kernels
     for k in kernels:
         for rel in table[k]["files"]:
             assert os.path.exists(os.path.join(bench.ROOT, rel)), (k, rel)
