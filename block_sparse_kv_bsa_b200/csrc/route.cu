@@ -912,80 +912,80 @@ __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a,
       if (mass_k < v.mass - 1.2e-7f * static_cast<float>(K + 1)) {
         select_run(thr, need_eq, [&](int n) { flag[n] = 1; });
       } else {
-      int sel_local = 0;
-      select_run(thr, need_eq, [&](int) { ++sel_local; });
-      int sel_tot;
-      int at = block_excl_scan(sel_local, warp_tot, &sel_tot);
-      // ascending order of ~((key << 32) | ~n) = descending key, ascending n
-      select_run(thr, need_eq, [&](int n) {
-        sortbuf[at++] = ~((static_cast<uint64_t>(keys[n]) << 32) |
-                          (0xFFFFFFFFu - static_cast<uint32_t>(n)));
-      });
-      __syncthreads();
-      if (K <= kVeloxRankMax) {
-        // Rank by counting (the values are distinct): one barrier instead of
-        // a sorting network.
-        for (int u = t; u < K; u += kTopkThreads) {
-          const uint64_t x = sortbuf[u];
-          int rank = 0;
-          for (int i = 0; i < K; ++i) rank += sortbuf[i] < x;
-          const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~x));
-          nidx[rank] = n;
-          pr[rank] = expf(sr[n] - smax) / zsum;
-        }
+        int sel_local = 0;
+        select_run(thr, need_eq, [&](int) { ++sel_local; });
+        int sel_tot;
+        int at = block_excl_scan(sel_local, warp_tot, &sel_tot);
+        // ascending order of ~((key << 32) | ~n) = descending key, ascending n
+        select_run(thr, need_eq, [&](int n) {
+          sortbuf[at++] = ~((static_cast<uint64_t>(keys[n]) << 32) |
+                            (0xFFFFFFFFu - static_cast<uint32_t>(n)));
+        });
         __syncthreads();
-        if (t == 0) {
-          float acc = 0.f;
-          int m = K;
-          for (int r = 0; r < K; ++r) {
-            acc += pr[r];
-            if (acc >= v.mass) {
-              m = r + 1;
-              break;
-            }
+        if (K <= kVeloxRankMax) {
+          // Rank by counting (the values are distinct): one barrier instead of
+          // a sorting network.
+          for (int u = t; u < K; u += kTopkThreads) {
+            const uint64_t x = sortbuf[u];
+            int rank = 0;
+            for (int i = 0; i < K; ++i) rank += sortbuf[i] < x;
+            const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~x));
+            nidx[rank] = n;
+            pr[rank] = expf(sr[n] - smax) / zsum;
           }
-          s_m = m;
-        }
-        __syncthreads();
-        for (int r = t; r < s_m; r += kTopkThreads) flag[nidx[r]] = 1;
-      } else {
-        int P = 2;
-        while (P < K) P <<= 1;
-        for (int i = K + t; i < P; i += kTopkThreads) sortbuf[i] = ~0ull;
-        __syncthreads();
-        for (int kk = 2; kk <= P; kk <<= 1) {
-          for (int jj = kk >> 1; jj > 0; jj >>= 1) {
-            for (int i = t; i < P; i += kTopkThreads) {
-              const int ixj = i ^ jj;
-              if (ixj > i) {
-                const uint64_t x = sortbuf[i], y = sortbuf[ixj];
-                const bool up = (i & kk) == 0;
-                if (up ? (x > y) : (x < y)) {
-                  sortbuf[i] = y;
-                  sortbuf[ixj] = x;
-                }
+          __syncthreads();
+          if (t == 0) {
+            float acc = 0.f;
+            int m = K;
+            for (int r = 0; r < K; ++r) {
+              acc += pr[r];
+              if (acc >= v.mass) {
+                m = r + 1;
+                break;
               }
             }
-            __syncthreads();
+            s_m = m;
           }
-        }
-        if (t == 0) {
-          float acc = 0.f;
-          int m = K;
-          for (int r = 0; r < K; ++r) {
-            const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]));
-            acc += expf(sr[n] - smax) / zsum;
-            if (acc >= v.mass) {
-              m = r + 1;
-              break;
+          __syncthreads();
+          for (int r = t; r < s_m; r += kTopkThreads) flag[nidx[r]] = 1;
+        } else {
+          int P = 2;
+          while (P < K) P <<= 1;
+          for (int i = K + t; i < P; i += kTopkThreads) sortbuf[i] = ~0ull;
+          __syncthreads();
+          for (int kk = 2; kk <= P; kk <<= 1) {
+            for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+              for (int i = t; i < P; i += kTopkThreads) {
+                const int ixj = i ^ jj;
+                if (ixj > i) {
+                  const uint64_t x = sortbuf[i], y = sortbuf[ixj];
+                  const bool up = (i & kk) == 0;
+                  if (up ? (x > y) : (x < y)) {
+                    sortbuf[i] = y;
+                    sortbuf[ixj] = x;
+                  }
+                }
+              }
+              __syncthreads();
             }
           }
-          s_m = m;
+          if (t == 0) {
+            float acc = 0.f;
+            int m = K;
+            for (int r = 0; r < K; ++r) {
+              const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]));
+              acc += expf(sr[n] - smax) / zsum;
+              if (acc >= v.mass) {
+                m = r + 1;
+                break;
+              }
+            }
+            s_m = m;
+          }
+          __syncthreads();
+          for (int r = t; r < s_m; r += kTopkThreads)
+            flag[static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]))] = 1;
         }
-        __syncthreads();
-        for (int r = t; r < s_m; r += kTopkThreads)
-          flag[static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]))] = 1;
-      }
       }
     }
   }
