@@ -189,8 +189,41 @@ __device__ __forceinline__ void invert_block_slots(const int32_t* perm, int N, i
   static_assert(NT >= kBlk, "one thread per slot clears the table");
   if (threadIdx.x < kBlk) s_tok[threadIdx.x] = -1;
   __syncthreads();
+  auto take = [&](int r, int p) {
+    if (p < 0 || p >= N) {
+      if (report_bad) report(d_err, BSA_DEV_BAD_PERM);
+      return;
+    }
+    const unsigned d = static_cast<unsigned>(p - slot0);
+    if (d < static_cast<unsigned>(kBlk)) s_tok[d] = r;
+  };
   constexpr int kScan = 16;
-  for (int base = 0; base < N; base += kScan * NT) {
+  // Four entries per load when perm is 16-byte aligned: one round of loads
+  // covers 64 * NT tokens, so a chunk's scan costs one memory latency.
+  int done = 0;
+  if ((reinterpret_cast<uintptr_t>(perm) & 15u) == 0) {
+    const int n4 = N / 4;
+    const int4* perm4 = reinterpret_cast<const int4*>(perm);
+    for (int base = 0; base < n4; base += kScan * NT) {
+      int4 pv[kScan];
+#pragma unroll
+      for (int k = 0; k < kScan; ++k) {
+        const int i = base + threadIdx.x + k * NT;
+        pv[k] = i < n4 ? __ldg(perm4 + i) : make_int4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int k = 0; k < kScan; ++k) {
+        const int i = base + threadIdx.x + k * NT;
+        if (i >= n4) break;
+        take(4 * i, pv[k].x);
+        take(4 * i + 1, pv[k].y);
+        take(4 * i + 2, pv[k].z);
+        take(4 * i + 3, pv[k].w);
+      }
+    }
+    done = 4 * n4;
+  }
+  for (int base = done; base < N; base += kScan * NT) {
     int pv[kScan];
 #pragma unroll
     for (int k = 0; k < kScan; ++k) {
@@ -201,13 +234,7 @@ __device__ __forceinline__ void invert_block_slots(const int32_t* perm, int N, i
     for (int k = 0; k < kScan; ++k) {
       const int r = base + threadIdx.x + k * NT;
       if (r >= N) break;
-      const int p = pv[k];
-      if (p < 0 || p >= N) {
-        if (report_bad) report(d_err, BSA_DEV_BAD_PERM);
-        continue;
-      }
-      const unsigned d = static_cast<unsigned>(p - slot0);
-      if (d < static_cast<unsigned>(kBlk)) s_tok[d] = r;
+      take(r, pv[k]);
     }
   }
   __syncthreads();
