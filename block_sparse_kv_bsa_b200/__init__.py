@@ -248,12 +248,15 @@ class KVCache:
 
 
 def bsa_kv_append(cache: KVCache, k_tok: torch.Tensor, v_tok: torch.Tensor,
-                  T: int, H: int, W: int, d_err: Optional[torch.Tensor] = None) -> int:
-    """Append one chunk (bf16 [B, T*H*W, Hh, D] K and V); returns its first block."""
+                  T: int, H: int, W: int, d_err: Optional[torch.Tensor] = None,
+                  table: bool = True) -> int:
+    """Append one chunk (bf16 [B, T*H*W, Hh, D] K and V); returns its first block.
+    table=False passes no permutation table: the kernels locate the Gilbert
+    slots themselves (the same order)."""
     shape = (cache.B, T * H * W, cache.Hh, cache.D)
     _need(k_tok, "k_tok", torch.bfloat16, cache.device, shape)
     _need(v_tok, "v_tok", torch.bfloat16, cache.device, shape)
-    perm = gilbert_perm_device(T, H, W, cache.device)
+    perm = gilbert_perm_device(T, H, W, cache.device) if table else None
     err = error_word(cache.device) if d_err is None else d_err
     cs = cache.c_struct()
     first = cache.n_blocks
@@ -277,7 +280,7 @@ def bsa_kv_pool_means(cache: KVCache, first: int = 0, count: Optional[int] = Non
 
 
 def bsa_tokens_to_blocks(x_tok: torch.Tensor, T: int, H: int, W: int,
-                         out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                         out: Optional[torch.Tensor] = None, table: bool = True) -> torch.Tensor:
     """[B, T*H*W, Hh, D] raster tokens -> [B, Hh, nb*128, D] Gilbert blocks (zero pads)."""
     if x_tok.dim() != 4:
         raise ValueError("x_tok must be [B, T*H*W, Hh, D]")
@@ -287,7 +290,7 @@ def bsa_tokens_to_blocks(x_tok: torch.Tensor, T: int, H: int, W: int,
     if out is None:
         out = torch.empty((B, Hh, nb * BLK, D), dtype=torch.bfloat16, device=x_tok.device)
     _need(out, "out", torch.bfloat16, x_tok.device, (B, Hh, nb * BLK, D))
-    perm = gilbert_perm_device(T, H, W, x_tok.device)
+    perm = gilbert_perm_device(T, H, W, x_tok.device) if table else None
     _check("bsa_tokens_to_blocks", _lib.bsa_tokens_to_blocks(
         _ptr(x_tok), _ptr(out), B, Hh, D, int(T), int(H), int(W), _ptr(perm),
         _ptr(error_word(x_tok.device)), _stream(x_tok.device)))
@@ -296,7 +299,7 @@ def bsa_tokens_to_blocks(x_tok: torch.Tensor, T: int, H: int, W: int,
 
 def bsa_tokens_to_blocks_mean(x_tok: torch.Tensor, T: int, H: int, W: int,
                               out: Optional[torch.Tensor] = None,
-                              mean: Optional[torch.Tensor] = None
+                              mean: Optional[torch.Tensor] = None, table: bool = True
                               ) -> Tuple[torch.Tensor, torch.Tensor]:
     """bsa_tokens_to_blocks plus the fp32 mean of every block's valid rows:
     returns (blocks [B, Hh, nb*128, D], means [B, Hh, nb, D])."""
@@ -311,7 +314,7 @@ def bsa_tokens_to_blocks_mean(x_tok: torch.Tensor, T: int, H: int, W: int,
         mean = torch.empty((B, Hh, nb, D), dtype=torch.float32, device=x_tok.device)
     _need(out, "out", torch.bfloat16, x_tok.device, (B, Hh, nb * BLK, D))
     _need(mean, "mean", torch.float32, x_tok.device, (B, Hh, nb, D))
-    perm = gilbert_perm_device(T, H, W, x_tok.device)
+    perm = gilbert_perm_device(T, H, W, x_tok.device) if table else None
     _check("bsa_tokens_to_blocks_mean", _lib.bsa_tokens_to_blocks_mean(
         _ptr(x_tok), _ptr(out), _ptr(mean), B, Hh, D, int(T), int(H), int(W), _ptr(perm),
         _ptr(error_word(x_tok.device)), _stream(x_tok.device)))
@@ -319,7 +322,7 @@ def bsa_tokens_to_blocks_mean(x_tok: torch.Tensor, T: int, H: int, W: int,
 
 
 def bsa_blocks_to_tokens(x_blk: torch.Tensor, T: int, H: int, W: int,
-                         out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                         out: Optional[torch.Tensor] = None, table: bool = True) -> torch.Tensor:
     """[B, Hh, nb*128, D] Gilbert blocks -> [B, T*H*W, Hh, D] raster tokens."""
     if x_blk.dim() != 4:
         raise ValueError("x_blk must be [B, Hh, nb*128, D]")
@@ -330,7 +333,7 @@ def bsa_blocks_to_tokens(x_blk: torch.Tensor, T: int, H: int, W: int,
     if out is None:
         out = torch.empty((B, T * H * W, Hh, D), dtype=torch.bfloat16, device=x_blk.device)
     _need(out, "out", torch.bfloat16, x_blk.device, (B, T * H * W, Hh, D))
-    perm = gilbert_perm_device(T, H, W, x_blk.device)
+    perm = gilbert_perm_device(T, H, W, x_blk.device) if table else None
     _check("bsa_blocks_to_tokens", _lib.bsa_blocks_to_tokens(
         _ptr(x_blk), _ptr(out), B, Hh, D, int(T), int(H), int(W), _ptr(perm),
         _ptr(error_word(x_blk.device)), _stream(x_blk.device)))
@@ -558,7 +561,8 @@ def bsa_attn(q_blk: torch.Tensor, cache: KVCache, idx: torch.Tensor, cnt: torch.
 def bsa_attn_tokens(q_blk: torch.Tensor, cache: KVCache, idx: torch.Tensor, cnt: torch.Tensor,
                     T: int, H: int, W: int, q_valid: Optional[torch.Tensor] = None,
                     sm_scale: Optional[float] = None, o: Optional[torch.Tensor] = None,
-                    lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+                    lse: Optional[torch.Tensor] = None,
+                    table: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
     """bsa_attn writing O and LSE in raster token order; returns
     (O bf16 [B, T*H*W, Hh, D], LSE fp32 [B, T*H*W, Hh])."""
     dev = cache.device
@@ -585,7 +589,7 @@ def bsa_attn_tokens(q_blk: torch.Tensor, cache: KVCache, idx: torch.Tensor, cnt:
         lse = torch.empty((B, N, Hh), dtype=torch.float32, device=dev)
     _need(o, "o", torch.bfloat16, dev, (B, N, Hh, D))
     _need(lse, "lse", torch.float32, dev, (B, N, Hh))
-    perm = gilbert_perm_device(T, H, W, dev)
+    perm = gilbert_perm_device(T, H, W, dev) if table else None
     cs = cache.c_struct()
     _check("bsa_attn_tokens", _lib.bsa_attn_tokens(
         _ptr(q_blk), ctypes.byref(cs), _ptr(q_valid), _ptr(idx), _ptr(cnt), int(max_sel),

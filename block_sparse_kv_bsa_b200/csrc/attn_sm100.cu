@@ -60,6 +60,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "gilbert.cuh"
 
 namespace bsa {
 
@@ -120,6 +121,7 @@ struct AttnArgs {
   int32_t* d_err;
   const int32_t* perm;      // token -> curve slot (token-order output only)
   int n_tok;                // tokens of the chunk (token-order output only)
+  int T, H, W;              // chunk grid (token-order output without perm)
   int Hh, n_q_blocks, max_sel, max_blocks, n_blocks;
   float scale_log2;
 };
@@ -354,35 +356,43 @@ bsa_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   } else if (warp == 3) {
     // ---------------- row -> raster token table (token-order output) ----------------
     // s_tok[r] = the token whose curve slot is j*128 + r, or -1 (pad row):
-    // the lanes scan perm with 16 loads in flight each.  Released to the
+    // the lanes scan perm with 16 loads in flight each, or, without a table,
+    // locate the slots on the Gilbert curve themselves.  Released to the
     // softmax warps through named barrier 10 (arrive; they sync before
     // their stores).
     if (kTokOut) {
       int* s_tok = reinterpret_cast<int*>(sm + L::kSlotTok);
-      for (int i = lane; i < kBlk; i += 32) s_tok[i] = -1;
-      __syncwarp();
       const int slot0 = j * kBlk;
-      constexpr int kScan = 16;
-      for (int base = 0; base < a.n_tok; base += kScan * 32) {
-        int pv[kScan];
+      if (a.perm == nullptr) {
+        // No table: each lane locates its slots on the Gilbert curve.
+        for (int i = lane; i < kBlk; i += 32)
+          s_tok[i] = slot0 + i < a.n_tok ? curve_token(a.T, a.H, a.W, slot0 + i) : -1;
+        __syncwarp();
+      } else {
+        for (int i = lane; i < kBlk; i += 32) s_tok[i] = -1;
+        __syncwarp();
+        constexpr int kScan = 16;
+        for (int base = 0; base < a.n_tok; base += kScan * 32) {
+          int pv[kScan];
 #pragma unroll
-        for (int k = 0; k < kScan; ++k) {
-          const int t = base + lane + k * 32;
-          pv[k] = t < a.n_tok ? __ldg(a.perm + t) : -1;
-        }
-#pragma unroll
-        for (int k = 0; k < kScan; ++k) {
-          const int t = base + lane + k * 32;
-          if (t >= a.n_tok) break;
-          if (pv[k] < 0 || pv[k] >= a.n_tok) {
-            report(a.d_err, BSA_DEV_BAD_PERM);
-            continue;
+          for (int k = 0; k < kScan; ++k) {
+            const int t = base + lane + k * 32;
+            pv[k] = t < a.n_tok ? __ldg(a.perm + t) : -1;
           }
-          const unsigned d = static_cast<unsigned>(pv[k] - slot0);
-          if (d < static_cast<unsigned>(kBlk)) s_tok[d] = t;
+#pragma unroll
+          for (int k = 0; k < kScan; ++k) {
+            const int t = base + lane + k * 32;
+            if (t >= a.n_tok) break;
+            if (pv[k] < 0 || pv[k] >= a.n_tok) {
+              report(a.d_err, BSA_DEV_BAD_PERM);
+              continue;
+            }
+            const unsigned d = static_cast<unsigned>(pv[k] - slot0);
+            if (d < static_cast<unsigned>(kBlk)) s_tok[d] = t;
+          }
         }
+        __syncwarp();
       }
-      __syncwarp();
       // A slot of a token row that no token maps to: perm is no permutation.
       const int rows = min(kBlk, a.n_tok - slot0);
       for (int i = lane; i < rows; i += 32)
@@ -727,8 +737,8 @@ namespace bsa {
 // NULL for block-order output.
 static bsa_status attn_call(const void* q_blk, const bsa_kv_cache* c, const int32_t* q_valid,
                             const int32_t* idx, const int32_t* cnt, int n_q_blocks, int max_sel,
-                            float sm_scale, const int32_t* perm, int n_tok, void* o, float* lse,
-                            int32_t* d_err, void* stream) {
+                            float sm_scale, bool tok_out, const int32_t* perm, int T, int H,
+                            int W, void* o, float* lse, int32_t* d_err, void* stream) {
   if (q_blk == nullptr || c == nullptr || idx == nullptr || cnt == nullptr || o == nullptr ||
       lse == nullptr || c->k == nullptr || c->v == nullptr || c->block_valid == nullptr)
     return BSA_ERR_INVALID_ARG;
@@ -751,7 +761,10 @@ static bsa_status attn_call(const void* q_blk, const bsa_kv_cache* c, const int3
   a.lse = lse;
   a.d_err = d_err;
   a.perm = perm;
-  a.n_tok = n_tok;
+  a.n_tok = T * H * W;
+  a.T = T;
+  a.H = H;
+  a.W = W;
   a.Hh = c->Hh;
   a.n_q_blocks = n_q_blocks;
   a.max_sel = max_sel;
@@ -759,7 +772,7 @@ static bsa_status attn_call(const void* q_blk, const bsa_kv_cache* c, const int3
   a.n_blocks = c->n_blocks;
   a.scale_log2 = sm_scale * kLog2e;
   cudaStream_t s = as_stream(stream);
-  if (perm != nullptr)
+  if (tok_out)
     return c->D == 128 ? launch_attn<128, true>(q_blk, c, a, items, s)
                        : launch_attn<64, true>(q_blk, c, a, items, s);
   return c->D == 128 ? launch_attn<128, false>(q_blk, c, a, items, s)
@@ -772,8 +785,8 @@ extern "C" bsa_status bsa_attn(const void* q_blk, const bsa_kv_cache* c, const i
                                const int32_t* idx, const int32_t* cnt, int n_q_blocks, int max_sel,
                                float sm_scale, void* o_blk, float* lse, int32_t* d_err,
                                void* stream) {
-  return attn_call(q_blk, c, q_valid, idx, cnt, n_q_blocks, max_sel, sm_scale, nullptr, 0, o_blk,
-                   lse, d_err, stream);
+  return attn_call(q_blk, c, q_valid, idx, cnt, n_q_blocks, max_sel, sm_scale, false, nullptr, 0,
+                   0, 0, o_blk, lse, d_err, stream);
 }
 
 extern "C" bsa_status bsa_attn_tokens(const void* q_blk, const bsa_kv_cache* c,
@@ -781,10 +794,10 @@ extern "C" bsa_status bsa_attn_tokens(const void* q_blk, const bsa_kv_cache* c,
                                       const int32_t* cnt, int max_sel, float sm_scale, int T,
                                       int H, int W, const int32_t* d_perm, void* o_tok,
                                       float* lse_tok, int32_t* d_err, void* stream) {
-  if (d_perm == nullptr || T <= 0 || H <= 0 || W <= 0) return BSA_ERR_INVALID_ARG;
+  if (T <= 0 || H <= 0 || W <= 0) return BSA_ERR_INVALID_ARG;
   const long long n = static_cast<long long>(T) * H * W;
   if (n > kTokOutMaxTokens) return BSA_ERR_UNSUPPORTED;
   const int nb = static_cast<int>((n + kBlk - 1) / kBlk);
-  return attn_call(q_blk, c, q_valid, idx, cnt, nb, max_sel, sm_scale, d_perm,
-                   static_cast<int>(n), o_tok, lse_tok, d_err, stream);
+  return attn_call(q_blk, c, q_valid, idx, cnt, nb, max_sel, sm_scale, true, d_perm, T, H, W,
+                   o_tok, lse_tok, d_err, stream);
 }

@@ -200,4 +200,10 @@ __host__ __device__ inline V3 gilbert_cell(int T, int H, int W, int p) {
   return v3(-1, -1, -1);  // unreachable for valid input
 }
 
+// Raster index (t*H + h)*W + w of the cell at curve position p.
+__host__ __device__ inline int curve_token(int T, int H, int W, int p) {
+  const V3 c = gilbert_cell(T, H, W, p);
+  return (c.t * H + c.h) * W + c.w;
+}
+
 }  // namespace bsa

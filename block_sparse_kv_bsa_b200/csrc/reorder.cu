@@ -19,6 +19,11 @@
 
 namespace bsa {
 
+// The curve walk kept out of line: the kernels' table path stays compact.
+__device__ __noinline__ int curve_token_call(int T, int H, int W, int p) {
+  return curve_token(T, H, W, p);
+}
+
 constexpr int kRowsPerCta = 32;
 constexpr int kHeadsPerCta = 8;
 constexpr int kReorderThreads = 256;
@@ -37,6 +42,7 @@ struct ReorderArgs {
   int B, Hh;
   long long blk_stride; // blocks per (b, h) in the block tensor
   int base_block;       // first block of the chunk in the block tensor
+  int T, H, W;          // chunk grid (used when perm is NULL)
 };
 
 // kToBlocks: raster tokens -> block slots (scatter, zero pads).
@@ -46,26 +52,40 @@ __global__ void __launch_bounds__(kReorderThreads)
 reorder_kernel(ReorderArgs a) {
   pdl_wait();     // global memory only after the predecessor grid completed
   pdl_trigger();
+  // Row rr of the CTA moves token s_tk[rr] to curve slot s_slot[rr].  With a
+  // table, rows are tokens (slot = perm[token]; a scatter into blocks also
+  // covers the chunk's pad slots as rows past N).  Without one (perm ==
+  // NULL), rows are curve slots and each locates its token on the curve.
   __shared__ int s_slot[kRowsPerCta];
+  __shared__ int s_tk[kRowsPerCta];
   const int r0 = blockIdx.x * kRowsPerCta;
   const int h0 = blockIdx.y * kHeadsPerCta;
   const int b = blockIdx.z;
-  const int rows_total = kToBlocks ? a.nb * kBlk : a.N;
+  const bool by_slot = a.perm == nullptr;
+  const int rows_total = (kToBlocks || by_slot) ? a.nb * kBlk : a.N;
 
   if (threadIdx.x < kRowsPerCta) {
-    int r = r0 + threadIdx.x;
-    int slot = -1;
-    if (r < a.N) {
-      int p = __ldg(a.perm + r);
+    const int r = r0 + threadIdx.x;
+    int slot = -1, tk = -1;
+    if (by_slot) {
+      if (r < rows_total) {
+        slot = r;
+        tk = r < a.N ? curve_token_call(a.T, a.H, a.W, r) : -1;
+      }
+    } else if (r < a.N) {
+      const int p = __ldg(a.perm + r);
       if (p < 0 || p >= a.N) {
         report(a.d_err, BSA_DEV_BAD_PERM);
       } else {
         slot = p;
+        tk = r;
       }
     } else if (kToBlocks && r < rows_total) {
       slot = r;  // pad slot: zero-filled
     }
+    if (!kToBlocks && tk < 0) slot = -1;   // nothing to write for a pad slot
     s_slot[threadIdx.x] = slot;
+    s_tk[threadIdx.x] = tk;
     if (kToBlocks && a.block_valid != nullptr && blockIdx.y == 0 && b == 0 && r < rows_total &&
         (r % kBlk) == 0) {
       int blk = r / kBlk;
@@ -94,16 +114,17 @@ reorder_kernel(ReorderArgs a) {
       int rr = e / (kVecPerRow * kHeadsPerCta);
       int h = h0 + hh;
       int r = r0 + rr;
-      int slot = s_slot[rr];
+      const int slot = s_slot[rr];
       if (h >= a.Hh || r >= rows_total || slot < 0) continue;
+      const int tk = s_tk[rr];
       long long blk_row = (static_cast<long long>(b) * a.Hh + h) * a.blk_stride * kBlk +
                           static_cast<long long>(a.base_block) * kBlk + slot;
-      long long tok_row = (static_cast<long long>(b) * a.N + r) * tok_row_vecs +
+      long long tok_row = (static_cast<long long>(b) * a.N + (tk < 0 ? 0 : tk)) * tok_row_vecs +
                           static_cast<long long>(h) * kVecPerRow;
       live[u] = true;
       if (kToBlocks) {
         dsto[u] = blk_row * kVecPerRow + v;
-        if (r < a.N) {
+        if (tk >= 0) {
           v0[u] = ld_nc_v4(a.src0 + tok_row + v);
           if (a.src1 != nullptr) v1[u] = ld_nc_v4(a.src1 + tok_row + v);
         } else {
@@ -126,7 +147,7 @@ reorder_kernel(ReorderArgs a) {
 
 template <bool kToBlocks>
 static bsa_status launch_reorder(const ReorderArgs& a, int D, cudaStream_t s) {
-  const int rows = kToBlocks ? a.nb * kBlk : a.N;
+  const int rows = (kToBlocks || a.perm == nullptr) ? a.nb * kBlk : a.N;
   dim3 grid((rows + kRowsPerCta - 1) / kRowsPerCta, (a.Hh + kHeadsPerCta - 1) / kHeadsPerCta,
             a.B);
   if (D == 128) {
@@ -183,10 +204,22 @@ static bsa_status launch_block_means(const bsa_kv_cache* c, int first, int count
 // CTA's NT threads (NT >= 128) scan perm in rounds of kScan independent loads
 // per thread (one L2 round trip per round); entries outside [0, N) are
 // skipped, and reported when `report_bad`.  Ends with a CTA barrier.
+// s_tok[d] = the token at curve slot slot0 + d (d < 128), or -1 for a pad
+// slot.  With a table, the CTA scans perm (token -> slot); without one
+// (perm == NULL), each thread locates its slot on the curve.
 template <int NT>
 __device__ __forceinline__ void invert_block_slots(const int32_t* perm, int N, int slot0,
-                                                   int* s_tok, bool report_bad, int32_t* d_err) {
+                                                   int* s_tok, bool report_bad, int32_t* d_err,
+                                                   int T, int H, int W) {
   static_assert(NT >= kBlk, "one thread per slot clears the table");
+  if (perm == nullptr) {
+    if (threadIdx.x < kBlk) {
+      const int p = slot0 + static_cast<int>(threadIdx.x);
+      s_tok[threadIdx.x] = p < N ? curve_token_call(T, H, W, p) : -1;
+    }
+    __syncthreads();
+    return;
+  }
   if (threadIdx.x < kBlk) s_tok[threadIdx.x] = -1;
   __syncthreads();
   auto take = [&](int r, int p) {
@@ -261,6 +294,7 @@ struct AppendArgs {
   int32_t* block_valid;
   int32_t* d_err;
   int N, Hh, max_blocks, base_block;
+  int T, H, W;          // chunk grid (used when perm is NULL)
 };
 
 template <int VPR>
@@ -275,7 +309,8 @@ append_gather_kernel(AppendArgs a) {
   const int slot0 = j * kBlk;
   const int valid = min(kBlk, a.N - slot0);
   const bool first_cta = blockIdx.y == 0 && b == 0;
-  invert_block_slots<kAppendThreads>(a.perm, a.N, slot0, s_tok, j == 0 && first_cta, a.d_err);
+  invert_block_slots<kAppendThreads>(a.perm, a.N, slot0, s_tok, j == 0 && first_cta, a.d_err,
+                                     a.T, a.H, a.W);
   if (first_cta && threadIdx.x == 0) a.block_valid[a.base_block + j] = valid;
   // A slot of the chunk that no token maps to: perm is not a permutation.
   if (first_cta && threadIdx.x < valid && s_tok[threadIdx.x] < 0) report(a.d_err, BSA_DEV_BAD_PERM);
@@ -331,6 +366,7 @@ struct GatherMeanArgs {
   const int32_t* perm;
   int32_t* d_err;
   int N, Hh, nb;
+  int T, H, W;          // chunk grid (used when perm is NULL)
 };
 
 template <int VPR>
@@ -346,7 +382,7 @@ gather_mean_kernel(GatherMeanArgs a) {
   const int valid = min(kBlk, a.N - slot0);
   const bool first_cta = blockIdx.y == 0 && b == 0;
   invert_block_slots<kMeanGatherThreads>(a.perm, a.N, slot0, s_tok, j == 0 && first_cta,
-                                         a.d_err);
+                                         a.d_err, a.T, a.H, a.W);
   if (first_cta && threadIdx.x < valid && s_tok[threadIdx.x] < 0) report(a.d_err, BSA_DEV_BAD_PERM);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int h = blockIdx.y * kMeanHeads + warp;
@@ -417,7 +453,7 @@ extern "C" bsa_status bsa_gilbert_perm(int T, int H, int W, int32_t* host_perm) 
 extern "C" bsa_status bsa_kv_append(bsa_kv_cache* c, const void* k_tok, const void* v_tok, int T,
                                     int H, int W, const int32_t* d_perm, int32_t* d_err,
                                     void* stream) {
-  if (c == nullptr || k_tok == nullptr || v_tok == nullptr || d_perm == nullptr ||
+  if (c == nullptr || k_tok == nullptr || v_tok == nullptr ||
       c->k == nullptr || c->v == nullptr || c->block_valid == nullptr)
     return BSA_ERR_INVALID_ARG;
   bsa_status st = check_chunk(c->B, c->Hh, c->D, T, H, W);
@@ -439,6 +475,9 @@ extern "C" bsa_status bsa_kv_append(bsa_kv_cache* c, const void* k_tok, const vo
     g.vc = static_cast<uint4*>(c->v);
     g.kmean = c->kmean;
     g.perm = d_perm;
+    g.T = T;
+    g.H = H;
+    g.W = W;
     g.block_valid = c->block_valid;
     g.d_err = d_err;
     g.N = n;
@@ -454,6 +493,9 @@ extern "C" bsa_status bsa_kv_append(bsa_kv_cache* c, const void* k_tok, const vo
     a.src1 = static_cast<const uint4*>(v_tok);
     a.dst1 = static_cast<uint4*>(c->v);
     a.perm = d_perm;
+    a.T = T;
+    a.H = H;
+    a.W = W;
     a.block_valid = c->block_valid;
     a.d_err = d_err;
     a.N = n;
@@ -484,7 +526,7 @@ extern "C" bsa_status bsa_kv_pool_means(const bsa_kv_cache* c, int first, int co
 extern "C" bsa_status bsa_tokens_to_blocks(const void* x_tok, void* x_blk, int B, int Hh, int D,
                                            int T, int H, int W, const int32_t* d_perm,
                                            int32_t* d_err, void* stream) {
-  if (x_tok == nullptr || x_blk == nullptr || d_perm == nullptr) return BSA_ERR_INVALID_ARG;
+  if (x_tok == nullptr || x_blk == nullptr) return BSA_ERR_INVALID_ARG;
   bsa_status st = check_chunk(B, Hh, D, T, H, W);
   if (st != BSA_OK) return st;
   if (!aligned16(x_tok) || !aligned16(x_blk)) return BSA_ERR_INVALID_ARG;
@@ -493,6 +535,9 @@ extern "C" bsa_status bsa_tokens_to_blocks(const void* x_tok, void* x_blk, int B
   a.src0 = static_cast<const uint4*>(x_tok);
   a.dst0 = static_cast<uint4*>(x_blk);
   a.perm = d_perm;
+  a.T = T;
+  a.H = H;
+  a.W = W;
   a.d_err = d_err;
   a.N = n;
   a.nb = (n + kBlk - 1) / kBlk;
@@ -507,7 +552,7 @@ extern "C" bsa_status bsa_tokens_to_blocks_mean(const void* x_tok, void* x_blk, 
                                                 int B, int Hh, int D, int T, int H, int W,
                                                 const int32_t* d_perm, int32_t* d_err,
                                                 void* stream) {
-  if (x_tok == nullptr || x_blk == nullptr || x_mean == nullptr || d_perm == nullptr)
+  if (x_tok == nullptr || x_blk == nullptr || x_mean == nullptr)
     return BSA_ERR_INVALID_ARG;
   bsa_status st = check_chunk(B, Hh, D, T, H, W);
   if (st != BSA_OK) return st;
@@ -519,6 +564,9 @@ extern "C" bsa_status bsa_tokens_to_blocks_mean(const void* x_tok, void* x_blk, 
   a.x_blk = static_cast<uint4*>(x_blk);
   a.x_mean = x_mean;
   a.perm = d_perm;
+  a.T = T;
+  a.H = H;
+  a.W = W;
   a.d_err = d_err;
   a.N = n;
   a.Hh = Hh;
@@ -532,7 +580,7 @@ extern "C" bsa_status bsa_tokens_to_blocks_mean(const void* x_tok, void* x_blk, 
 extern "C" bsa_status bsa_blocks_to_tokens(const void* x_blk, void* x_tok, int B, int Hh, int D,
                                            int T, int H, int W, const int32_t* d_perm,
                                            int32_t* d_err, void* stream) {
-  if (x_tok == nullptr || x_blk == nullptr || d_perm == nullptr) return BSA_ERR_INVALID_ARG;
+  if (x_tok == nullptr || x_blk == nullptr) return BSA_ERR_INVALID_ARG;
   bsa_status st = check_chunk(B, Hh, D, T, H, W);
   if (st != BSA_OK) return st;
   if (!aligned16(x_tok) || !aligned16(x_blk)) return BSA_ERR_INVALID_ARG;
@@ -541,6 +589,9 @@ extern "C" bsa_status bsa_blocks_to_tokens(const void* x_blk, void* x_tok, int B
   a.src0 = static_cast<const uint4*>(x_blk);
   a.dst0 = static_cast<uint4*>(x_tok);
   a.perm = d_perm;
+  a.T = T;
+  a.H = H;
+  a.W = W;
   a.d_err = d_err;
   a.N = n;
   a.nb = (n + kBlk - 1) / kBlk;

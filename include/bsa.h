@@ -126,7 +126,11 @@ bsa_status bsa_gilbert_perm(int T, int H, int W, int32_t *host_perm);
  *   k_tok, v_tok  device bf16 [B, T*H*W, Hh, D] (cache's B, Hh, D)
  *   d_perm        device int32 [T*H*W], the table from bsa_gilbert_perm
  *                 (any permutation of [0, T*H*W) is accepted; entries
- *                 outside that range raise BSA_DEV_BAD_PERM and are skipped)
+ *                 outside that range raise BSA_DEV_BAD_PERM and are
+ *                 skipped), or NULL: the kernels then locate every slot on
+ *                 the Gilbert curve of (T, H, W) themselves (the order
+ *                 bsa_gilbert_perm tabulates), with no table and nothing
+ *                 allocated.  The same for every call below taking d_perm.
  * Errors: BSA_ERR_INVALID_ARG, BSA_ERR_CAPACITY (n_blocks + nb > max_blocks,
  *         cache unchanged), BSA_ERR_UNSUPPORTED, BSA_ERR_CUDA.
  */
@@ -247,7 +251,8 @@ bsa_status bsa_attn(const void *q_blk, const bsa_kv_cache *cache, const int32_t 
 /*
  * bsa_attn with O and LSE written straight to raster token order (Velox,
  * Methodology Step 6, followed by the inverse of the query reordering):
- * row r of query block j is the token t with d_perm[t] = 128*j + r, so
+ * row r of query block j is the token t with d_perm[t] = 128*j + r (the
+ * Gilbert order of (T, H, W) when d_perm is NULL), so
  *   o_tok[b, t, h, :] = O of that row           device bf16 [B, T*H*W, Hh, D]
  *   lse_tok[b, t, h]  = LSE of that row          device fp32 [B, T*H*W, Hh]
  * and pad rows (slots no token maps to) are not written.  This saves the

@@ -276,3 +276,38 @@ def test_route_from_query_means_equals_route(key, chunk, pooled):
     bsa.raise_on_device_error(DEV)
     assert torch.equal(cnt2, cnt)
     assert torch.equal(idx2, idx)
+
+
+@pytest.mark.parametrize("grid,D", [((3, 5, 7), 64), ((2, 8, 16), 128), ((5, 30, 52), 64),
+                                    ((4, 39, 40), 128), ((2, 96, 101), 64)])
+def test_without_table_equals_with_table(grid, D):
+    # With no permutation table (d_perm NULL) every kernel locates its slots
+    # on the Gilbert curve itself; the results equal the table path bit for
+    # bit: reordering both ways, reordering with means, and the append
+    # (including, at 19392 tokens, the scatter path for large chunks).
+    T, H, W = grid
+    n = T * H * W
+    x = synth.random_bf16((2, n, 3, D), seed=11, device=DEV)
+    a = bsa.bsa_tokens_to_blocks(x, T, H, W)
+    b = bsa.bsa_tokens_to_blocks(x, T, H, W, table=False)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    ta = bsa.bsa_blocks_to_tokens(a, T, H, W)
+    tb = bsa.bsa_blocks_to_tokens(a, T, H, W, table=False)
+    assert torch.equal(ta.view(torch.int16), tb.view(torch.int16))
+    if n <= 16384:
+        am, mm = bsa.bsa_tokens_to_blocks_mean(x, T, H, W)
+        bm, nm = bsa.bsa_tokens_to_blocks_mean(x, T, H, W, table=False)
+        assert torch.equal(am.view(torch.int16), bm.view(torch.int16))
+        assert torch.equal(mm, nm)
+    nb = (n + 127) // 128
+    caches = []
+    for table in (True, False):
+        c = bsa.KVCache(2, 3, D, nb + 2, device=DEV, pooled_keys=True)
+        bsa.bsa_kv_append(c, x, x.flip(0).contiguous(), T, H, W, table=table)
+        caches.append(c)
+    bsa.raise_on_device_error(DEV)
+    c0, c1 = caches
+    assert torch.equal(c0.k.view(torch.int16), c1.k.view(torch.int16))
+    assert torch.equal(c0.v.view(torch.int16), c1.v.view(torch.int16))
+    assert torch.equal(c0.kmean, c1.kmean)
+    assert torch.equal(c0.block_valid, c1.block_valid)

@@ -249,6 +249,15 @@ def test_attn_tokens_equals_attn_then_reorder(key):
     perm = torch.from_numpy(bsa.bsa_gilbert_perm(T, H, W).astype(np.int64)).to(DEV)
     lse_ref = lse_blk[:, :, perm].permute(0, 2, 1)            # [B, N, Hh]
     assert torch.equal(lse_tok, lse_ref)
+    # Without a permutation table the kernel locates the rows' tokens on the
+    # Gilbert curve itself: the same output.
+    o2 = torch.full_like(o_tok, 7.0)
+    l2 = torch.full_like(lse_tok, 7.0)
+    bsa.bsa_attn_tokens(step.q_blk, step.cache, idx, cnt, T, H, W, q_valid=step.q_valid,
+                        o=o2, lse=l2, table=False)
+    bsa.raise_on_device_error(DEV)
+    assert torch.equal(o2.view(torch.int16), o_tok.view(torch.int16))
+    assert torch.equal(l2, lse_tok)
 
 
 def test_attn_tokens_against_the_oracle_config3():
