@@ -20,12 +20,15 @@ namespace bsa {
 // lane's vector of a row below `valid`, and `seen(row, x)` is called once for
 // every row 0..127 with the vector that was added (zeros at and past
 // `valid`), so a caller can move the rows while it pools them.
-template <int VPR, class Load, class Seen>
+// NB rows per lane are loaded before any is added (more loads in flight for
+// a larger NB); the rows are still added in the same order, so the sums do
+// not depend on NB.
+template <int VPR, class Load, class Seen, int NB = 16>
 __device__ __forceinline__ void warp_colsum_rows(Load load, Seen seen, int valid, int g,
                                                  float (&acc)[8]) {
   constexpr int RPI = 32 / VPR;
-  constexpr int NB = 16;
   constexpr int kBatches = kBlk / (RPI * NB);
+  static_assert(kBlk % (RPI * NB) == 0, "batches must cover the 128 rows exactly");
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll

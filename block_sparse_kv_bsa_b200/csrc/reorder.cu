@@ -400,7 +400,9 @@ gather_mean_kernel(GatherMeanArgs a) {
   };
   auto store = [&](int row, uint4 x) { st_v4(dst + row * VPR, x); };
   float acc[8];
-  warp_colsum_rows<VPR>(load, store, valid, g, acc);
+  // 32 rows in flight per lane: this kernel has one warp per (block, head),
+  // only 8 warps per SM.
+  warp_colsum_rows<VPR, decltype(load), decltype(store), 32>(load, store, valid, g, acc);
   if (g == 0) {
     float4* out = reinterpret_cast<float4*>(a.x_mean + blk * D + c * 8);
     const float inv = static_cast<float>(valid);
