@@ -7,12 +7,16 @@
 // added outside the budget).  The additive form used here is
 //   s'[j, n] = sm_scale * <qmean_j, kmean_n> + lambda * min(g[j, n] / g_ref, 1).
 //
-// Three launches, all stream-ordered, no host round trip:
-//   1. pool_q      mean of each query block's valid rows -> qm (workspace)
-//   2. pool_score  stream every history K block once (one warp per block),
-//                  pool it in registers, and score it against all query means
-//                  of its head at once; only the model scores go to the
-//                  workspace (the K stream is the HBM-bound part of routing)
+// Up to three launches, all stream-ordered, no host round trip:
+//   1. pool_q      mean of each query block's valid rows -> qm (workspace);
+//                  skipped when the caller passes the query means
+//   2. scores      from the pooled-key cache (the key means written at
+//                  append): the product of query means and key means, on the
+//                  tensor core for up to 64 query blocks (score_tc.cu), else
+//                  on the FMA pipes; without the cache, pool_score streams
+//                  every history K block once (one warp per block), pools it
+//                  in registers and scores it against all query means of its
+//                  head (the HBM-bound form of routing)
 //   3. topk        add the prior (g read row by row), then an exact top-K per
 //                  row by radix select on order-preserving score keys held in
 //                  shared memory, ties to the lower index, emitted in ascending
@@ -42,11 +46,12 @@ struct RouteArgs {
   const float* g;          // [B, n_own, n_hist] or null
   const float* kmean;      // [B, Hh, max_blocks, D] pooled keys, or null
   float* qm;               // [B, Hh, n_own, D]
-  float* s;                // [B, Hh, n_own, n_hist]
+  float* s;                // [B, Hh, n_own, s_ld]: row (b, h, j) holds its n_hist scores
   int32_t* idx;
   int32_t* cnt;
   int32_t* d_err;
   int B, Hh, n_own, n_hist, own_first, max_blocks, top_k, max_sel;
+  int s_ld;                // score row stride: n_hist rounded up to 32 (128-byte rows)
   float sm_scale, lam, g_ref;
 };
 
@@ -146,7 +151,7 @@ pool_score_kernel(RouteArgs a) {
 #pragma unroll
         for (int t = 1; t < 4; ++t) dv = c == t ? d[t] : dv;
         const int j = j0 + c * RPI;
-        if (j < a.n_own) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * dv;
+        if (j < a.n_own) a.s[(bh * a.n_own + j) * a.s_ld + n] = a.sm_scale * dv;
       }
     }
   };
@@ -220,7 +225,7 @@ __device__ __forceinline__ void score_means_tile(const RouteArgs& a, const float
       const int n = n0 + tk + 16 * y;
       float even, odd;
       f2_unpack(acc[x][y], even, odd);
-      if (n < a.n_hist) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * (even + odd);
+      if (n < a.n_hist) a.s[(bh * a.n_own + j) * a.s_ld + n] = a.sm_scale * (even + odd);
     }
   }
 }
@@ -286,132 +291,12 @@ score_means_kernel(RouteArgs a) {
   }
 }
 
-// Pipelined form of the same product, for up to 64 query blocks: a
-// persistent grid (one CTA of 256 threads per SM) walks the (head, 128
-// history blocks) tiles blockIdx.x, blockIdx.x + gridDim.x, ...  Each tile's
-// query means and key means are copied to shared memory by cp.async into
-// one of two stages, so the next tile's copy is in flight while the current
-// tile is scored (the one-shot kernel above waits for its copies with the
-// SM idle, once per wave).  Thread (warp w, lane l) scores query blocks
-// w + 8x against history blocks l + 32y (y < 4): the query rows are warp
-// broadcasts and the 32 key rows of a load sit in distinct bank groups.
-constexpr int kPipeTileN = 128;
-constexpr int kPipeThreads = 256;
-constexpr int kPipeMaxOwn = 64;
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
-  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gmem),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_prev() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
-}
-
-template <int D, int X>
-__device__ __forceinline__ void score_pipe_tile(const RouteArgs& a, const float* qs,
-                                                const float* ks, long long bh, int n0) {
-  constexpr int P = D + 4;
-  const int tk = threadIdx.x % 32, tq = threadIdx.x / 32;
-  uint64_t acc[X][4];
-#pragma unroll
-  for (int x = 0; x < X; ++x)
-#pragma unroll
-    for (int y = 0; y < 4; ++y) acc[x][y] = 0ull;   // {+0.f, +0.f}
-#pragma unroll 2
-  for (int d = 0; d < D; d += 4) {
-    ulonglong2 q[X], k[4];
-#pragma unroll
-    for (int x = 0; x < X; ++x)
-      q[x] = *reinterpret_cast<const ulonglong2*>(qs + (tq + 8 * x) * P + d);
-#pragma unroll
-    for (int y = 0; y < 4; ++y)
-      k[y] = *reinterpret_cast<const ulonglong2*>(ks + (tk + 32 * y) * P + d);
-    // All first halves, then all second halves: 4X independent FMAs
-    // between the two that update one accumulator.
-#pragma unroll
-    for (int x = 0; x < X; ++x)
-#pragma unroll
-      for (int y = 0; y < 4; ++y) acc[x][y] = f2_fma(q[x].x, k[y].x, acc[x][y]);
-#pragma unroll
-    for (int x = 0; x < X; ++x)
-#pragma unroll
-      for (int y = 0; y < 4; ++y) acc[x][y] = f2_fma(q[x].y, k[y].y, acc[x][y]);
-  }
-#pragma unroll
-  for (int x = 0; x < X; ++x) {
-    const int j = tq + 8 * x;
-    if (j >= a.n_own) continue;
-#pragma unroll
-    for (int y = 0; y < 4; ++y) {
-      const int n = n0 + tk + 32 * y;
-      float even, odd;
-      f2_unpack(acc[x][y], even, odd);
-      if (n < a.n_hist) a.s[(bh * a.n_own + j) * a.n_hist + n] = a.sm_scale * (even + odd);
-    }
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(kPipeThreads, 1) score_means_pipe_kernel(RouteArgs a) {
-  pdl_wait();     // global memory only after the predecessor grid completed
-  pdl_trigger();
-  constexpr int P = D + 4;
-  constexpr int R4 = D / 4;                      // 16-byte pieces per row
-  extern __shared__ __align__(16) float sm[];
-  const int nq8 = (a.n_own + 7) & ~7;            // query rows read by the product
-  const int stage = (nq8 + kPipeTileN) * P;      // floats per stage
-  const int per_head = (a.n_hist + kPipeTileN - 1) / kPipeTileN;
-  const int n_tiles = a.B * a.Hh * per_head;
-  auto copy_tile = [&](int tile, int st) {
-    const long long bh = tile / per_head;        // b * Hh + h
-    const int n0 = (tile % per_head) * kPipeTileN;
-    float* qs = sm + st * stage;
-    float* ks = qs + nq8 * P;
-    for (int i = threadIdx.x; i < (nq8 + kPipeTileN) * R4; i += kPipeThreads) {
-      const int r = i / R4, c4 = i % R4;
-      if (r < nq8) {
-        const bool v = r < a.n_own;              // rows past n_own are zero-filled
-        cp_async16(qs + r * P + c4 * 4, v ? a.qm + (bh * a.n_own + r) * D + c4 * 4 : a.qm, v);
-      } else {
-        const int rk = r - nq8;
-        const bool v = n0 + rk < a.n_hist;
-        cp_async16(ks + rk * P + c4 * 4,
-                   v ? a.kmean + (bh * a.max_blocks + n0 + rk) * D + c4 * 4 : a.kmean, v);
-      }
-    }
-  };
-  int tile = blockIdx.x;
-  if (tile >= n_tiles) return;
-  copy_tile(tile, 0);
-  cp_async_commit();
-  const int groups = nq8 / 8;
-  for (int k = 0; tile < n_tiles; ++k, tile += gridDim.x) {
-    // The copy into the other stage: that stage was last read in step k-1,
-    // which every thread finished before the barrier ending step k-1.
-    if (tile + static_cast<int>(gridDim.x) < n_tiles) copy_tile(tile + gridDim.x, (k + 1) & 1);
-    cp_async_commit();                           // (an empty group at the end)
-    cp_async_wait_prev();                        // this thread's copies of tile
-    __syncthreads();                             // ... and everyone's
-    const float* qs = sm + (k & 1) * stage;
-    const float* ks = qs + nq8 * P;
-    const long long bh = tile / per_head;
-    const int n0 = (tile % per_head) * kPipeTileN;
-    switch (groups) {
-      case 1: score_pipe_tile<D, 1>(a, qs, ks, bh, n0); break;
-      case 2: score_pipe_tile<D, 2>(a, qs, ks, bh, n0); break;
-      case 3: score_pipe_tile<D, 3>(a, qs, ks, bh, n0); break;
-      case 4: score_pipe_tile<D, 4>(a, qs, ks, bh, n0); break;
-      case 5: score_pipe_tile<D, 5>(a, qs, ks, bh, n0); break;
-      case 6: score_pipe_tile<D, 6>(a, qs, ks, bh, n0); break;
-      case 7: score_pipe_tile<D, 7>(a, qs, ks, bh, n0); break;
-      default: score_pipe_tile<D, 8>(a, qs, ks, bh, n0); break;
-    }
-    __syncthreads();                             // stage k & 1 is copied into at step k + 1
-  }
-}
+// For up to 64 query blocks the same product runs on the tensor core
+// (score_tc.cu: three tf32 passes over hi/lo splits of both means).
+bool score_means_tc_fits(int n_own, int D);
+bsa_status launch_score_means_tc(const float* qm, const float* kmean, float* s, int s_ld, int BH,
+                                 int n_own, int n_hist, int max_blocks, int D, float sm_scale,
+                                 int sms, int32_t* d_err, cudaStream_t st);
 
 // Streaming multiprocessors of the current device (cached per device).
 static int device_sms() {
@@ -478,7 +363,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(RouteArgs a) {
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const long long row = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
   int32_t* out = a.idx + row * a.max_sel;
-  const float* sr = a.s + row * a.n_hist;
+  const float* sr = a.s + row * a.s_ld;
   const float* gr = a.g != nullptr ? a.g + (static_cast<long long>(b) * a.n_own + j) * a.n_hist
                                    : nullptr;
   const int K = a.top_k < a.n_hist ? a.top_k : a.n_hist;
@@ -652,7 +537,7 @@ __global__ void __launch_bounds__(kTopkRowThreads, KPL <= 18 ? 8 : 6) topk_row_k
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const long long row = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
   int32_t* out = a.idx + row * a.max_sel;
-  const float* sr = a.s + row * a.n_hist;
+  const float* sr = a.s + row * a.s_ld;
   const float* gr = a.g != nullptr ? a.g + (static_cast<long long>(b) * a.n_own + j) * a.n_hist
                                    : nullptr;
   const int nh = a.n_hist;
@@ -823,7 +708,7 @@ __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a,
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const long long row = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
   int32_t* out = a.idx + row * a.max_sel;
-  const float* sr = a.s + row * nh;
+  const float* sr = a.s + row * a.s_ld;
   const float* gr = a.g != nullptr ? a.g + (static_cast<long long>(b) * a.n_own + j) * nh : nullptr;
   const bool covered = v.coverage != nullptr && v.coverage[b * a.n_own + j] >= v.eta_cov;
   const int p0 = min(max(v.prev_first, 0), nh);
@@ -1023,7 +908,7 @@ static void route_ws_layout(int B, int Hh, int D, int n_own, int n_hist, size_t*
                             size_t* s_bytes) {
   *qm_bytes = align256(sizeof(float) * static_cast<size_t>(B) * Hh * n_own * D);
   *s_bytes = align256(sizeof(float) * static_cast<size_t>(B) * Hh * n_own *
-                      static_cast<size_t>(n_hist > 0 ? n_hist : 0));
+                      static_cast<size_t>(n_hist > 0 ? (n_hist + 31) & ~31 : 0));
 }
 
 }  // namespace bsa
@@ -1098,6 +983,7 @@ static bsa_status route_scores(const void* q_blk, const float* q_mean, const bsa
   a.own_first = own_first;
   a.max_blocks = c->max_blocks;
   a.max_sel = max_sel;
+  a.s_ld = (n_hist + 31) & ~31;
   a.sm_scale = sm_scale;
   a.lam = lambda;
   a.g_ref = g_ref;
@@ -1106,26 +992,14 @@ static bsa_status route_scores(const void* q_blk, const float* q_mean, const bsa
   const int per_cta = kScoreWarps * kScoreBlocksPerWarp;
   dim3 sgrid((n_hist + per_cta - 1) / per_cta, c->Hh, c->B);
   dim3 mgrid((n_hist + kMeanTileN - 1) / kMeanTileN, c->Hh, c->B);
-  // Pipelined product: up to 64 query blocks, one CTA per SM (at most one
-  // per tile); 0 selects the one-shot kernel.
-  const int nq8 = (n_own + 7) & ~7;
-  const size_t pipe_smem = 2 * sizeof(float) * static_cast<size_t>(nq8 + kPipeTileN) * (c->D + 4);
-  int pipe_grid = 0;
-  if (n_own <= kPipeMaxOwn && n_hist > 0) {
-    const long long tiles = static_cast<long long>(c->B) * c->Hh *
-                            ((n_hist + kPipeTileN - 1) / kPipeTileN);
-    pipe_grid = static_cast<int>(std::min<long long>(tiles, device_sms()));
-  }
+  const bool tc = n_hist > 0 && c->kmean != nullptr && score_means_tc_fits(n_own, c->D) &&
+                  static_cast<long long>(c->B) * c->Hh <= (1 << 24);
   if (c->D == 128) {
     if (q_mean == nullptr)
       BSA_TRY(launch_pdl(pool_q_kernel<16>, pgrid, dim3(kPoolQWarps * 32), 0, s, a));
-    if (n_hist > 0 && c->kmean != nullptr && pipe_grid > 0) {
-      if (cudaFuncSetAttribute(score_means_pipe_kernel<128>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(pipe_smem)) != cudaSuccess)
-        return BSA_ERR_CUDA;
-      BSA_TRY(launch_pdl(score_means_pipe_kernel<128>, dim3(pipe_grid), dim3(kPipeThreads),
-                         pipe_smem, s, a));
+    if (tc) {
+      BSA_TRY(launch_score_means_tc(a.qm, c->kmean, a.s, a.s_ld, c->B * c->Hh, n_own, n_hist,
+                                    c->max_blocks, c->D, sm_scale, device_sms(), d_err, s));
     } else if (n_hist > 0 && c->kmean != nullptr) {
       if (cudaFuncSetAttribute(score_means_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(mean_smem)) != cudaSuccess)
@@ -1140,13 +1014,9 @@ static bsa_status route_scores(const void* q_blk, const float* q_mean, const bsa
   } else {
     if (q_mean == nullptr)
       BSA_TRY(launch_pdl(pool_q_kernel<8>, pgrid, dim3(kPoolQWarps * 32), 0, s, a));
-    if (n_hist > 0 && c->kmean != nullptr && pipe_grid > 0) {
-      if (cudaFuncSetAttribute(score_means_pipe_kernel<64>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(pipe_smem)) != cudaSuccess)
-        return BSA_ERR_CUDA;
-      BSA_TRY(launch_pdl(score_means_pipe_kernel<64>, dim3(pipe_grid), dim3(kPipeThreads),
-                         pipe_smem, s, a));
+    if (tc) {
+      BSA_TRY(launch_score_means_tc(a.qm, c->kmean, a.s, a.s_ld, c->B * c->Hh, n_own, n_hist,
+                                    c->max_blocks, c->D, sm_scale, device_sms(), d_err, s));
     } else if (n_hist > 0 && c->kmean != nullptr) {
       if (cudaFuncSetAttribute(score_means_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(mean_smem)) != cudaSuccess)

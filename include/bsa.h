@@ -196,7 +196,10 @@ bsa_status bsa_route_workspace_size(int B, int Hh, int D, int n_q_blocks, int n_
  *   route = the top_k largest s over the history (ties to the lower block
  *           index; every history block when top_k >= n_hist), sorted
  *           ascending, followed by the own chunk [own_first, own_first+n_own).
- * Arithmetic is fp32 with a fixed reduction order.
+ * Arithmetic is fp32 with a fixed reduction order; with the pooled-key
+ * cache and at most 64 query blocks, <qm, km> runs on the tensor core as
+ * three tf32 products of hi/lo splits of both means (about fp32's
+ * precision, fixed order), so results are deterministic either way.
  *   q_blk      device bf16 [B, Hh, n_own*128, D] (block order)
  *   q_valid    device int32 [n_own] valid rows per query block, or NULL to
  *              use cache->block_valid[own_first + j]

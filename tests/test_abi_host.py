@@ -72,7 +72,7 @@ def test_gilbert_perm_rejects_bad_args():
 def test_workspace_size_formula():
     n = bsa.bsa_route_workspace_size(1, 24, 128, 49, 2303)
     qm = -(-4 * 24 * 49 * 128 // 256) * 256
-    s = -(-4 * 24 * 49 * 2303 // 256) * 256
+    s = -(-4 * 24 * 49 * 2304 // 256) * 256     # score rows padded to 32 floats
     assert n == qm + s
     with pytest.raises(bsa.BsaError):
         bsa.bsa_route_workspace_size(1, 24, 96, 49, 10)
