@@ -61,6 +61,7 @@ constexpr int kTcTmaWarp = 8;
 constexpr int kTcMmaWarp = 9;
 constexpr int kTcStages = 4;          // key slices in flight (shared and tensor memory)
 constexpr uint32_t kTcColA = 128;     // first column of the key ring
+constexpr int kTcTrStride = 36;       // floats per query row of an epilogue transpose
 constexpr long long kTcWaitLimit = 1LL << 31;  // SM clocks (about a second)
 
 enum : int {
@@ -85,7 +86,8 @@ struct TcLayout {
   static constexpr int kQHi = 0;
   static constexpr int kQLo = kQHi + kQBytes;
   static constexpr int kK = kQLo + kQBytes;                // stage s at kK + s * kKSlice
-  static constexpr int kBars = kK + kTcStages * kKSlice;
+  static constexpr int kTr = kK + kTcStages * kKSlice;     // epilogue transposes
+  static constexpr int kBars = kTr + 4 * kTcMaxOwn * kTcTrStride * 4;
   static constexpr int kMisc = kBars + TB_COUNT * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;             // 1024-byte alignment slack
@@ -335,11 +337,19 @@ score_means_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
   } else if (warp < 8) {
     // ---------------- epilogue ----------------
     // Thread (warp w, lane l) holds history block n0 + 32 (w - 4) + l: its
-    // scores against query blocks 0..63 are its accumulator row.
+    // scores against query blocks 0..63 are its accumulator row.  Each warp
+    // transposes its 32 x 64 scores through shared memory ([query][key],
+    // 36 floats per query row: conflict-free both ways) and writes every
+    // query row's 32 scores as 8 16-byte pieces, four rows per store.
+    // Score rows are 128-byte aligned (s_ld a multiple of 32), so a warp's
+    // 32 blocks lie in one row whenever the first does; scores of blocks
+    // past n_hist land in the row's padding, which nothing reads.
     if (nt > 0) {
       const int wq = warp - 4;               // TMEM lanes 32*wq .. 32*wq + 31
       const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+      float* tr = reinterpret_cast<float*>(sm + L::kTr) + wq * kTcMaxOwn * kTcTrStride;
       float* row0 = a.s + bh * a.q_rows_per_head * a.s_ld;
+      const int rows = a.n_own;
       bool ok = true;
       for (int t = 0; t < nt; ++t) {
         const int acc = t & 1;
@@ -347,8 +357,6 @@ score_means_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                        s_abort, kTcWaitLimit));
         if (!ok) break;
         tc_fence_after();
-        const int n = (t_first + t) * kTcKeys + wq * 32 + lane;
-        float* dst = row0 + n;
 #pragma unroll
         for (int h = 0; h < kTcMaxOwn; h += 32) {
           float v[32];
@@ -357,13 +365,20 @@ score_means_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
             tc_fence_before();
             mbar_arrive(&bars[TB_ACC_EMPTY + acc]);
           }
-          if (n < a.n_hist) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (h + e < a.n_own)
-                dst[(h + e) * a.s_ld] = a.sm_scale * v[e];
+          for (int e = 0; e < 32; ++e) tr[(h + e) * kTcTrStride + lane] = a.sm_scale * v[e];
+        }
+        __syncwarp();
+        const int n0 = (t_first + t) * kTcKeys + wq * 32;
+        if (n0 < a.s_ld) {
+          float* dst = row0 + n0 + (lane & 7) * 4;
+          for (int i = lane; i < rows * 8; i += 32) {
+            const int j = i >> 3;
+            const float4 x = *reinterpret_cast<const float4*>(tr + j * kTcTrStride + (lane & 7) * 4);
+            *reinterpret_cast<float4*>(dst + static_cast<long long>(j) * a.s_ld) = x;
           }
         }
+        __syncwarp();
       }
       if (!ok && lane == 0) {
         report(a.d_err, BSA_DEV_WAIT_TIMEOUT);
