@@ -512,6 +512,46 @@ __device__ void radix_threshold(const uint32_t* keys, int n, int K, int* hist, u
   *need_eq = remaining;
 }
 
+// Warp-wide search for the m-th largest of the keys the lanes hold (v, 0 =
+// no key): the largest t with #{v >= t} >= m, bit by bit from the top.  The
+// caller passes lo <= answer <= hi; the bits above the highest bit where lo
+// and hi differ are the answer's too, so the search starts below them.  It
+// stops early once a count is exactly m (*exact: #{v >= t} == m).
+template <int NV>
+__device__ __forceinline__ uint32_t warp_kth_key(const uint32_t (&v)[NV], int m, uint32_t lo,
+                                                 uint32_t hi, bool* exact) {
+  const int top = lo == hi ? -1 : 31 - __clz(lo ^ hi);
+  uint32_t thr = top < 0 ? lo : lo & ~((2u << top) - 1u);
+  bool ex = false;
+#pragma unroll 1
+  for (int bit = top; bit >= 0; --bit) {
+    const uint32_t cand = thr | (1u << bit);
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) c += v[i] >= cand;
+    const int tot = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
+    if (tot >= m) {
+      thr = cand;
+      if (tot == m) {
+        ex = true;
+        break;
+      }
+    }
+  }
+  if (!ex) {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) c += v[i] >= thr;
+    ex = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c))) == m;
+  }
+  *exact = ex;
+  return thr;
+}
+
+// Candidates of the pivot pass of topk_row_kernel (shared memory, in block
+// index order).
+constexpr int kTopkCandCap = 512;
+
 // Top-K of a row of at most 128 * KPL history blocks: one CTA of 128
 // threads per row, thread t holding the keys of blocks c * 128 + t (c < KPL)
 // in registers.
@@ -523,6 +563,15 @@ __device__ void radix_threshold(const uint32_t* keys, int n, int K, int* hist, u
 //      keys equal to t.
 //   3. Write the selected blocks in ascending order: one ballot per
 //      32-block group, the group totals in shared memory, one barrier.
+// For a long row and a small K a pivot pass runs first and usually settles
+// the row with far fewer comparisons: warp 0 takes the keys of every 8th
+// block as a sample and finds a pivot P, the sample's m-th largest key, m
+// chosen so that about 2K keys of the row lie at or above P; one block-wide
+// count checks that between K and kTopkCandCap keys do (then P <= the K-th
+// largest key, so every key of the top K is a candidate), the candidates are
+// compacted in block order into shared memory, and warp 0 selects the top K
+// among them as in 1-3 (ties to the lower block).  Otherwise 1-3 run on the
+// whole row.
 // The selected set and its order are those of topk_kernel.
 constexpr int kTopkRowThreads = 128;
 
@@ -533,6 +582,11 @@ __global__ void __launch_bounds__(kTopkRowThreads, KPL <= 18 ? 8 : 6) topk_row_k
   constexpr int kWarps = kTopkRowThreads / 32;
   __shared__ unsigned part[2][kWarps];
   __shared__ unsigned grp[2][KPL][kWarps];     // per-(group, warp) ballot counts: eq, sel
+  constexpr int kSamp = (16 * KPL + 31) / 32;   // sample keys per lane of warp 0
+  __shared__ uint32_t samp[32 * kSamp];
+  __shared__ uint32_t ckey[kTopkCandCap];
+  __shared__ uint16_t cidx[kTopkCandCap];
+  __shared__ uint32_t s_pivot;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const long long row = (static_cast<long long>(b) * a.Hh + h) * a.n_own + j;
@@ -578,59 +632,159 @@ __global__ void __launch_bounds__(kTopkRowThreads, KPL <= 18 ? 8 : 6) topk_row_k
     // part[] alternates between two buffers: a warp can only overwrite a
     // buffer after the next barrier, which every warp reaches only after
     // reading it.
-    uint32_t thr = 0;
-    bool exact = false;
     int parity = 0;
-#pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = thr | (1u << bit);
-      const int cnt = block_count(cand, false, parity);
-      parity ^= 1;
-      if (cnt >= K) {
-        thr = cand;
-        if (cnt == K) { exact = true; break; }
-      }
-    }
-    // exact: take key >= thr (K of them); else key > thr plus the first
-    // need_eq keys == thr.
-    const int need_eq = exact ? 0 : K - block_count(thr, true, parity);
     const unsigned below = (1u << lane) - 1u;
-    bool eq[KPL];
+    bool done = false;
+    if (K <= kTopkCandCap / 4 && nh >= 6 * K) {
+      // ---- pivot pass ----
+      if ((t & 7) == 0) {
 #pragma unroll
-    for (int c = 0; c < KPL; ++c) {
-      eq[c] = !exact && c * kTopkRowThreads + t < nh && key[c] == thr;
-      const unsigned m = __ballot_sync(0xffffffffu, eq[c]);
-      if (lane == 0) grp[0][c][warp] = __popc(m);
-    }
-    __syncthreads();
-    bool sel[KPL];
-    int before = 0;   // equal keys in earlier groups
-#pragma unroll
-    for (int c = 0; c < KPL; ++c) {
-      const int n = c * kTopkRowThreads + t;
-      int rank = before + __popc(__ballot_sync(0xffffffffu, eq[c]) & below);
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const int e = static_cast<int>(grp[0][c][w]);
-        rank += w < warp ? e : 0;
-        before += e;
+        for (int c = 0; c < KPL; ++c) samp[(t >> 3) * KPL + c] = key[c];
       }
-      sel[c] = n < nh && (exact ? key[c] >= thr : (key[c] > thr || (eq[c] && rank < need_eq)));
-      const unsigned m = __ballot_sync(0xffffffffu, sel[c]);
-      if (lane == 0) grp[1][c][warp] = __popc(m);
-    }
-    __syncthreads();
-    int pos = 0;      // selected blocks in earlier groups
+      for (int i = 16 * KPL + t; i < 32 * kSamp; i += kTopkRowThreads) samp[i] = 0u;
+      __syncthreads();
+      if (warp == 0) {
+        uint32_t v[kSamp];
+        int nv = 0;
+        uint32_t lo = 0xffffffffu, hi = 0u;
 #pragma unroll
-    for (int c = 0; c < KPL; ++c) {
-      int at = pos + __popc(__ballot_sync(0xffffffffu, sel[c]) & below);
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const int e = static_cast<int>(grp[1][c][w]);
-        at += w < warp ? e : 0;
-        pos += e;
+        for (int i = 0; i < kSamp; ++i) {
+          v[i] = samp[i * 32 + lane];
+          nv += v[i] != 0u;
+          lo = v[i] != 0u ? min(lo, v[i]) : lo;
+          hi = max(hi, v[i]);
+        }
+        nv = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(nv)));
+        lo = __reduce_min_sync(0xffffffffu, lo);
+        hi = __reduce_max_sync(0xffffffffu, hi);
+        // About 2K keys of the row at or above the sample's m-th largest.
+        int m = static_cast<int>((2LL * K * nv + nh - 1) / nh);
+        m = max(1, min(m, nv));
+        bool ex;
+        const uint32_t p = warp_kth_key(v, m, lo, hi, &ex);
+        if (lane == 0) s_pivot = p;
       }
-      if (sel[c]) out[at] = c * kTopkRowThreads + t;
+      __syncthreads();
+      const uint32_t piv = s_pivot;
+      const int n_cand = block_count(piv, false, parity);
+      parity ^= 1;
+      if (n_cand >= K && n_cand <= kTopkCandCap) {
+        // Candidates in block order: group c, then thread.
+#pragma unroll
+        for (int c = 0; c < KPL; ++c) {
+          const unsigned m = __ballot_sync(0xffffffffu, key[c] >= piv);
+          if (lane == 0) grp[0][c][warp] = __popc(m);
+        }
+        __syncthreads();
+        int pos = 0;
+#pragma unroll
+        for (int c = 0; c < KPL; ++c) {
+          const bool cand = key[c] >= piv;
+          int at = pos + __popc(__ballot_sync(0xffffffffu, cand) & below);
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) {
+            const int e = static_cast<int>(grp[0][c][w]);
+            at += w < warp ? e : 0;
+            pos += e;
+          }
+          if (cand) {
+            ckey[at] = key[c];
+            cidx[at] = static_cast<uint16_t>(c * kTopkRowThreads + t);
+          }
+        }
+        __syncthreads();
+        if (warp == 0) {
+          constexpr int kC = kTopkCandCap / 32;
+          uint32_t v[kC];
+          uint32_t hi = 0u;
+#pragma unroll
+          for (int i = 0; i < kC; ++i) {
+            v[i] = i * 32 + lane < n_cand ? ckey[i * 32 + lane] : 0u;
+            hi = max(hi, v[i]);
+          }
+          hi = __reduce_max_sync(0xffffffffu, hi);
+          bool ex;
+          const uint32_t th = warp_kth_key(v, K, piv, hi, &ex);
+          int need_eq = 0;
+          if (!ex) {
+            int gt = 0;
+#pragma unroll
+            for (int i = 0; i < kC; ++i) gt += v[i] > th;
+            need_eq = K - static_cast<int>(__reduce_add_sync(0xffffffffu,
+                                                             static_cast<unsigned>(gt)));
+          }
+          int at = 0, eq_before = 0;
+#pragma unroll
+          for (int i = 0; i < kC; ++i) {
+            if (i * 32 >= n_cand) break;
+            const bool valid = i * 32 + lane < n_cand;
+            const bool is_eq = valid && v[i] == th;
+            const unsigned em = __ballot_sync(0xffffffffu, is_eq);
+            const int r_eq = eq_before + __popc(em & below);
+            const bool sel =
+                valid && (ex ? v[i] >= th : (v[i] > th || (is_eq && r_eq < need_eq)));
+            const unsigned sm = __ballot_sync(0xffffffffu, sel);
+            if (sel) out[at + __popc(sm & below)] = cidx[i * 32 + lane];
+            at += __popc(sm);
+            eq_before += __popc(em);
+          }
+        }
+        done = true;
+      }
+    }
+    if (!done) {
+      uint32_t thr = 0;
+      bool exact = false;
+#pragma unroll 1
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = thr | (1u << bit);
+        const int cnt = block_count(cand, false, parity);
+        parity ^= 1;
+        if (cnt >= K) {
+          thr = cand;
+          if (cnt == K) { exact = true; break; }
+        }
+      }
+      // exact: take key >= thr (K of them); else key > thr plus the first
+      // need_eq keys == thr.
+      const int need_eq = exact ? 0 : K - block_count(thr, true, parity);
+      bool eq[KPL];
+#pragma unroll
+      for (int c = 0; c < KPL; ++c) {
+        eq[c] = !exact && c * kTopkRowThreads + t < nh && key[c] == thr;
+        const unsigned m = __ballot_sync(0xffffffffu, eq[c]);
+        if (lane == 0) grp[0][c][warp] = __popc(m);
+      }
+      __syncthreads();
+      bool sel[KPL];
+      int before = 0;   // equal keys in earlier groups
+#pragma unroll
+      for (int c = 0; c < KPL; ++c) {
+        const int n = c * kTopkRowThreads + t;
+        int rank = before + __popc(__ballot_sync(0xffffffffu, eq[c]) & below);
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          const int e = static_cast<int>(grp[0][c][w]);
+          rank += w < warp ? e : 0;
+          before += e;
+        }
+        sel[c] = n < nh && (exact ? key[c] >= thr : (key[c] > thr || (eq[c] && rank < need_eq)));
+        const unsigned m = __ballot_sync(0xffffffffu, sel[c]);
+        if (lane == 0) grp[1][c][warp] = __popc(m);
+      }
+      __syncthreads();
+      int pos = 0;      // selected blocks in earlier groups
+#pragma unroll
+      for (int c = 0; c < KPL; ++c) {
+        int at = pos + __popc(__ballot_sync(0xffffffffu, sel[c]) & below);
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          const int e = static_cast<int>(grp[1][c][w]);
+          at += w < warp ? e : 0;
+          pos += e;
+        }
+        if (sel[c]) out[at] = c * kTopkRowThreads + t;
+      }
     }
   }
   for (int i = t; i < a.n_own; i += kTopkRowThreads) out[K + i] = a.own_first + i;

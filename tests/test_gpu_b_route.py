@@ -92,6 +92,38 @@ def test_route_all_equal_scores_take_lowest_indices():
     assert torch.all(idx[..., :K] == exp)
 
 
+@pytest.mark.parametrize("n_top", [100, 1000])
+def test_route_exact_ties_at_the_cut_take_lowest_indices(n_top):
+    # Q = 0 and a prior of three levels: every fused score is the prior
+    # alone, with exact ties.  n_top history blocks per row at the top level
+    # (K = 64 of them are taken): 100 leaves few candidates at the cut (the
+    # row top-K's pivot pass settles it), 1000 too many for that pass (the
+    # search over the whole row does).  Either way the route is the top K
+    # with ties to the lower block, exactly as the oracle's.
+    import oracle
+    w = synth.CONFIGS[4]
+    step = hx.build_step(w, DEV, chunk=48)
+    step.q_blk.zero_()
+    nh, J = step.n_hist, step.n_own
+    rng = np.random.default_rng(11 + n_top)
+    g = np.zeros((w.B, J, nh), np.float32)
+    for b in range(w.B):
+        for j in range(J):
+            p = rng.permutation(nh)
+            g[b, j, p[:n_top]] = w.g_ref
+            g[b, j, p[n_top:n_top + 300]] = 0.5 * w.g_ref
+    step.g = torch.from_numpy(g).to(DEV)
+    idx, cnt = hx.route(step)
+    bsa.raise_on_device_error(DEV)
+    fused = oracle.fuse_prior(np.zeros((w.B, 1, J, nh)), g.astype(np.float64), w.lam, w.g_ref)
+    idx_h = idx.cpu().numpy()
+    for b in range(w.B):
+        for j in range(J):
+            want = oracle.top_k_with_own(fused[b, 0, j], step.top_k, step.own_first, J)
+            for h in (0, 13):
+                assert np.array_equal(idx_h[b, h, j, :len(want)], want), (b, h, j)
+
+
 def test_route_rejects_bad_arguments():
     step = hx.build_step(synth.CONFIGS[1], DEV)
     with pytest.raises(bsa.BsaError) as e:     # max_sel too small
