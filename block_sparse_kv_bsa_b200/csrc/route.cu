@@ -552,6 +552,49 @@ __device__ __forceinline__ uint32_t warp_kth_key(const uint32_t (&v)[NV], int m,
 // index order).
 constexpr int kTopkCandCap = 512;
 
+// Top K of the n_cand candidate keys ckey[] (blocks cidx[], in ascending
+// block order, all >= lo), by one warp holding NV per lane: the K-th
+// largest key as in warp_kth_key, then every larger key and the first
+// K - #{larger} keys equal to it, written to out[] in block order.
+template <int NV>
+__device__ __forceinline__ void warp_select_candidates(const uint32_t* ckey, const uint16_t* cidx,
+                                                       int n_cand, int K, uint32_t lo,
+                                                       int32_t* out) {
+  const int lane = threadIdx.x & 31;
+  const unsigned below = (1u << lane) - 1u;
+  uint32_t v[NV];
+  uint32_t hi = 0u;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    v[i] = i * 32 + lane < n_cand ? ckey[i * 32 + lane] : 0u;
+    hi = max(hi, v[i]);
+  }
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  bool ex;
+  const uint32_t th = warp_kth_key(v, K, lo, hi, &ex);
+  int need_eq = 0;
+  if (!ex) {
+    int gt = 0;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) gt += v[i] > th;
+    need_eq = K - static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(gt)));
+  }
+  int at = 0, eq_before = 0;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    if (i * 32 >= n_cand) break;
+    const bool valid = i * 32 + lane < n_cand;
+    const bool is_eq = valid && v[i] == th;
+    const unsigned em = __ballot_sync(0xffffffffu, is_eq);
+    const int r_eq = eq_before + __popc(em & below);
+    const bool sel = valid && (ex ? v[i] >= th : (v[i] > th || (is_eq && r_eq < need_eq)));
+    const unsigned sm = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[at + __popc(sm & below)] = cidx[i * 32 + lane];
+    at += __popc(sm);
+    eq_before += __popc(em);
+  }
+}
+
 // Top-K of a row of at most 128 * KPL history blocks: one CTA of 128
 // threads per row, thread t holding the keys of blocks c * 128 + t (c < KPL)
 // in registers.
@@ -586,6 +629,8 @@ __global__ void __launch_bounds__(kTopkRowThreads, KPL <= 18 ? 8 : 6) topk_row_k
   __shared__ uint32_t samp[32 * kSamp];
   __shared__ uint32_t ckey[kTopkCandCap];
   __shared__ uint16_t cidx[kTopkCandCap];
+  __shared__ uint32_t cmask[KPL * kWarps];        // candidate flags, word = 32 blocks
+  __shared__ uint32_t kbuf[KPL * kTopkRowThreads];  // candidate keys by block
   __shared__ uint32_t s_pivot;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -669,65 +714,51 @@ __global__ void __launch_bounds__(kTopkRowThreads, KPL <= 18 ? 8 : 6) topk_row_k
       const int n_cand = block_count(piv, false, parity);
       parity ^= 1;
       if (n_cand >= K && n_cand <= kTopkCandCap) {
-        // Candidates in block order: group c, then thread.
-#pragma unroll
-        for (int c = 0; c < KPL; ++c) {
-          const unsigned m = __ballot_sync(0xffffffffu, key[c] >= piv);
-          if (lane == 0) grp[0][c][warp] = __popc(m);
-        }
-        __syncthreads();
-        int pos = 0;
+        // Candidates in block order through a bitmask: word c * 4 + warp
+        // holds the flags of blocks (c * 4 + warp) * 32 + lane, so words
+        // ascend with the block; each candidate's key goes to kbuf[block].
 #pragma unroll
         for (int c = 0; c < KPL; ++c) {
           const bool cand = key[c] >= piv;
-          int at = pos + __popc(__ballot_sync(0xffffffffu, cand) & below);
-#pragma unroll
-          for (int w = 0; w < kWarps; ++w) {
-            const int e = static_cast<int>(grp[0][c][w]);
-            at += w < warp ? e : 0;
-            pos += e;
-          }
-          if (cand) {
-            ckey[at] = key[c];
-            cidx[at] = static_cast<uint16_t>(c * kTopkRowThreads + t);
-          }
+          const unsigned m = __ballot_sync(0xffffffffu, cand);
+          if (lane == 0) cmask[c * kWarps + warp] = m;
+          if (cand) kbuf[c * kTopkRowThreads + t] = key[c];
         }
         __syncthreads();
         if (warp == 0) {
-          constexpr int kC = kTopkCandCap / 32;
-          uint32_t v[kC];
-          uint32_t hi = 0u;
+          // Lane l takes words l, l + 32, ...: one warp scan of the word
+          // counts per round places each word's blocks after the earlier
+          // words' ones.
+          constexpr int kWords = KPL * kWarps;
+          int at = 0;
+#pragma unroll 1
+          for (int w0 = 0; w0 < kWords; w0 += 32) {
+            const int w = w0 + lane;
+            unsigned m = w < kWords ? cmask[w] : 0u;
+            const int cnt = __popc(m);
+            int incl = cnt;
 #pragma unroll
-          for (int i = 0; i < kC; ++i) {
-            v[i] = i * 32 + lane < n_cand ? ckey[i * 32 + lane] : 0u;
-            hi = max(hi, v[i]);
+            for (int off = 1; off < 32; off <<= 1) {
+              const int x = __shfl_up_sync(0xffffffffu, incl, off);
+              if (lane >= off) incl += x;
+            }
+            int p = at + incl - cnt;
+            while (m != 0u) {
+              const int n = w * 32 + __ffs(m) - 1;
+              m &= m - 1u;
+              ckey[p] = kbuf[n];
+              cidx[p] = static_cast<uint16_t>(n);
+              ++p;
+            }
+            at += __shfl_sync(0xffffffffu, incl, 31);
           }
-          hi = __reduce_max_sync(0xffffffffu, hi);
-          bool ex;
-          const uint32_t th = warp_kth_key(v, K, piv, hi, &ex);
-          int need_eq = 0;
-          if (!ex) {
-            int gt = 0;
-#pragma unroll
-            for (int i = 0; i < kC; ++i) gt += v[i] > th;
-            need_eq = K - static_cast<int>(__reduce_add_sync(0xffffffffu,
-                                                             static_cast<unsigned>(gt)));
-          }
-          int at = 0, eq_before = 0;
-#pragma unroll
-          for (int i = 0; i < kC; ++i) {
-            if (i * 32 >= n_cand) break;
-            const bool valid = i * 32 + lane < n_cand;
-            const bool is_eq = valid && v[i] == th;
-            const unsigned em = __ballot_sync(0xffffffffu, is_eq);
-            const int r_eq = eq_before + __popc(em & below);
-            const bool sel =
-                valid && (ex ? v[i] >= th : (v[i] > th || (is_eq && r_eq < need_eq)));
-            const unsigned sm = __ballot_sync(0xffffffffu, sel);
-            if (sel) out[at + __popc(sm & below)] = cidx[i * 32 + lane];
-            at += __popc(sm);
-            eq_before += __popc(em);
-          }
+          __syncwarp();
+          if (n_cand <= 128)
+            warp_select_candidates<4>(ckey, cidx, n_cand, K, piv, out);
+          else if (n_cand <= 256)
+            warp_select_candidates<8>(ckey, cidx, n_cand, K, piv, out);
+          else
+            warp_select_candidates<16>(ckey, cidx, n_cand, K, piv, out);
         }
         done = true;
       }
