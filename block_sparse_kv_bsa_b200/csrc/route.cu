@@ -316,6 +316,10 @@ __device__ __forceinline__ uint32_t score_key(float x) {
   uint32_t u = __float_as_uint(x);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+// Its inverse: the float a key came from, bit for bit.
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
 // Block-wide exclusive prefix of a per-thread flag (threads in index order).
 // Returns this thread's exclusive count; *total gets the block total.
@@ -946,20 +950,23 @@ __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a,
       select_run(thr, need_eq, [&](int n) { flag[n] = 1; });
     }
   } else {
+    // The scores are read from global memory once, here; later passes take
+    // them back from the keys (key_score inverts score_key exactly).
+    float mx = -INFINITY;
     for (int n = t; n < nh; n += kTopkThreads) {
-      keys[n] = score_key(sr[n]);
+      const float f = sr[n];
+      keys[n] = score_key(f);
       flag[n] = 0;
+      mx = fmaxf(mx, f);
     }
     const int K = min(v.k_unc, nh);
     if (K > 0) {
       // Row maximum and normaliser of softmax(s), in a fixed order.
-      float mx = -INFINITY;
-      for (int n = t; n < nh; n += kTopkThreads) mx = fmaxf(mx, sr[n]);
       red[t] = mx;
       __syncthreads();
       const float smax = block_tree(red, [](float x, float y) { return fmaxf(x, y); });
       float z = 0.f;
-      for (int n = t; n < nh; n += kTopkThreads) z += expf(sr[n] - smax);
+      for (int n = t; n < nh; n += kTopkThreads) z += expf(key_score(keys[n]) - smax);
       red[t] = z;
       __syncthreads();
       const float zsum = block_tree(red, [](float x, float y) { return x + y; });
@@ -973,12 +980,19 @@ __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a,
       // rounding) being the exact total; so when this sum is below the mass
       // cut by more than 1.2e-7 (K + 1), the walk below, whose running sum
       // only grows, stays below the cut to the end and takes all K: their
-      // order is not needed.
+      // order is not needed.  The K terms are those of the keys above thr
+      // plus need_eq copies of the term of thr (equal keys, equal scores),
+      // added last.
       float mass_local = 0.f;
-      select_run(thr, need_eq, [&](int n) { mass_local += expf(sr[n] - smax) / zsum; });
+      for (int n = r0; n < r1; ++n)
+        if (keys[n] > thr) mass_local += expf(key_score(keys[n]) - smax) / zsum;
       red[t] = mass_local;
       __syncthreads();
-      const float mass_k = block_tree(red, [](float x, float y) { return x + y; });
+      float mass_k = block_tree(red, [](float x, float y) { return x + y; });
+      if (need_eq > 0) {
+        const float e_thr = expf(key_score(thr) - smax) / zsum;
+        for (int i = 0; i < need_eq; ++i) mass_k += e_thr;
+      }
       if (mass_k < v.mass - 1.2e-7f * static_cast<float>(K + 1)) {
         select_run(thr, need_eq, [&](int n) { flag[n] = 1; });
       } else {
@@ -1001,7 +1015,7 @@ __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a,
             for (int i = 0; i < K; ++i) rank += sortbuf[i] < x;
             const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~x));
             nidx[rank] = n;
-            pr[rank] = expf(sr[n] - smax) / zsum;
+            pr[rank] = expf(key_score(keys[n]) - smax) / zsum;
           }
           __syncthreads();
           if (t == 0) {
@@ -1044,7 +1058,7 @@ __global__ void __launch_bounds__(kTopkThreads) velox_select_kernel(RouteArgs a,
             int m = K;
             for (int r = 0; r < K; ++r) {
               const int n = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(~sortbuf[r]));
-              acc += expf(sr[n] - smax) / zsum;
+              acc += expf(key_score(keys[n]) - smax) / zsum;
               if (acc >= v.mass) {
                 m = r + 1;
                 break;
