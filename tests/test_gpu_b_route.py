@@ -161,6 +161,18 @@ def test_route_from_pooled_keys(key, chunk):
     assert torch.equal(idx, ib) and torch.equal(cnt, cb)
 
 
+@pytest.mark.parametrize("grid", [(8, 32, 32), (5, 26, 64)])
+def test_route_from_pooled_keys_at_the_tensor_core_product_limit(grid):
+    # 64 query blocks (8 x 32 x 32): the most the tensor-core product holds,
+    # every row of its query-mean operand in use; 65 (5 x 26 x 64): the first
+    # count scored on the FMA pipes instead.  211 history blocks: one full
+    # 128-block tile and a ragged one.
+    w = dataclasses.replace(synth.CONFIGS[3], grid=grid, Hh=4, hist_direct=211)
+    b = hx.build_step(w, DEV, pooled_keys=True)
+    assert b.n_own == (64 if grid == (8, 32, 32) else 65)
+    _check(b)
+
+
 def test_route_from_pooled_keys_many_query_blocks():
     # 98 query blocks (an 8 x 30 x 52 chunk): more than the pipelined pooled
     # product takes (64), so the one-shot kernel scores them.
