@@ -677,18 +677,20 @@ class State:
 
     def velox_point(self, reps: int = 10) -> dict:
         """The page's own route at this chunk (Velox constants; synthetic
-        coverage and prior), timed, and bsa_attn timed on those routes."""
+        coverage and prior), timed, and bsa_attn timed on those routes.  The
+        route takes the query means of the step's Q reordering, as the step's
+        own route does (bsa_route_velox_qmean)."""
         w, bsa = self.w, self.bsa
         cov = torch.from_numpy(synth.coverage(w, CHUNK, self.n_own)).to(self.device)
         kw = dict(g=self.g, coverage=cov, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale,
                   tau=0.1, eta_cov=0.9, k_cov=80, k_unc=150, mass=0.9,
                   prev_first=self.own_first - self.n_own, n_prev=self.n_own, window_half=13,
-                  q_valid=self.q_valid, workspace=self.ws)
-        idx, cnt = bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist, self.own_first,
+                  q_mean=self.q_mean, workspace=self.ws)
+        idx, cnt = bsa.bsa_route_velox(None, self.cache, self.n_hist, self.own_first,
                                        self.n_own, **kw)
         o = torch.empty_like(self.q_blk)
         lse = torch.empty(self.q_blk.shape[:3], dtype=torch.float32, device=self.device)
-        rt = _time_call(lambda: bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist,
+        rt = _time_call(lambda: bsa.bsa_route_velox(None, self.cache, self.n_hist,
                                                     self.own_first, self.n_own, idx=idx,
                                                     cnt=cnt, **kw), reps)
         at = _time_call(lambda: bsa.bsa_attn(self.q_blk, self.cache, idx, cnt,
@@ -703,6 +705,7 @@ class State:
                                            "min": int(c.min().item()),
                                            "max": int(c.max().item())},
                 "covered_query_blocks": int((cov >= 0.9).sum().item()),
+                "query_means": "from the step's Q reordering (bsa_route_velox_qmean)",
                 "constants": "tau 0.1, g_ref 0.2, lambda 2, eta_cov 0.9, K_cov 80, "
                              "K_unc 150, mass 0.9, window +/-13 in the previous chunk"}
 
@@ -729,12 +732,12 @@ class State:
         kw = dict(g=g, coverage=cov, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale, tau=0.1,
                   eta_cov=0.9, k_cov=80, k_unc=150, mass=0.9,
                   prev_first=self.own_first - self.n_own, n_prev=self.n_own, window_half=13,
-                  q_valid=self.q_valid, workspace=self.ws)
-        idx, cnt = bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist, self.own_first,
+                  q_mean=self.q_mean, workspace=self.ws)
+        idx, cnt = bsa.bsa_route_velox(None, self.cache, self.n_hist, self.own_first,
                                        self.n_own, **kw)
         o = torch.empty_like(self.q_blk)
         lse = torch.empty(self.q_blk.shape[:3], dtype=torch.float32, device=self.device)
-        rt = _time_call(lambda: bsa.bsa_route_velox(self.q_blk, self.cache, self.n_hist,
+        rt = _time_call(lambda: bsa.bsa_route_velox(None, self.cache, self.n_hist,
                                                     self.own_first, self.n_own, idx=idx,
                                                     cnt=cnt, **kw), 10)
         at = _time_call(lambda: bsa.bsa_attn(self.q_blk, self.cache, idx, cnt,

@@ -49,6 +49,7 @@ EXPORTS = ("bsa_abi_version", "bsa_status_string", "bsa_gilbert_perm", "bsa_kv_a
            "bsa_kv_pool_means",
            "bsa_tokens_to_blocks", "bsa_tokens_to_blocks_mean", "bsa_blocks_to_tokens",
            "bsa_route_workspace_size", "bsa_route", "bsa_route_qmean", "bsa_route_velox",
+           "bsa_route_velox_qmean",
            "bsa_route_noalloc", "bsa_attn", "bsa_attn_tokens",
            "bsa_geometry_prior",
            "bsa_check_device_error",
@@ -109,6 +110,8 @@ _sig = {
                                 _p, _i, _p, _p, _p, _p]),
     "bsa_route_velox": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f,
                              ctypes.POINTER(CVeloxRoute), _p, _p, _i, _p, _sz, _p, _p]),
+    "bsa_route_velox_qmean": (_i, [_p, ctypes.POINTER(CCache), _i, _i, _i, _p, _f, _f, _f,
+                                   ctypes.POINTER(CVeloxRoute), _p, _p, _i, _p, _sz, _p, _p]),
     "bsa_route_noalloc": (_i, [_p, ctypes.POINTER(CCache), _p, _i, _i, _i, _p, _f, _f, _f, _i,
                                _p, _p, _i, _p, _p]),
     "bsa_attn": (_i, [_p, ctypes.POINTER(CCache), _p, _p, _p, _i, _i, _f, _p, _p, _p, _p]),
@@ -432,7 +435,7 @@ def velox_max_sel(n_hist: int, n_own: int, k_cov: int = 80, k_unc: int = 150, n_
     return min(n_hist, budget + 2 * window_half + 1 + n_ref) + n_own
 
 
-def bsa_route_velox(q_blk: torch.Tensor, cache: KVCache, n_hist: int, own_first: int,
+def bsa_route_velox(q_blk: Optional[torch.Tensor], cache: KVCache, n_hist: int, own_first: int,
                     n_own: int, g: Optional[torch.Tensor] = None,
                     coverage: Optional[torch.Tensor] = None, lam: float = 2.0,
                     g_ref: float = 0.2, sm_scale: Optional[float] = None, tau: float = 0.1,
@@ -441,10 +444,17 @@ def bsa_route_velox(q_blk: torch.Tensor, cache: KVCache, n_hist: int, own_first:
                     ref_first: int = 0, n_ref: int = 0, q_valid: Optional[torch.Tensor] = None,
                     max_sel: Optional[int] = None, idx: Optional[torch.Tensor] = None,
                     cnt: Optional[torch.Tensor] = None,
-                    workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """The page's full route; returns (idx [B,Hh,n_own,max_sel] padded with -1, cnt)."""
+                    workspace: Optional[torch.Tensor] = None,
+                    q_mean: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The page's full route; returns (idx [B,Hh,n_own,max_sel] padded with -1, cnt).
+    With ``q_mean`` ([B, Hh, n_own, D] fp32, e.g. from
+    bsa_tokens_to_blocks_mean) the query means are taken from it
+    (bsa_route_velox_qmean) and ``q_blk`` may be None."""
     dev = cache.device
-    _need(q_blk, "q_blk", torch.bfloat16, dev, (cache.B, cache.Hh, n_own * BLK, cache.D))
+    if q_mean is not None:
+        _need(q_mean, "q_mean", torch.float32, dev, (cache.B, cache.Hh, n_own, cache.D))
+    else:
+        _need(q_blk, "q_blk", torch.bfloat16, dev, (cache.B, cache.Hh, n_own * BLK, cache.D))
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(cache.D)
     if max_sel is None:
@@ -468,6 +478,13 @@ def bsa_route_velox(q_blk: torch.Tensor, cache: KVCache, n_hist: int, own_first:
                        float(tau), int(k_cov), int(k_unc), float(mass), int(prev_first),
                        int(n_prev), int(window_half), int(ref_first), int(n_ref))
     cs = cache.c_struct()
+    if q_mean is not None:
+        _check("bsa_route_velox_qmean", _lib.bsa_route_velox_qmean(
+            _ptr(q_mean), ctypes.byref(cs), int(n_hist), int(own_first), int(n_own), _ptr(g),
+            float(lam), float(g_ref), float(sm_scale), ctypes.byref(opts), _ptr(idx), _ptr(cnt),
+            int(max_sel), _ptr(workspace), workspace.numel(), _ptr(error_word(dev)),
+            _stream(dev)))
+        return idx, cnt
     _check("bsa_route_velox", _lib.bsa_route_velox(
         _ptr(q_blk), ctypes.byref(cs), _ptr(q_valid), int(n_hist), int(own_first), int(n_own),
         _ptr(g), float(lam), float(g_ref), float(sm_scale), ctypes.byref(opts), _ptr(idx),

@@ -1306,12 +1306,14 @@ extern "C" bsa_status bsa_route_qmean(const float* q_mean, const bsa_kv_cache* c
                     sm_scale, top_k, idx, cnt, max_sel, workspace, ws_bytes, d_err, stream);
 }
 
-extern "C" bsa_status bsa_route_velox(const void* q_blk, const bsa_kv_cache* c,
-                                      const int32_t* q_valid, int n_hist, int own_first,
-                                      int n_own, const float* g, float lambda, float g_ref,
-                                      float sm_scale, const bsa_velox_route* opts, int32_t* idx,
-                                      int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
-                                      int32_t* d_err, void* stream) {
+// bsa_route_velox and bsa_route_velox_qmean: the scores (query means from
+// q_blk or given), then the page's selection.
+static bsa_status route_velox(const void* q_blk, const float* q_mean, const bsa_kv_cache* c,
+                              const int32_t* q_valid, int n_hist, int own_first, int n_own,
+                              const float* g, float lambda, float g_ref, float sm_scale,
+                              const bsa_velox_route* opts, int32_t* idx, int32_t* cnt,
+                              int max_sel, void* workspace, size_t ws_bytes, int32_t* d_err,
+                              void* stream) {
   if (opts == nullptr) return BSA_ERR_INVALID_ARG;
   const bsa_velox_route& o = *opts;
   if (o.k_cov < 0 || o.k_unc < 0 || o.n_prev < 0 || o.window_half < 0 || o.n_ref < 0 ||
@@ -1328,7 +1330,7 @@ extern "C" bsa_status bsa_route_velox(const void* q_blk, const bsa_kv_cache* c,
   if (max_sel < bound) return BSA_ERR_CAPACITY;
   cudaStream_t s = as_stream(stream);
   RouteArgs a;
-  bsa_status st = route_scores(q_blk, nullptr, c, q_valid, n_hist, own_first, n_own, g, lambda,
+  bsa_status st = route_scores(q_blk, q_mean, c, q_valid, n_hist, own_first, n_own, g, lambda,
                                g_ref, sm_scale, idx, cnt, max_sel, workspace, ws_bytes, d_err, s,
                                &a);
   if (st != BSA_OK) return st;
@@ -1342,6 +1344,28 @@ extern "C" bsa_status bsa_route_velox(const void* q_blk, const bsa_kv_cache* c,
   dim3 qgrid(n_own, c->Hh, c->B);
   BSA_TRY(launch_pdl(velox_select_kernel, qgrid, dim3(kTopkThreads), smem, s, a, v));
   return launch_status();
+}
+
+extern "C" bsa_status bsa_route_velox(const void* q_blk, const bsa_kv_cache* c,
+                                      const int32_t* q_valid, int n_hist, int own_first,
+                                      int n_own, const float* g, float lambda, float g_ref,
+                                      float sm_scale, const bsa_velox_route* opts, int32_t* idx,
+                                      int32_t* cnt, int max_sel, void* workspace, size_t ws_bytes,
+                                      int32_t* d_err, void* stream) {
+  if (q_blk == nullptr) return BSA_ERR_INVALID_ARG;
+  return route_velox(q_blk, nullptr, c, q_valid, n_hist, own_first, n_own, g, lambda, g_ref,
+                     sm_scale, opts, idx, cnt, max_sel, workspace, ws_bytes, d_err, stream);
+}
+
+extern "C" bsa_status bsa_route_velox_qmean(const float* q_mean, const bsa_kv_cache* c,
+                                            int n_hist, int own_first, int n_own, const float* g,
+                                            float lambda, float g_ref, float sm_scale,
+                                            const bsa_velox_route* opts, int32_t* idx,
+                                            int32_t* cnt, int max_sel, void* workspace,
+                                            size_t ws_bytes, int32_t* d_err, void* stream) {
+  if (q_mean == nullptr) return BSA_ERR_INVALID_ARG;
+  return route_velox(nullptr, q_mean, c, nullptr, n_hist, own_first, n_own, g, lambda, g_ref,
+                     sm_scale, opts, idx, cnt, max_sel, workspace, ws_bytes, d_err, stream);
 }
 
 // ---------------------------------------------------------------------------

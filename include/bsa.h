@@ -336,6 +336,20 @@ bsa_status bsa_route_velox(const void *q_blk, const bsa_kv_cache *cache, const i
                            void *workspace, size_t ws_bytes, int32_t *d_err, void *stream);
 
 /*
+ * bsa_route_velox with the query-block means given instead of the query
+ * blocks (Velox, Methodology Steps 4-5), e.g. from bsa_tokens_to_blocks_mean:
+ *   q_mean  device fp32 [B, Hh, n_own, D], 16-byte aligned
+ * Everything else, the result and the errors are those of bsa_route_velox.
+ * With the means of bsa_tokens_to_blocks_mean the routes equal
+ * bsa_route_velox's bit for bit.
+ */
+bsa_status bsa_route_velox_qmean(const float *q_mean, const bsa_kv_cache *cache, int n_hist,
+                                 int own_first, int n_own, const float *g, float lambda,
+                                 float g_ref, float sm_scale, const bsa_velox_route *opts,
+                                 int32_t *idx, int32_t *cnt, int max_sel, void *workspace,
+                                 size_t ws_bytes, int32_t *d_err, void *stream);
+
+/*
  * Geometric overlap prior g and coverage from slabs (Velox, Methodology
  * Step 3; slabs as in Step 1).  Each slab (a source-camera token rectangle
  * [u0, u1] x [v0, v1] in pixel-edge coordinates plus a depth interval

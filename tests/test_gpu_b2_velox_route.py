@@ -133,3 +133,23 @@ def test_velox_route_rejects_small_max_sel():
         bsa.bsa_route_velox(step.q_blk, step.cache, step.n_hist, step.own_first, step.n_own,
                             max_sel=10)
     assert e.value.status == 3
+
+
+@pytest.mark.parametrize("chunk", [12, 48])
+def test_velox_route_from_query_means_equals_from_query_blocks(chunk):
+    # bsa_route_velox_qmean on the means of bsa_tokens_to_blocks_mean gives
+    # bsa_route_velox's routes (query blocks pooled by the route) bit for bit.
+    w = synth.CONFIGS[4]
+    T, H, W = w.grid
+    step = hx.build_step(w, DEV, chunk=chunk, pooled_keys=True)
+    nbc = step.n_own
+    cov = torch.from_numpy(_coverage(w, nbc, seed=chunk)).to(DEV)
+    kw = dict(g=step.g, coverage=cov, lam=w.lam, g_ref=w.g_ref, sm_scale=w.sm_scale,
+              prev_first=step.own_first - nbc, n_prev=nbc, ref_first=0, n_ref=4, **P)
+    i1, c1 = bsa.bsa_route_velox(step.q_blk, step.cache, step.n_hist, step.own_first, nbc,
+                                 q_valid=step.q_valid, **kw)
+    _, qm = bsa.bsa_tokens_to_blocks_mean(step.q_tok, T, H, W)
+    i2, c2 = bsa.bsa_route_velox(None, step.cache, step.n_hist, step.own_first, nbc, q_mean=qm,
+                                 **kw)
+    bsa.raise_on_device_error(DEV)
+    assert torch.equal(i1, i2) and torch.equal(c1, c2)
